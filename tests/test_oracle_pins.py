@@ -1,0 +1,427 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU needed).
+
+Each test checks one oracle function against something it does not compute
+itself: a constant or worked shape the pages state (tests/golden), the e4m3fn
+and bf16 format definitions as implemented by torch's own casts (library
+routines), exact rational or integer arithmetic, closed forms and invariants.
+The cases are chosen so that a plausible slip (a dropped scale, a transposed
+operand, a swapped scale index, a wrong constant, a floor instead of a ceiling
+division) fails at least one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
+FACTS = json.load(open(GOLDEN))
+E4M3_MAX = FACTS["e4m3_max"]["value"]
+CLAMP = FACTS["amax_clamp_min"]["value"]
+BLOCK = FACTS["block_size"]["value"]
+
+
+def f32(v):
+    return np.float32(v)
+
+
+def torch_e4m3_bytes(a):
+    """torch's own fp32 -> float8_e4m3fn cast, as raw bytes."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+# --------------------------------------------------------------------------
+# e4m3fn codec
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_table_matches_torch_dtype():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = oracle.e4m3_table()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok])
+    # signed zeros
+    assert np.array_equal(np.signbit(ours[ok]), np.signbit(ref[ok]))
+
+
+def test_e4m3_decode_format_facts():
+    assert FACTS["e4m3_bits"]["exponent_bits"] == 4 and FACTS["e4m3_bits"]["mantissa_bits"] == 3
+    assert oracle.e4m3_decode(0x7E) == E4M3_MAX          # largest finite value, 448
+    assert oracle.e4m3_decode(0xFE) == -E4M3_MAX
+    assert math.isnan(oracle.e4m3_decode(0x7F)) and math.isnan(oracle.e4m3_decode(0xFF))
+    assert oracle.e4m3_decode(0x08) == 2.0 ** -6          # smallest normal
+    assert oracle.e4m3_decode(0x01) == 2.0 ** -9          # smallest subnormal
+    assert oracle.e4m3_decode(0x07) == 7 * 2.0 ** -9      # largest subnormal
+    assert oracle.e4m3_decode(0x38) == 1.0                # exponent bias 7
+    v = oracle.e4m3_decode(0x80)
+    assert v == 0.0 and math.copysign(1.0, v) < 0
+    finite = [oracle.e4m3_decode(c) for c in range(256) if c & 0x7F != 0x7F]
+    assert max(finite) == E4M3_MAX and min(finite) == -E4M3_MAX
+    assert len(finite) == 254
+
+
+def test_e4m3_encode_roundtrips_every_finite_code():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        assert oracle.e4m3_encode(oracle.e4m3_decode(c)) == c, hex(c)
+
+
+def _rounding_sweep():
+    """fp32 patterns around every e4m3 rounding decision point in |f| < 512:
+    for each fp32 exponent field and each value of the top 3 mantissa bits,
+    the low 20 bits take values at, next to and around the halfway pattern."""
+    lows = [0, 1, 2, 3, 0x7FFFD, 0x7FFFE, 0x7FFFF, 0x80000, 0x80001, 0x80002,
+            0xFFFFD, 0xFFFFE, 0xFFFFF]
+    rng = np.random.default_rng(1)
+    lows += list(rng.integers(0, 1 << 20, 40))
+    pats = []
+    for exp_field in range(0, 0x88):
+        for top in range(8):
+            for low in lows:
+                pats.append((exp_field << 23) | (top << 20) | int(low))
+    pats = np.array(pats, dtype=np.uint32)
+    pats = np.concatenate([pats, pats | np.uint32(0x80000000)])
+    return pats.view(np.float32)
+
+
+def test_e4m3_encode_matches_torch_cast_at_rounding_points():
+    f = _rounding_sweep()
+    f = f[np.abs(f) <= 464.0]     # torch maps anything that rounds past 448 to NaN
+    assert np.array_equal(oracle.e4m3_encode_array(f), torch_e4m3_bytes(f))
+
+
+def test_e4m3_encode_matches_torch_cast_random():
+    rng = np.random.default_rng(2)
+    mag = np.exp2(rng.uniform(-16, np.log2(464.0), 2_000_000)).astype(np.float32)
+    sign = np.where(rng.random(mag.size) < 0.5, -1, 1).astype(np.float32)
+    f = mag * sign
+    f = f[np.abs(f) <= 464.0]
+    assert np.array_equal(oracle.e4m3_encode_array(f), torch_e4m3_bytes(f))
+
+
+def test_e4m3_encode_ties_to_even_and_saturates():
+    # 464 is halfway between 448 (mantissa 110, even) and 480 (not representable)
+    assert oracle.e4m3_encode(464.0) == 0x7E
+    for v in (464.0001, 479.0, 480.0, 1e6, float("inf")):
+        assert oracle.e4m3_encode(v) == 0x7E
+        assert oracle.e4m3_encode(-v) == 0xFE
+    assert oracle.e4m3_encode(float("nan")) & 0x7F == 0x7F
+    # halfway between 1.0 (even) and 1.125 goes to 1.0; between 1.125 and 1.25 to 1.25
+    assert oracle.e4m3_encode(1.0625) == 0x38
+    assert oracle.e4m3_encode(1.1875) == 0x3A
+    # below half the smallest subnormal -> zero, exactly half -> zero (even), above -> 2^-9
+    assert oracle.e4m3_encode(2.0 ** -10) == 0x00
+    assert oracle.e4m3_encode(float(np.nextafter(f32(2.0 ** -10), f32(1)))) == 0x01
+    assert oracle.e4m3_encode(-0.0) == 0x80
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding
+# --------------------------------------------------------------------------
+
+def test_bf16_rne_matches_torch_cast():
+    rng = np.random.default_rng(3)
+    bits = rng.integers(0, 1 << 32, 400_000, dtype=np.uint64).astype(np.uint32)
+    low = np.array([0x7FFF, 0x8000, 0x8001, 0x0000, 0xFFFF], dtype=np.uint32)
+    edge = (bits[:5000, None] & np.uint32(0xFFFF0000)) | low[None, :]
+    bits = np.concatenate([bits, edge.ravel()])
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    ours = np.array([oracle.bf16_from_f32(v) for v in f[:100_000]], dtype=np.uint16)
+    ref = torch.from_numpy(f[:100_000].copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------
+# Scale rule
+# --------------------------------------------------------------------------
+
+def _exact_pow2_ceil(s):
+    """2^ceil(log2 s) by exact rational comparison (independent of frexp)."""
+    r = Fraction(float(s))
+    e = 0
+    while Fraction(2) ** e < r:
+        e += 1
+    while Fraction(2) ** (e - 1) >= r:
+        e -= 1
+    return float(Fraction(2) ** e)
+
+
+def test_ue8m0_round_up_is_exact_power_of_two_ceiling():
+    rng = np.random.default_rng(4)
+    vals = np.exp2(rng.uniform(-30, 30, 3000)).astype(np.float32)
+    vals = np.concatenate([vals, np.float32([1.0, 0.5, 2.0 ** -22, 1.5, 0.75,
+                                             np.nextafter(f32(1), f32(2)),
+                                             np.nextafter(f32(1), f32(0))])])
+    for v in vals:
+        assert oracle.ue8m0_round_up(v) == _exact_pow2_ceil(v), v
+
+
+def test_block_scale_pages_constants():
+    # amax equal to the e4m3 maximum gives a unit scale
+    assert oracle.block_scale(E4M3_MAX, False) == 1.0
+    assert oracle.block_scale(E4M3_MAX, True) == 1.0
+    # all-zero block: clamp to 1e-4 (fp32), then divide by 448 in fp32
+    zero_s = f32(CLAMP) / f32(E4M3_MAX)
+    assert oracle.block_scale(0.0, False) == zero_s
+    assert oracle.block_scale(5e-5, False) == zero_s
+    assert oracle.block_scale(0.0, True) == 2.0 ** -22   # 2.23e-7 lies in (2^-23, 2^-22]
+    # above the clamp the scale is amax/448, one fp32 division
+    assert oracle.block_scale(1.0, False) == f32(1.0) / f32(448.0)
+    assert oracle.block_scale(449.0, True) == 2.0
+    assert oracle.block_scale(224.0, True) == 0.5
+
+
+# --------------------------------------------------------------------------
+# act_quant
+# --------------------------------------------------------------------------
+
+def _bf16(x):
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_act_quant_pages_example_shapes():
+    ex = FACTS["act_quant_example"]
+    x = torch.randn(*ex["x_shape"], generator=torch.Generator().manual_seed(0))
+    q, s = oracle.act_quant(x.numpy(), block=BLOCK)
+    assert list(q.shape) == ex["q_shape"] and list(s.shape) == ex["s_shape"]
+
+
+def test_act_quant_scales_are_per_1x128_block():
+    x = torch.zeros(2, 4 * BLOCK)
+    x[0, 5] = 1.0            # block 0 of row 0: amax 1
+    x[0, BLOCK + 7] = -448.0  # block 1: amax 448 -> s = 1
+    x[0, 2 * BLOCK] = 3.0    # block 2: amax 3
+    # block 3 all zero -> clamp
+    x[1, :] = 2.0
+    q, s = oracle.act_quant(_bf16(x))
+    zero_s = f32(CLAMP) / f32(E4M3_MAX)
+    assert s[0, 0] == f32(1.0) / f32(448.0)
+    assert s[0, 1] == 1.0
+    assert s[0, 2] == f32(3.0) / f32(448.0)
+    assert s[0, 3] == zero_s
+    assert np.all(s[1] == f32(2.0) / f32(448.0))
+    # the amax element of a block maps to +-448 (None format)
+    assert q[0, 5] == 0x7E and q[0, BLOCK + 7] == 0xFE and q[0, 2 * BLOCK] == 0x7E
+    assert np.all(q[1] == 0x7E)
+    # zeros stay zeros
+    assert np.all(q[0, 3 * BLOCK:] == 0)
+
+
+def test_act_quant_unit_scale_block_is_plain_cast():
+    # a block whose amax is exactly 448 has s = 1, so q is the plain cast of x
+    rng = np.random.default_rng(5)
+    x = rng.normal(0, 50, (8, BLOCK)).astype(np.float32)
+    x = np.clip(x, -447, 447)
+    x[:, 3] = 448.0
+    xb = _bf16(torch.from_numpy(x))
+    q, s = oracle.act_quant(xb)
+    assert np.all(s == 1.0)
+    xf = oracle.bf16_bits_to_f32(xb)
+    assert np.array_equal(q, torch_e4m3_bytes(xf).reshape(q.shape))
+
+
+def _dec(q):
+    t = oracle.e4m3_table()
+    return t[q]
+
+
+def test_act_quant_invariants_and_roundtrip_bound():
+    x = torch.randn(64, 8 * BLOCK, generator=torch.Generator().manual_seed(6))
+    x[3, 100] = 300.0
+    x[10, 129:140] = 1e-6
+    x[20, 256:384] = 0.0
+    for fmt in (None, "ue8m0"):
+        xb = _bf16(x)
+        q, s = oracle.act_quant(xb, scale_fmt=fmt)
+        xf = oracle.bf16_bits_to_f32(xb).astype(np.float64).reshape(64, 8, BLOCK)
+        d = _dec(q).reshape(64, 8, BLOCK)
+        assert np.all(np.abs(d) <= E4M3_MAX)
+        amax = np.abs(xf).max(axis=2)
+        s_none = np.maximum(amax, f32(CLAMP)).astype(np.float32) / np.float32(448.0)
+        if fmt is None:
+            assert np.array_equal(s, s_none)
+        else:
+            m, _ = np.frexp(s)
+            assert np.all(m == 0.5)                          # exact powers of two
+            assert np.all(s >= s_none) and np.all(s < 2 * s_none)
+        # |dec(q)*s - x| <= half an e4m3 step of x/s, times s (plus fp32 division rounding)
+        y = xf / s[..., None]
+        step = np.where(np.abs(y) < 2.0 ** -6, 2.0 ** -9,
+                        np.exp2(np.floor(np.log2(np.maximum(np.abs(y), 1e-300))) - 3))
+        err = np.abs(d * s[..., None] - xf)
+        assert np.all(err <= (0.5 * step + np.abs(y) * 2.0 ** -23) * s[..., None] * (1 + 1e-12))
+
+
+def test_act_quant_matches_library_division_and_cast():
+    """q = cast_e4m3(fl32(x / s)) with torch's fp32 division and torch's cast."""
+    x = torch.randn(32, 16 * BLOCK, generator=torch.Generator().manual_seed(7)) * 3
+    x[torch.rand(x.shape, generator=torch.Generator().manual_seed(8)) < 0.01] *= 50
+    for fmt in (None, "ue8m0"):
+        for as_bf16 in (True, False):
+            arr = _bf16(x) if as_bf16 else x.numpy()
+            q, s = oracle.act_quant(arr, scale_fmt=fmt)
+            xf = torch.from_numpy(oracle.bf16_bits_to_f32(arr) if as_bf16 else arr.copy())
+            st = torch.from_numpy(s).repeat_interleave(BLOCK, dim=1)
+            ref = (xf / st).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(q, ref)
+
+
+# --------------------------------------------------------------------------
+# Test-data weight quantizer
+# --------------------------------------------------------------------------
+
+def test_weight_quant_tiles_and_ragged_edges():
+    rng = np.random.default_rng(9)
+    w = rng.normal(0, 0.02, (300, 576)).astype(np.float32)
+    w[0, 0] = 448.0
+    w[200:300, 512:576] = 0.0
+    q, s = oracle.weight_quant(w)
+    assert s.shape == (3, 5)                     # ceil(300/128), ceil(576/128)
+    assert s[0, 0] == 1.0
+    assert s[2, 4] == f32(CLAMP) / f32(E4M3_MAX)  # the all-zero ragged corner
+    for bi in range(3):
+        for bj in range(5):
+            tile = w[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]
+            a = max(np.abs(tile).max(), f32(CLAMP))
+            assert s[bi, bj] == np.float32(a) / np.float32(448.0)
+            st = torch.from_numpy(tile.copy()) / float(s[bi, bj])
+            ref = st.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(q[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128], ref)
+
+
+# --------------------------------------------------------------------------
+# weight_dequant
+# --------------------------------------------------------------------------
+
+def test_weight_dequant_pages_example_shape():
+    ex = FACTS["weight_dequant_example"]
+    q = np.zeros(ex["w_shape"], dtype=np.uint8)
+    s = np.ones(ex["s_shape"], dtype=np.float32)
+    y = oracle.weight_dequant(q, s)
+    assert y.shape == tuple(ex["w_shape"])
+    with pytest.raises(ValueError):
+        oracle.weight_dequant(q, np.ones((7, 8), dtype=np.float32))
+
+
+@pytest.mark.parametrize("shape", [(256, 256), (200, 576), (129, 130)])
+def test_weight_dequant_matches_library_multiply_and_cast(shape):
+    M, N = shape
+    g = torch.Generator().manual_seed(10)
+    codes = torch.randint(0, 254, (M, N), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8)
+    rb, cb = -(-M // 128), -(-N // 128)
+    s = torch.rand(rb, cb, generator=g) * (1e-3 - 1e-5) + 1e-5
+    s[0, -1] = -3.5e-4      # any finite scale is accepted
+    y = oracle.weight_dequant(codes.numpy(), s.numpy())
+    y32 = oracle.weight_dequant(codes.numpy(), s.numpy(), out="f32")
+    # element (i, j) takes the scale at (i // 128) * cdiv(N, 128) + j // 128
+    st = s.repeat_interleave(128, 0)[:M].repeat_interleave(128, 1)[:, :N]
+    prod = codes.view(torch.float8_e4m3fn).to(torch.float32) * st
+    assert np.array_equal(y32, prod.numpy())
+    ref = prod.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(y, ref)
+
+
+# --------------------------------------------------------------------------
+# GEMM reference
+# --------------------------------------------------------------------------
+
+def _random_problem(M, N, K, seed, ue8m0=False):
+    g = torch.Generator().manual_seed(seed)
+    codes_a = torch.randint(0, 254, (M, K), generator=g)
+    codes_a = (codes_a + (codes_a >= 0x7F).long()).to(torch.uint8).numpy()
+    codes_w = torch.randint(0, 254, (N, K), generator=g)
+    codes_w = (codes_w + (codes_w >= 0x7F).long()).to(torch.uint8).numpy()
+    sa = (torch.rand(M, K // 128, generator=g) * 2 + 0.01).numpy().astype(np.float32)
+    sw = (torch.rand(-(-N // 128), K // 128, generator=g) * 0.01 + 1e-4).numpy().astype(np.float32)
+    if ue8m0:
+        sa = np.exp2(np.round(np.log2(sa))).astype(np.float32)
+        sw = np.exp2(np.round(np.log2(sw))).astype(np.float32)
+    return codes_a, sa, codes_w, sw
+
+
+def _exact_gemm(qa, sa, qw, sw):
+    """Exact y and bound with integer arithmetic: every e4m3 value times 2^9 is
+    an integer, so each 128-wide partial sum is an integer times 2^-18; the
+    scales are then applied as exact rationals."""
+    table = oracle.e4m3_table()
+    ia = np.rint(table[qa] * 512).astype(np.int64)
+    iw = np.rint(table[qw] * 512).astype(np.int64)
+    M, K = qa.shape
+    N = qw.shape[0]
+    y = [[Fraction(0)] * N for _ in range(M)]
+    b = [[Fraction(0)] * N for _ in range(M)]
+    for kb in range(K // 128):
+        sl = slice(kb * 128, (kb + 1) * 128)
+        P = ia[:, sl] @ iw[:, sl].T
+        Pabs = np.abs(ia[:, sl]) @ np.abs(iw[:, sl]).T
+        for m in range(M):
+            fa = Fraction(float(sa[m, kb]))
+            for n in range(N):
+                sc = fa * Fraction(float(sw[n // 128, kb])) / (1 << 18)
+                y[m][n] += sc * int(P[m, n])
+                b[m][n] += abs(sc) * int(Pabs[m, n])
+    return y, b
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 128, 128), (4, 256, 256), (2, 320, 384)])
+def test_gemm_matches_exact_integer_arithmetic(M, N, K):
+    qa, sa, qw, sw = _random_problem(M, N, K, seed=M * 1000 + N + K)
+    y, bnd = oracle.gemm(qa, sa, qw, sw)
+    ye, be = _exact_gemm(qa, sa, qw, sw)
+    for m in range(M):
+        for n in range(N):
+            tol = float(be[m][n]) * 2.0 ** -50
+            assert abs(Fraction(float(y[m, n])) - ye[m][n]) <= Fraction(tol), (m, n)
+            assert abs(bnd[m, n] - float(be[m][n])) <= tol
+
+
+def test_gemm_matches_library_matmul_tiny_config():
+    # the tiny linear: x [128,512] ~N(0,1) with 1% outliers x50, W [256,512] ~N(0,0.02)
+    from fp8_block_scaled_10_b200 import workloads as wl
+    x = wl.normal_with_outliers(128, 512, seed=0, frac=0.01, factor=50.0)
+    w = wl.weight_f32(256, 512, seed=1)
+    qa, sa = oracle.act_quant(wl.bf16_bits(x))
+    qw, sw = oracle.weight_quant(w.numpy())
+    assert sw.shape == (2, 4)
+    y, bnd = oracle.gemm(qa, sa, qw, sw)
+    table = torch.from_numpy(oracle.e4m3_table())
+    a_hat = table[torch.from_numpy(qa).long()] * torch.from_numpy(sa).double().repeat_interleave(128, 1)
+    w_hat = table[torch.from_numpy(qw).long()] * \
+        torch.from_numpy(sw).double().repeat_interleave(128, 0)[:256].repeat_interleave(128, 1)
+    ref = (a_hat @ w_hat.T).numpy()
+    ref_b = (a_hat.abs() @ w_hat.abs().T).numpy()
+    assert np.all(np.abs(y - ref) <= 1e-12 * ref_b)
+    assert np.allclose(bnd, ref_b, rtol=1e-12, atol=0)
+
+
+def test_gemm_special_cases():
+    # all-ones W with unit scales reduces y to the row sums of the dequantized A
+    qa, sa, _, _ = _random_problem(5, 128, 256, seed=11)
+    qw = np.full((128, 256), 0x38, dtype=np.uint8)     # e4m3 1.0
+    sw = np.ones((1, 2), dtype=np.float32)
+    y, _ = oracle.gemm(qa, sa, qw, sw)
+    a_hat = oracle.e4m3_table()[qa] * np.repeat(sa.astype(np.float64), 128, axis=1)
+    assert np.allclose(y, a_hat.sum(axis=1, keepdims=True).repeat(128, 1), rtol=1e-14, atol=1e-300)
+    # a single nonzero K block isolates its (sa * sw) pair
+    qa, sa, qw, sw = _random_problem(4, 256, 384, seed=12)
+    qa[:, :128] = 0
+    qa[:, 256:] = 0
+    y, _ = oracle.gemm(qa, sa, qw, sw)
+    t = oracle.e4m3_table()
+    for m in range(4):
+        for n in (0, 127, 128, 255):
+            p = float(np.dot(t[qa[m, 128:256]], t[qw[n, 128:256]]))
+            assert y[m, n] == float(sa[m, 1]) * float(sw[n // 128, 1]) * p
+    # sign: negating A negates y exactly
+    yn, _ = oracle.gemm(qa ^ np.uint8(0x80), sa, qw, sw)
+    assert np.array_equal(yn, -y)
