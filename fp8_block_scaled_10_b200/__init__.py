@@ -1,0 +1,253 @@
+"""FP8 block-scaled linear-layer kernels for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libfp8bs.so`` (``include/fp8bs.h``).
+It only marshals arguments: tensors are allocated with torch on the current
+CUDA device and every computation runs in the library's CUDA kernels on
+torch's current stream.  There is no CPU fallback; if the library is missing
+or cannot load, every call raises.
+
+Calls keep the names and defaults of the DeepSeek-V3 inference kernels that
+the pages describe:
+
+* ``act_quant(x, block_size=128, scale_fmt=None) -> (q, s)``
+* ``weight_dequant(x, s, block_size=128) -> y``
+* ``fp8_gemm(a, a_s, b, b_s) -> y``
+* ``fp8_linear(x, weight, weight_scale, scale_fmt=None) -> y``
+* ``fp8_gemm_grouped(a, a_s, w, w_s, m_offsets) -> y``
+* ``weight_quant(w, block_size=128, scale_fmt=None) -> (q, s)``
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "act_quant", "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
+    "fp8_gemm_grouped", "gemm_workspace_size", "device_error", "lib", "Fp8bsError",
+    "LIB_PATH", "HEADER_PATH",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8bs.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp8bs.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+DTYPE_BF16, DTYPE_F32 = 0, 1
+SCALE_FMT_NONE, SCALE_FMT_UE8M0 = 0, 1
+
+
+class Fp8bsError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("%s: %s" % (_STATUS_NAMES.get(status, status), message))
+        self.status = status
+
+
+_STATUS_NAMES = {OK: "FP8BS_OK", ERR_INVALID_ARG: "FP8BS_ERR_INVALID_ARG",
+                 ERR_UNSUPPORTED: "FP8BS_ERR_UNSUPPORTED", ERR_WORKSPACE: "FP8BS_ERR_WORKSPACE",
+                 ERR_CUDA: "FP8BS_ERR_CUDA", ERR_TIMEOUT: "FP8BS_ERR_TIMEOUT"}
+
+_lib = None
+
+
+def lib():
+    """The loaded ``libfp8bs.so`` (ctypes.CDLL) with argument types declared."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libfp8bs.so is not built (python -m fp8_block_scaled_10_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "fp8bs_version": (i32, []),
+        "fp8bs_status_string": (ctypes.c_char_p, [i32]),
+        "fp8bs_last_error_message": (ctypes.c_char_p, []),
+        "fp8bs_get_device_error": (i32, [p, ctypes.POINTER(i32)]),
+        "fp8bs_act_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
+        "fp8bs_weight_dequant": (i32, [p, p, i64, i64, i64, p, i32, p]),
+        "fp8bs_weight_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
+        "fp8bs_gemm_workspace_size": (sz, [i64, i64, i64]),
+        "fp8bs_fp8_gemm": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
+        "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
+        "fp8bs_fp8_gemm_grouped": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def header_symbols():
+    """Names of the entry points that include/fp8bs.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"FP8BS_API[^;(]*?\b(fp8bs_\w+)\s*\(", text)))
+
+
+def _check(status):
+    if status != OK:
+        msg = lib().fp8bs_last_error_message().decode(errors="replace")
+        raise Fp8bsError(status, msg)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("fp8bs runs on CUDA tensors only (got a %s tensor)" % t.device)
+        if not t.is_contiguous():
+            raise ValueError("fp8bs expects contiguous tensors")
+
+
+def _codes(t):
+    """uint8 view of an e4m3fn (or uint8) tensor."""
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8)
+    if t.dtype == torch.uint8:
+        return t
+    raise TypeError("expected float8_e4m3fn or uint8 codes, got %s" % t.dtype)
+
+
+def _scale_fmt(scale_fmt):
+    if scale_fmt is None:
+        return SCALE_FMT_NONE
+    if scale_fmt == "ue8m0":
+        return SCALE_FMT_UE8M0
+    raise ValueError("scale_fmt must be None or 'ue8m0'")
+
+
+def act_quant(x, block_size=128, scale_fmt=None):
+    """Dynamic 1 x block_size quantization of the last dimension.
+
+    Returns ``q`` (float8_e4m3fn, same shape as x) and ``s`` (float32,
+    ``x.shape[:-1] + (x.shape[-1] // block_size,)``)."""
+    _need_cuda(x)
+    if x.dtype == torch.bfloat16:
+        dt = DTYPE_BF16
+    elif x.dtype == torch.float32:
+        dt = DTYPE_F32
+    else:
+        raise TypeError("x must be bfloat16 or float32")
+    if x.shape[-1] % block_size != 0:
+        raise ValueError("last dimension must be a multiple of block_size")
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty(*x.shape[:-1], cols // block_size, dtype=torch.float32, device=x.device)
+    _check(lib().fp8bs_act_quant(_ptr(x), dt, rows, cols, block_size, _scale_fmt(scale_fmt),
+                                 _ptr(q), _ptr(s), _stream(x.device)))
+    return q, s
+
+
+def weight_dequant(x, s, block_size=128, out_dtype=torch.bfloat16):
+    """y[i, j] = x[i, j] * s[i // block_size, j // block_size] (fp32 product,
+    rounded to ``out_dtype``, bfloat16 or float32)."""
+    x = _codes(x)
+    _need_cuda(x, s)
+    if x.dim() != 2:
+        raise ValueError("weight_dequant expects a 2-D weight")
+    M, N = x.shape
+    if tuple(s.shape) != (-(-M // block_size), -(-N // block_size)) or s.dtype != torch.float32:
+        raise ValueError("s must be float32 of shape (cdiv(M, block), cdiv(N, block))")
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[out_dtype]
+    y = torch.empty(M, N, dtype=out_dtype, device=x.device)
+    _check(lib().fp8bs_weight_dequant(_ptr(x), _ptr(s), M, N, block_size, _ptr(y), dt,
+                                      _stream(x.device)))
+    return y
+
+
+def weight_quant(w, block_size=128, scale_fmt=None):
+    """128 x 128 block quantization of a dense 2-D weight -> (q e4m3fn, s float32)."""
+    _need_cuda(w)
+    if w.dim() != 2:
+        raise ValueError("weight_quant expects a 2-D weight")
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[w.dtype]
+    M, N = w.shape
+    q = torch.empty(M, N, dtype=torch.float8_e4m3fn, device=w.device)
+    s = torch.empty(-(-M // block_size), -(-N // block_size), dtype=torch.float32, device=w.device)
+    _check(lib().fp8bs_weight_quant(_ptr(w), dt, M, N, block_size, _scale_fmt(scale_fmt),
+                                    _ptr(q), _ptr(s), _stream(w.device)))
+    return q, s
+
+
+def gemm_workspace_size(M, N, K):
+    """Bytes of scratch fp8_gemm needs for an M x N x K problem on this device."""
+    return int(lib().fp8bs_gemm_workspace_size(M, N, K))
+
+
+def _workspace(M, N, K, device):
+    n = gemm_workspace_size(M, N, K)
+    if n == 0:
+        return None, 0
+    return torch.empty(n, dtype=torch.uint8, device=device), n
+
+
+def fp8_gemm(a, a_s, b, b_s):
+    """y = a @ b^T on block-scaled FP8 operands, bf16 output.
+
+    a: [..., K] e4m3fn, a_s: [..., K/128] float32, b: [N, K] e4m3fn,
+    b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] bfloat16."""
+    a, b = _codes(a), _codes(b)
+    _need_cuda(a, a_s, b, b_s)
+    K = a.shape[-1]
+    M = a.numel() // K if K else 0
+    N = b.shape[0]
+    y = torch.empty(*a.shape[:-1], N, dtype=torch.bfloat16, device=a.device)
+    ws, nws = _workspace(M, N, K, a.device)
+    _check(lib().fp8bs_fp8_gemm(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, _ptr(y),
+                                _ptr(ws), nws, _stream(a.device)))
+    return y
+
+
+def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False):
+    """FP8 linear forward: act_quant(x) then fp8_gemm with the block-scaled weight.
+
+    x: [..., K] bfloat16, weight: [N, K] e4m3fn, weight_scale: [cdiv(N,128), K/128]."""
+    w = _codes(weight)
+    _need_cuda(x, w, weight_scale)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    N = w.shape[0]
+    y = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
+    q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty(*x.shape[:-1], K // 128, dtype=torch.float32, device=x.device)
+    ws, nws = _workspace(M, N, K, x.device)
+    _check(lib().fp8bs_fp8_linear(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
+                                  _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s), _ptr(ws), nws,
+                                  _stream(x.device)))
+    return (y, q, s) if return_quant else y
+
+
+def fp8_gemm_grouped(a, a_s, w, w_s, m_offsets):
+    """Per-expert FP8 GEMMs over rows grouped contiguously by expert.
+
+    a: [M_total, K] e4m3fn, a_s: [M_total, K/128], w: [G, N, K] e4m3fn,
+    w_s: [G, cdiv(N,128), K/128], m_offsets: [G+1] int64 on the device."""
+    a, w = _codes(a), _codes(w)
+    _need_cuda(a, a_s, w, w_s, m_offsets)
+    if m_offsets.dtype != torch.int64:
+        raise TypeError("m_offsets must be int64")
+    G, N, K = w.shape
+    M = a.shape[0]
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    _check(lib().fp8bs_fp8_gemm_grouped(G, _ptr(m_offsets), M, _ptr(a), _ptr(a_s), _ptr(w),
+                                        _ptr(w_s), N, K, _ptr(y), _stream(a.device)))
+    return y
+
+
+def device_error(device=None):
+    """Synchronize the current stream, then read and clear the device error word."""
+    code = ctypes.c_int(0)
+    _check(lib().fp8bs_get_device_error(_stream(device), ctypes.byref(code)))
+    return code.value

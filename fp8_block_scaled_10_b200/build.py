@@ -1,0 +1,58 @@
+"""Build libfp8bs.so (the CUDA kernels and their C ABI) in-tree for sm_100a.
+
+    python -m fp8_block_scaled_10_b200.build [--force]
+
+nvcc cross-compiles without a GPU.  No fast-math flags: the quantizers rely
+on IEEE division and on fp32 subnormals being kept.
+"""
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libfp8bs.so")
+SOURCES = [os.path.join(CSRC, "fp8bs.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
+    [os.path.join(INCLUDE, "fp8bs.h")]
+
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-std=c++17", "-lineinfo",
+    "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared",
+    "-Xptxas", "-v",
+    "-I", INCLUDE, "-I", CSRC,
+    "-DFP8BS_BUILD",
+]
+
+
+def _stale():
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(d) > t for d in DEPS)
+
+
+def build(force=False, verbose=False):
+    """Compile libfp8bs.so if it is missing or older than its sources."""
+    if not force and not _stale():
+        return LIB
+    tmp = LIB + ".tmp.%d" % os.getpid()
+    cmd = [NVCC, *FLAGS, *SOURCES, "-o", tmp]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libfp8bs.so")
+    with open(os.path.join(PKG, "ptxas_report.txt"), "w") as f:
+        f.write(res.stderr)
+    if verbose:
+        sys.stderr.write(res.stderr)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

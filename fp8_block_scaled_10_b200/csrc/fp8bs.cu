@@ -1,0 +1,469 @@
+// C ABI of libfp8bs.so (declared in include/fp8bs.h): argument checks, launch
+// configuration, TMA descriptors and the per-device error word.  The kernels
+// live in quant.cuh (act_quant, weight_dequant, weight_quant, split-K
+// reduction) and gemm.cuh (block-scaled FP8 GEMM).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fp8bs.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+#include "sm100.cuh"
+
+namespace fp8bs {
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+fp8bs_status fail(fp8bs_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+fp8bs_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FP8BS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Opts the GEMM kernel into its dynamic shared memory and checks that the
+// registers it is launched with cover its warpgroup register split (a split
+// larger than the launch total would make setmaxnreg.inc wait forever).
+template <int BN, bool G>
+fp8bs_status setup_gemm_kernel() {
+  using C = gemm::Cfg<BN>;
+  cudaError_t e = cudaFuncSetAttribute(gemm::fp8_gemm_kernel<BN, G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::smem_bytes(G));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (C::kSplitRegs) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, gemm::fp8_gemm_kernel<BN, G>);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    const long launch_total = static_cast<long>(fa.numRegs) * C::kThreads;
+    const long split_total = 128L * C::kCtrlRegs + 32L * C::kEpiWarps * C::kEpiRegs;
+    if (fa.numRegs > 168 || split_total > launch_total)
+      return fail(FP8BS_ERR_UNSUPPORTED,
+                  "GEMM BN=%d register split %ld exceeds launch total %ld (%d regs/thread)", BN,
+                  split_total, launch_total, fa.numRegs);
+  }
+  return FP8BS_OK;
+}
+
+// One-time per-device setup: SM count, shared-memory opt-in of the GEMM
+// kernels, and the driver's tensor-map encoder.
+fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8BS_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+      return fail(FP8BS_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                  dev, major, minor);
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    fp8bs_status r;
+    if ((r = setup_gemm_kernel<128, false>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, true>()) != FP8BS_OK)
+      return r;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *dev_out = dev;
+  *info_out = &d;
+  return FP8BS_OK;
+}
+
+// 2-D tensor map over a row-major uint8 matrix [rows, cols] read in boxes of
+// [box_rows, 128] with the 128-byte swizzle; out-of-range rows read as zero.
+fp8bs_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                       int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t elem[2] = {1u, 1u};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                              strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP8BS_OK;
+}
+
+int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
+  const int64_t need = (work_items + per_cta - 1) / per_cta;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, max_ctas)));
+}
+
+// ---------------------------------------------------------------------------
+// GEMM planning: tile width BN and split-K factor.
+// ---------------------------------------------------------------------------
+struct Plan {
+  int bn;
+  int m_tiles, n_tiles;
+  int splits, kb_per_split;
+  int units;
+};
+
+double wave_efficiency(int64_t units, int sms) {
+  const int64_t waves = (units + sms - 1) / sms;
+  return static_cast<double>(units) / static_cast<double>(waves * sms);
+}
+
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
+  Plan best{};
+  double best_score = -1.0;
+  const int kbn = static_cast<int>(K / 128);
+  for (int bn : {256, 128}) {
+    const int m_tiles = static_cast<int>((M + 127) / 128);
+    const int n_tiles = static_cast<int>((N + bn - 1) / bn);
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    // Split K only when the tiles alone cannot fill the GPU.
+    const int max_split = tiles >= sms ? 1 : std::min(16, std::max(1, kbn / 4));
+    for (int s = 1; s <= max_split; ++s) {
+      const int per = (kbn + s - 1) / s;
+      const int splits = (kbn + per - 1) / per;
+      if (splits != s) continue;
+      const int64_t units = tiles * splits;
+      // Work in units of 128x128x128 MMA blocks, per SM, including idle SMs
+      // in the last wave; narrow tiles and extra splits pay a small overhead
+      // (more A re-reads, a reduction pass).
+      const double eff = wave_efficiency(units, sms);
+      const double overhead = (bn == 128 ? 0.97 : 1.0) * (splits > 1 ? 0.95 - 0.002 * splits : 1.0);
+      const double score = eff * overhead;
+      if (score > best_score + 1e-9) {
+        best_score = score;
+        best = Plan{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units)};
+      }
+    }
+  }
+  return best;
+}
+
+size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
+  return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
+}
+
+template <int BN, bool G>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p,
+                        int grid, cudaStream_t st) {
+  gemm::fp8_gemm_kernel<BN, G><<<grid, gemm::Cfg<BN>::kThreads, gemm::Cfg<BN>::smem_bytes(G), st>>>(
+      ta, tw, p);
+  return cudaGetLastError();
+}
+
+fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                 const float* w_s, uint16_t* y, int64_t N, int64_t K) {
+  if (!a || !a_s || !w || !w_s || !y) return fail(FP8BS_ERR_INVALID_ARG, "null operand pointer");
+  if (K <= 0 || K % 128 != 0) return fail(FP8BS_ERR_INVALID_ARG, "K=%lld must be a positive multiple of 128", (long long)K);
+  if (N <= 0 || N > (1 << 30)) return fail(FP8BS_ERR_INVALID_ARG, "N=%lld out of range", (long long)N);
+  if (!aligned16(a) || !aligned16(w) || !aligned16(y))
+    return fail(FP8BS_ERR_INVALID_ARG, "a, w and y must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(a_s) & 3u) || (reinterpret_cast<uintptr_t>(w_s) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "scale pointers must be 4-byte aligned");
+  return FP8BS_OK;
+}
+
+fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
+                      int64_t M, int64_t N, int64_t K, uint16_t* y, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (M == 0) return FP8BS_OK;
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  const Plan pl = plan_gemm(M, N, K, info->sms);
+  const size_t need = plan_workspace(pl, M, N);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+
+  CUtensorMap ta, tw;
+  if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
+  gemm::Params p{};
+  p.sa = a_s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ws = static_cast<float*>(ws);
+  p.m_offsets = nullptr;
+  p.M = M;
+  p.N = static_cast<int>(N);
+  p.kbn = static_cast<int>(K / 128);
+  p.nbn = static_cast<int>((N + 127) / 128);
+  p.m_tiles = pl.m_tiles;
+  p.n_tiles = pl.n_tiles;
+  p.splits = pl.splits;
+  p.kb_per_split = pl.kb_per_split;
+  p.num_units = pl.units;
+  p.groups = 1;
+  const int grid = std::min(pl.units, info->sms);
+  cudaError_t e = pl.bn == 256 ? launch_gemm<256, false>(ta, tw, p, grid, st)
+                               : launch_gemm<128, false>(ta, tw, p, grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
+  if (pl.splits > 1) {
+    const int64_t MN = M * N;
+    splitk_reduce_kernel<<<grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st>>>(
+        static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+  }
+  return FP8BS_OK;
+}
+
+fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
+                           int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
+                           cudaStream_t st) {
+  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  if (rows < 0 || cols <= 0 || cols % block != 0)
+    return fail(FP8BS_ERR_INVALID_ARG, "cols=%lld must be a positive multiple of block", (long long)cols);
+  if (x_dtype != FP8BS_DTYPE_BF16 && x_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "x_dtype");
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
+  if (rows == 0) return FP8BS_OK;
+  if (!x || !q || !s) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "x and q must be 16-byte aligned, s 4-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const int64_t nblocks = rows * (cols / 128);
+  // 16 half-warps per CTA, kActUnroll blocks each per iteration; up to 8 CTAs per SM.
+  const int grid = grid_for(nblocks, 16 * kActUnroll, info->sms * 8);
+  const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
+  if (x_dtype == FP8BS_DTYPE_BF16) {
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    if (ue) act_quant_kernel<__nv_bfloat16, true><<<grid, kActThreads, 0, st>>>(xb, q, s, nblocks);
+    else act_quant_kernel<__nv_bfloat16, false><<<grid, kActThreads, 0, st>>>(xb, q, s, nblocks);
+  } else {
+    const auto* xf = static_cast<const float*>(x);
+    if (ue) act_quant_kernel<float, true><<<grid, kActThreads, 0, st>>>(xf, q, s, nblocks);
+    else act_quant_kernel<float, false><<<grid, kActThreads, 0, st>>>(xf, q, s, nblocks);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return FP8BS_OK;
+}
+
+}  // namespace
+}  // namespace fp8bs
+
+using namespace fp8bs;
+
+extern "C" {
+
+int fp8bs_version(void) { return 100; }
+
+const char* fp8bs_status_string(fp8bs_status status) {
+  switch (status) {
+    case FP8BS_OK: return "FP8BS_OK";
+    case FP8BS_ERR_INVALID_ARG: return "FP8BS_ERR_INVALID_ARG";
+    case FP8BS_ERR_UNSUPPORTED: return "FP8BS_ERR_UNSUPPORTED";
+    case FP8BS_ERR_WORKSPACE: return "FP8BS_ERR_WORKSPACE";
+    case FP8BS_ERR_CUDA: return "FP8BS_ERR_CUDA";
+    case FP8BS_ERR_TIMEOUT: return "FP8BS_ERR_TIMEOUT";
+  }
+  return "FP8BS_UNKNOWN_STATUS";
+}
+
+const char* fp8bs_last_error_message(void) { return t_last_error; }
+
+fp8bs_status fp8bs_get_device_error(void* stream, int* code) {
+  if (!code) return fail(FP8BS_ERR_INVALID_ARG, "code is null");
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  }
+  *code = v;
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
+                             int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
+                             void* stream) {
+  return run_act_quant(x, x_dtype, rows, cols, block, fmt, q, s, as_stream(stream));
+}
+
+fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, int64_t N,
+                                  int64_t block, void* y, fp8bs_dtype y_dtype, void* stream) {
+  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  if (M < 0 || N < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
+  if (y_dtype != FP8BS_DTYPE_BF16 && y_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "y_dtype");
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!q || !s || !y) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(y) || (reinterpret_cast<uintptr_t>(s) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "q and y must be 16-byte aligned, s 4-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  cudaStream_t st = as_stream(stream);
+  const int64_t nbn = (N + 127) / 128;
+  const bool bf = y_dtype == FP8BS_DTYPE_BF16;
+  if (N % 16 == 0 && N / 16 <= 0xFFFFFFFFll) {
+    const uint32_t cpr = static_cast<uint32_t>(N / 16);
+    const int grid = grid_for(M * cpr, kDeqThreads * kDeqUnroll, info->sms * 8);
+    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, cpr, nbn);
+    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, cpr, nbn);
+  } else {
+    const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
+    if (bf) weight_dequant_any_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);
+    else weight_dequant_any_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "weight_dequant launch");
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, int64_t N,
+                                int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
+                                void* stream) {
+  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  if (M < 0 || N < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
+  if (w_dtype != FP8BS_DTYPE_BF16 && w_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "w_dtype");
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!w || !q || !s) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  const int64_t rb = (M + 127) / 128, cb = (N + 127) / 128;
+  if (rb > 65535 || cb > 0x7FFFFFFF) return fail(FP8BS_ERR_INVALID_ARG, "matrix too large");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const dim3 grid(static_cast<unsigned>(cb), static_cast<unsigned>(rb));
+  const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
+  cudaStream_t st = as_stream(stream);
+  if (w_dtype == FP8BS_DTYPE_F32)
+    weight_quant_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(w), q, s, M, N, cb, ue);
+  else
+    weight_quant_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "weight_quant launch");
+  return FP8BS_OK;
+}
+
+size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  int dev;
+  DeviceInfo* info;
+  if (device_setup(&dev, &info) != FP8BS_OK) return 0;
+  return plan_workspace(plan_gemm(M, N, K, info->sms), M, N);
+}
+
+fp8bs_status fp8bs_fp8_gemm(const uint8_t* a, const float* a_s, const uint8_t* w,
+                            const float* w_s, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return run_gemm(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream));
+}
+
+fp8bs_status fp8bs_fp8_linear(const uint16_t* x, int64_t M, int64_t K, fp8bs_scale_fmt fmt,
+                              const uint8_t* w, const float* w_s, int64_t N, uint16_t* y,
+                              uint8_t* q, float* s, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  fp8bs_status r = check_gemm_operands(q, s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M == 0) return FP8BS_OK;
+  cudaStream_t st = as_stream(stream);
+  if ((r = run_act_quant(x, FP8BS_DTYPE_BF16, M, K, 128, fmt, q, s, st)) != FP8BS_OK) return r;
+  return run_gemm(q, s, w, w_s, M, N, K, y, workspace, workspace_bytes, st);
+}
+
+fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t M_total,
+                                    const uint8_t* a, const float* a_s, const uint8_t* w,
+                                    const float* w_s, int64_t N, int64_t K, uint16_t* y,
+                                    void* stream) {
+  if (G < 1 || G > gemm::kMaxGroups) return fail(FP8BS_ERR_INVALID_ARG, "G=%lld out of [1, %d]", (long long)G, gemm::kMaxGroups);
+  if (!m_offsets || (reinterpret_cast<uintptr_t>(m_offsets) & 7u))
+    return fail(FP8BS_ERR_INVALID_ARG, "m_offsets must be an 8-byte aligned device pointer");
+  fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M_total < 0 || M_total > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M_total out of range");
+  if (M_total == 0) return FP8BS_OK;
+  if (G * N > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "G*N too large");
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  const int bn = N >= 256 ? 256 : 128;
+  CUtensorMap ta, tw;
+  if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
+  gemm::Params p{};
+  p.sa = a_s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ws = nullptr;
+  p.m_offsets = m_offsets;
+  p.M = M_total;
+  p.N = static_cast<int>(N);
+  p.kbn = static_cast<int>(K / 128);
+  p.nbn = static_cast<int>((N + 127) / 128);
+  p.m_tiles = 0;
+  p.n_tiles = static_cast<int>((N + bn - 1) / bn);
+  p.splits = 1;
+  p.kb_per_split = p.kbn;
+  p.num_units = 0;
+  p.groups = static_cast<int>(G);
+  // Units are only known on the device; an upper bound sizes the grid.
+  const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
+  cudaError_t e = bn == 256 ? launch_gemm<256, true>(ta, tw, p, grid, as_stream(stream))
+                            : launch_gemm<128, true>(ta, tw, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
+  return FP8BS_OK;
+}
+
+}  // extern "C"

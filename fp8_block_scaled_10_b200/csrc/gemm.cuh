@@ -1,0 +1,420 @@
+// Block-scaled FP8 GEMM for sm_100a: y = A * W^T with A [M, K] and W [N, K]
+// in e4m3fn, activation scales a_s [M, K/128] (one per 1x128 block) and weight
+// scales w_s [cdiv(N,128), K/128] (one per 128x128 block), FP32 accumulation,
+// bf16 output:
+//   y[m, n] = sum_kb a_s[m, kb] * w_s[n/128, kb] * P_kb[m, n],
+//   P_kb    = sum over the 128 k of block kb of A[m, k] * W[n, k].
+// ("How weight_dequant Handles Per-Block Scaling in DeepSeek-V3 FP8 GEMM",
+// section "Relationship to FP8 GEMM Operations": fp8_gemm(a, a_s, b, b_s) with
+// the scaling fused into the matrix product; "DeepSeek-V3: How Selective FP8
+// Stays Stable", section "Learning outcomes": partial sums promoted to FP32.)
+//
+// Blackwell form of the promotion.  Each 128-wide K block is one group of four
+// tcgen05.mma (K = 32 each) that writes a fresh FP32 partial P_kb into one of
+// two TMEM buffers; the epilogue warps read it back with tcgen05.ld and fold
+// it into register accumulators with one FMA per element by
+// a_s[m, kb] * w_s[nb, kb], while the tensor core fills the other buffer.
+//
+// Roles (persistent CTAs, one per SM, walking work units in a fixed order):
+//   warp 0     TMA producer: A tile [128 x 128] and W tile [BN x 128] per K
+//              block into a ring of shared-memory stages (128B swizzle).
+//   warp 1     owns the TMEM allocation; one lane issues the MMAs.
+//   epilogue   warps kFirstEpiWarp..: warp w reads TMEM lanes 32*(w%4)..+31
+//              (one output row per thread) and 128 columns (column group
+//              (w - kFirstEpiWarp) / 4).
+// A work unit is (m tile, n tile, K split).  With one split the epilogue
+// writes bf16; with several it writes FP32 partials that a reduction kernel
+// sums.  Grouped mode (experts) walks (expert, m tile, n tile) units whose
+// rows come from device-side prefix offsets.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+namespace fp8bs {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 128;
+constexpr int kMaxGroups = 1024;
+
+struct Params {
+  const float* sa;          // [M_total, kbn]
+  const float* sw;          // [G][nbn][kbn]
+  __nv_bfloat16* y;         // [M_total, N]
+  float* ws;                // [splits][M][N] FP32 partials when splits > 1
+  const int64_t* m_offsets; // grouped mode: [G + 1] prefix row offsets (device)
+  int64_t M;                // rows of A (M_total in grouped mode)
+  int N;
+  int kbn;                  // K / 128
+  int nbn;                  // cdiv(N, 128)
+  int m_tiles;              // dense mode
+  int n_tiles;
+  int splits;
+  int kb_per_split;
+  int num_units;            // dense mode; grouped mode derives it on the device
+  int groups;               // grouped mode
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kEpiWarps = BN / 32;
+  // BN = 256: warps 0-3 form a control warpgroup that hands registers to the
+  // two epilogue warpgroups (setmaxnreg); BN = 128: warps 0-1 control, 2-5
+  // epilogue, and every thread can hold the 128 accumulators at launch.
+  static constexpr int kFirstEpiWarp = (BN == 256) ? 4 : 2;
+  static constexpr bool kSplitRegs = (BN == 256);
+  static constexpr int kCtrlRegs = 40;
+  static constexpr int kEpiRegs = 232;
+  static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
+  static constexpr int kABytes = BM * BK;
+  static constexpr int kBBytes = BN * BK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kCtrlBytes = 256;
+  // grouped mode: per-group m-tile prefix (int) and clamped [lo, hi) rows (int64)
+  static constexpr int kGroupBytes = 8 * 2 * kMaxGroups + 4 * (kMaxGroups + 1);
+  static constexpr int smem_bytes(bool grouped) {
+    return kStages * kStageBytes + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1024;
+  }
+};
+
+// Control block at the end of the tile ring.
+template <int kStages>
+struct Ctrl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t flush;
+  uint32_t tmem_base;
+  int abort_flag;
+  int num_units;
+};
+
+struct Unit {
+  int64_t row0;      // first A/y row of the tile
+  int64_t row_end;   // rows >= row_end are not stored
+  int64_t w_row0;    // first W row (grouped: expert * N + n0)
+  int group;
+  int n_tile;
+  int kb0, kb1;
+  int split;
+};
+
+// Dense units: m tile fastest, so the CTAs running at the same time share W
+// tiles (and sweep all of A, which stays in L2).
+__device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
+  Unit t;
+  const int m_tile = u % p.m_tiles;
+  const int rest = u / p.m_tiles;
+  t.split = rest % p.splits;
+  t.n_tile = rest / p.splits;
+  t.group = 0;
+  t.row0 = static_cast<int64_t>(m_tile) * BM;
+  t.row_end = p.M;
+  t.kb0 = t.split * p.kb_per_split;
+  t.kb1 = min(p.kbn, t.kb0 + p.kb_per_split);
+  return t;
+}
+
+// Grouped units: n tile fastest inside one global m tile, so the CTAs running
+// at the same time work on one or two experts and read each W_e once.
+// tile_prefix[g] is the number of m tiles of groups < g; rows[2g], rows[2g+1]
+// are group g's clamped row range [lo, hi).
+__device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix,
+                                             const int64_t* rows, int u) {
+  Unit t;
+  const int gm = u / p.n_tiles;
+  t.n_tile = u % p.n_tiles;
+  int a = 0, b = p.groups;
+  while (b - a > 1) {
+    const int mid = (a + b) >> 1;
+    if (tile_prefix[mid] <= gm) a = mid; else b = mid;
+  }
+  t.group = a;
+  t.row0 = rows[2 * a] + static_cast<int64_t>(gm - tile_prefix[a]) * BM;
+  t.row_end = rows[2 * a + 1];
+  t.split = 0;
+  t.kb0 = 0;
+  t.kb1 = p.kbn;
+  return t;
+}
+
+template <int BN, bool GROUPED>
+__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                    const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* a_tiles = smem;
+  uint8_t* b_tiles = smem + C::kStages * C::kABytes;
+  Ctrl<C::kStages>* ctrl = reinterpret_cast<Ctrl<C::kStages>*>(smem + C::kStages * C::kStageBytes);
+  static_assert(sizeof(Ctrl<C::kStages>) <= C::kCtrlBytes, "control block too large");
+  uint64_t* full = ctrl->full;
+  uint64_t* empty = ctrl->empty;
+  uint64_t* tfull = ctrl->tfull;
+  uint64_t* tempty = ctrl->tempty;
+  uint64_t* flush = &ctrl->flush;
+  volatile int* abort_flag = &ctrl->abort_flag;
+  int64_t* group_rows = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
+  int* tile_prefix = reinterpret_cast<int*>(group_rows + 2 * kMaxGroups);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::kEpiWarps);
+    }
+    mbar_init(flush, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_descriptor(&tmap_a);
+    tma_prefetch_descriptor(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (GROUPED) {
+    // Clamp the device offsets to [0, M], count each group's m tiles and form
+    // their exclusive prefix sum (warp 2, 32 groups per step).
+    if (warp == 2) {
+      int carry = 0;
+      for (int g0 = 0; g0 < p.groups; g0 += 32) {
+        const int g = g0 + lane;
+        int tiles = 0;
+        if (g < p.groups) {
+          int64_t lo = p.m_offsets[g], hi = p.m_offsets[g + 1];
+          lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
+          hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
+          tiles = static_cast<int>((hi - lo + BM - 1) / BM);
+          group_rows[2 * g] = lo;
+          group_rows[2 * g + 1] = hi;
+        }
+        int incl = tiles;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        if (g < p.groups) tile_prefix[g] = carry + incl - tiles;
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      if (lane == 0) {
+        tile_prefix[p.groups] = carry;
+        ctrl->num_units = carry * p.n_tiles;
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    ctrl->num_units = p.num_units;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctrl->tmem_base;
+  const int num_units = ctrl->num_units;
+
+  auto unit_of = [&](int u) -> Unit {
+    Unit t;
+    if (GROUPED) {
+      t = grouped_unit(p, tile_prefix, group_rows, u);
+      t.w_row0 = static_cast<int64_t>(t.group) * p.N + static_cast<int64_t>(t.n_tile) * BN;
+    } else {
+      t = dense_unit(p, u);
+      t.w_row0 = static_cast<int64_t>(t.n_tile) * BN;
+    }
+    return t;
+  };
+
+  if (warp < C::kFirstEpiWarp) {
+    if (C::kSplitRegs) reg_release<C::kCtrlRegs>();
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;       // stages with a TMA load issued
+      uint32_t armed_phase = 0; // parity each armed stage completes
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        const Unit t = unit_of(u);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
+                      static_cast<int32_t>(t.row0));
+          tma_load_2d(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
+                      static_cast<int32_t>(t.w_row0));
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (*abort_flag) {
+        // Let every load in flight land before the CTA exits.
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int tb = 0;
+      uint32_t tphase = 0;
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+        const Unit t = unit_of(u);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
+          tc_fence_after();
+          if (!mbar_wait(&full[stage], phase, abort_flag)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
+          const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_f8f6f4(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
+                       smem_desc_k_sw128(b_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[tb]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          tb ^= 1;
+          if (tb == 0) tphase ^= 1u;
+        }
+      }
+    mma_done:
+      // Every MMA issued must finish before the TMEM columns are released.
+      mma_commit(flush);
+      mbar_wait(flush, 0, nullptr);
+    }
+    __syncwarp();
+  }
+  } else {
+    if (C::kSplitRegs) reg_acquire<C::kEpiRegs>();
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - C::kFirstEpiWarp;
+    const int quad = warp & 3;
+    const int g = e >> 2;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const bool vec_store = (p.N % 8) == 0;
+    int tb = 0;
+    uint32_t tphase = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const Unit t = unit_of(u);
+      const int64_t row = t.row0 + row_in_tile;
+      const bool row_ok = row < t.row_end;
+      const int nb = (t.n_tile * BN) / 128 + g;
+      const bool nb_ok = nb < p.nbn;
+      const float* sa_row = p.sa + (row_ok ? row : 0) * static_cast<int64_t>(p.kbn);
+      const float* sw_row =
+          p.sw + (static_cast<int64_t>(t.group) * p.nbn + (nb_ok ? nb : 0)) * p.kbn;
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      float sa_next = row_ok ? __ldg(sa_row + t.kb0) : 0.0f;
+      float sw_next = nb_ok ? __ldg(sw_row + t.kb0) : 0.0f;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const float scale = sa_next * sw_next;
+        if (kb + 1 < t.kb1) {
+          sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
+          sw_next = nb_ok ? __ldg(sw_row + kb + 1) : 0.0f;
+        }
+        const bool ok = mbar_wait(&tfull[tb], tphase, abort_flag);
+        if (!__all_sync(0xFFFFFFFFu, ok)) goto epilogue_done;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(tb * BN + g * 128 + c * 32), v);
+          tmem_ld_wait();
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tb]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            acc[c * 32 + j] = fmaf(__uint_as_float(v[j]), scale, acc[c * 32 + j]);
+        }
+        tb ^= 1;
+        if (tb == 0) tphase ^= 1u;
+      }
+      if (row_ok) {
+        const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * 128;
+        if (p.splits == 1) {
+          __nv_bfloat16* yrow = p.y + row * p.N;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int64_t col = col0 + c * 8;
+            if (vec_store && col + 8 <= p.N) {
+              uint32_t h[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 b2 =
+                    __floats2bfloat162_rn(acc[c * 8 + 2 * j], acc[c * 8 + 2 * j + 1]);
+                h[j] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(h[0], h[1], h[2], h[3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (col + j < p.N) yrow[col + j] = __float2bfloat16_rn(acc[c * 8 + j]);
+            }
+          }
+        } else {
+          float* wrow = p.ws + (static_cast<int64_t>(t.split) * p.M + row) * p.N;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int64_t col = col0 + c * 4;
+            if ((p.N % 4) == 0 && col + 4 <= p.N) {
+              *reinterpret_cast<float4*>(wrow + col) =
+                  make_float4(acc[c * 4], acc[c * 4 + 1], acc[c * 4 + 2], acc[c * 4 + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (col + j < p.N) wrow[col + j] = acc[c * 4 + j];
+            }
+          }
+        }
+      }
+    }
+  epilogue_done:;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace gemm
+}  // namespace fp8bs

@@ -1,0 +1,308 @@
+// Streaming kernels of the FP8 block-scaled path: dynamic 1x128 activation
+// quantization (act_quant), 128x128-block weight dequantization
+// (weight_dequant), the per-tile weight quantizer (weight_quant) and the
+// split-K reduction of the GEMM.
+//
+// act_quant follows "Understanding Dynamic and Static Activation Quantization
+// Schemes in DeepSeek-V3", section "How Dynamic Activation Quantization
+// Works", and "DeepSeek-V3 quantization_config Parameters Explained", section
+// "The activation_scheme Parameter": per block of 128 channels,
+// s = max(amax, 1e-4) / 448 (optionally a power of two, "ue8m0"), q = x / s
+// cast to float8_e4m3fn.  weight_dequant follows "How weight_dequant Handles
+// Per-Block Scaling in DeepSeek-V3 FP8 GEMM", sections "Grid Mapping and Scale
+// Lookup" and "Dequantization Computation": y = fp8 * s[i/128, j/128] in fp32,
+// masked at ragged edges.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+namespace fp8bs {
+
+// ---------------------------------------------------------------------------
+// Scalar pieces
+// ---------------------------------------------------------------------------
+
+// s = max(amax, 1e-4f) / 448 with IEEE division; for ue8m0 the smallest power
+// of two >= s, taken on the bit pattern (s is a positive normal number here:
+// s >= 1e-4/448): a nonzero fraction bumps the exponent and clears the
+// fraction.
+__device__ __forceinline__ float block_scale(float amax, bool ue8m0) {
+  float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+  if (ue8m0) {
+    uint32_t u = __float_as_uint(s);
+    if (u & 0x007FFFFFu) u = (u & 0x7F800000u) + 0x00800000u;
+    s = __uint_as_float(u);
+  }
+  return s;
+}
+
+// Round-to-nearest-even, saturating fp32 -> e4m3fn of two values; `lo` lands
+// in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// True when fl32(x/s) might round to a different e4m3 code than t = x * r,
+// r = RN(1/s).  t is within 1.5 * 2^-23 |x/s| of x/s (two roundings of
+// relative size <= 2^-24), and fl32(x/s) within half an ulp of it, so the two
+// fp32 values are at most 3 ulps apart.  e4m3 rounding decisions for
+// 2^-6 <= |t| < 512 sit where the 20 bits below e4m3's 3-bit fraction equal
+// 0x80000 (the halfway point); any t within 4 ulps of such a pattern, and
+// any 0 < |t| < 2^-6 (the e4m3 subnormal range), takes the exact division
+// instead.  t == 0 needs nothing: then x == 0 and x / s is that same zero.
+__device__ __forceinline__ bool near_e4m3_midpoint(float t) {
+  const uint32_t u = __float_as_uint(t) & 0x7FFFFFFFu;
+  return (u - 1u < 0x3C7FFFFFu) || (((u & 0x000FFFFFu) - 0x0007FFFCu) < 9u);
+}
+
+// Quantizes 8 values of one block and packs the codes (element 0 in the low
+// byte).  For ue8m0, r = 1/s is an exact power of two, so x * r is exactly
+// the correctly rounded x / s.
+template <bool UE8M0>
+__device__ __forceinline__ uint2 quantize8(const float (&v)[8], float s, float r) {
+  float t[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) t[j] = v[j] * r;
+  if (!UE8M0) {
+    uint32_t mask = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mask |= static_cast<uint32_t>(near_e4m3_midpoint(t[j])) << j;
+    if (mask) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (mask & (1u << j)) t[j] = __fdiv_rn(v[j], s);
+    }
+  }
+  uint2 out;
+  out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+  out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
+  return out;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// ---------------------------------------------------------------------------
+// act_quant
+// ---------------------------------------------------------------------------
+// The input is a flat run of nblocks blocks of 128 elements (the last
+// dimension is a multiple of 128, so blocks never straddle rows) and block b's
+// scale is s[b].  A half-warp owns one block: each of its 16 lanes holds 8
+// consecutive elements (16 bytes of bf16), the amax is a 4-step xor shuffle
+// inside the half-warp, and each lane writes 8 code bytes.  Every warp
+// handles kUnroll block pairs per iteration with all loads issued first.
+constexpr int kActThreads = 256;
+constexpr int kActUnroll = 4;
+
+template <typename T, bool UE8M0>
+__global__ void __launch_bounds__(kActThreads)
+    act_quant_kernel(const T* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
+                     int64_t nblocks) {
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kActThreads) >> 5;
+  const int64_t step = nwarps * 2 * kActUnroll;
+
+  for (int64_t base = warp * 2 * kActUnroll; base < nblocks; base += step) {
+    float v[kActUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kActUnroll; ++u) {
+      const int64_t b = base + 2 * u + half;
+      if (b < nblocks) {
+        load8(x + b * 128 + l16 * 8, v[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kActUnroll; ++u) {
+      const int64_t b = base + 2 * u + half;
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[u][j]));
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+      const float sc = block_scale(amax, UE8M0);
+      const float r = __frcp_rn(sc);
+      if (b < nblocks) {
+        const uint2 codes = quantize8<UE8M0>(v[u], sc, r);
+        __stcs(reinterpret_cast<uint2*>(q + b * 128 + l16 * 8), codes);
+        if (l16 == 0) __stcs(s + b, sc);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// weight_dequant
+// ---------------------------------------------------------------------------
+
+// Value of an e4m3fn code, from the format definition: the 7 magnitude bits
+// EEEE MMM placed at bit 20 of an fp32 pattern give an fp32 number whose
+// exponent field is EEEE (bias 127 instead of 7) and whose fraction starts
+// with MMM; multiplying by 2^120 restores the bias exactly, for subnormal
+// codes too (they become fp32 subnormals, which are kept: no flush-to-zero).
+// S.1111.111 is NaN.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t mag = code & 0x7Fu;
+  float v = __uint_as_float(mag << 20) * 0x1p120f;
+  v = (mag == 0x7Fu) ? __uint_as_float(0x7FC00000u) : v;
+  return __uint_as_float(__float_as_uint(v) | ((code & 0x80u) << 24));
+}
+
+constexpr int kDeqThreads = 256;
+constexpr int kDeqUnroll = 2;
+
+// Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row;
+// all 16 share one block scale because 16 divides 128.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(kDeqThreads)
+    weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
+                          void* __restrict__ y, int64_t M, uint32_t chunks_per_row,
+                          int64_t nbn) {
+  const int64_t total = M * static_cast<int64_t>(chunks_per_row);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kDeqThreads * kDeqUnroll;
+  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDeqThreads * kDeqUnroll + threadIdx.x;
+       c0 < total; c0 += stride) {
+    uint4 raw[kDeqUnroll];
+    float sc[kDeqUnroll];
+    int64_t off[kDeqUnroll];
+#pragma unroll
+    for (int u = 0; u < kDeqUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(u) * kDeqThreads;
+      if (c < total) {
+        const int64_t row = c / chunks_per_row;
+        const int64_t col = (c - row * chunks_per_row) * 16;
+        off[u] = row * static_cast<int64_t>(chunks_per_row) * 16 + col;
+        raw[u] = __ldcs(reinterpret_cast<const uint4*>(q + off[u]));
+        sc[u] = __ldg(s + (row >> 7) * nbn + (col >> 7));
+      } else {
+        off[u] = -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDeqUnroll; ++u) {
+      if (off[u] < 0) continue;
+      const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = e4m3_value((w[j >> 2] >> (8 * (j & 3))) & 0xFFu) * sc[u];
+      if (OUT_BF16) {
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          h[j] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + off[u]);
+        __stcs(dst, make_uint4(h[0], h[1], h[2], h[3]));
+        __stcs(dst + 1, make_uint4(h[4], h[5], h[6], h[7]));
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + off[u]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          __stcs(dst + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+      }
+    }
+  }
+}
+
+// Element path for any N (ragged widths that are not a multiple of 16).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(kDeqThreads)
+    weight_dequant_any_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
+                              void* __restrict__ y, int64_t M, int64_t N, int64_t nbn) {
+  const int64_t total = M * N;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDeqThreads + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * kDeqThreads) {
+    const int64_t row = i / N, col = i - row * N;
+    const float v = e4m3_value(q[i]) * __ldg(s + (row >> 7) * nbn + (col >> 7));
+    if (OUT_BF16)
+      static_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(y)[i] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// weight_quant: one CTA per 128 x 128 tile (partial at the edges)
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float load_elem(const T* p);
+template <>
+__device__ __forceinline__ float load_elem<float>(const float* p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    weight_quant_kernel(const T* __restrict__ w, uint8_t* __restrict__ q, float* __restrict__ s,
+                        int64_t M, int64_t N, int64_t nbn, bool ue8m0) {
+  __shared__ float red[8];
+  const int64_t bi = blockIdx.y, bj = blockIdx.x;
+  const int64_t r0 = bi * 128, c0 = bj * 128;
+  const int rows = static_cast<int>(M - r0 < 128 ? M - r0 : 128);
+  const int cols = static_cast<int>(N - c0 < 128 ? N - c0 : 128);
+  float amax = 0.0f;
+  for (int e = threadIdx.x; e < rows * 128; e += 256) {
+    const int r = e >> 7, c = e & 127;
+    if (c < cols) amax = fmaxf(amax, fabsf(load_elem(w + (r0 + r) * N + c0 + c)));
+  }
+  for (int off = 16; off >= 1; off >>= 1)
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = block_scale(amax, ue8m0);
+  if (threadIdx.x == 0) s[bi * nbn + bj] = sc;
+  for (int e = threadIdx.x; e < rows * 128; e += 256) {
+    const int r = e >> 7, c = e & 127;
+    if (c < cols) {
+      const int64_t i = (r0 + r) * N + c0 + c;
+      q[i] = static_cast<uint8_t>(e4m3x2(__fdiv_rn(load_elem(w + i), sc), 0.0f) & 0xFFu);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K reduction: y[m, n] = bf16(sum_s ws[s][m][n]), summed in split order.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    splitk_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ y,
+                         int64_t MN, int splits) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < MN;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    float acc = 0.0f;
+    for (int sp = 0; sp < splits; ++sp) acc += ws[sp * MN + i];
+    y[i] = __float2bfloat16_rn(acc);
+  }
+}
+
+}  // namespace fp8bs

@@ -1,0 +1,204 @@
+/*
+ * fp8bs: FP8 block-scaled linear-layer kernels for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libfp8bs.so.  Every entry point takes plain pointers and sizes and
+ * a CUDA stream passed as void* (a cudaStream_t; NULL is the legacy default
+ * stream).  Unless stated otherwise, tensor pointers are DEVICE pointers owned
+ * by the caller, row-major and contiguous, and must be 16-byte aligned.
+ *
+ * Calls are asynchronous.  Argument errors are detected on the host and are
+ * returned before anything is launched.  A failed CUDA launch returns
+ * FP8BS_ERR_CUDA.  Kernel-side failures (a bounded device wait that gave up)
+ * are recorded in a per-device error word that fp8bs_get_device_error()
+ * reads and clears.  fp8bs_last_error_message() describes the last non-OK
+ * status returned on the calling host thread.
+ *
+ * The library allocates no device memory per call.  Kernels that need
+ * scratch space take it from a caller-provided workspace whose size the
+ * matching *_workspace_size() function returns.
+ *
+ * Sources of the operations (page title, then section):
+ *  [ACT] "Understanding Dynamic and Static Activation Quantization Schemes in
+ *        DeepSeek-V3", "How Dynamic Activation Quantization Works";
+ *        "DeepSeek-V3 quantization_config Parameters Explained: e4m3,
+ *        weight_block_size, and activation_scheme", "The activation_scheme
+ *        Parameter" and "The fmt Parameter".
+ *  [DEQ] "How weight_dequant Handles Per-Block Scaling in DeepSeek-V3 FP8
+ *        GEMM", "Grid Mapping and Scale Lookup", "Dequantization
+ *        Computation", "Python Wrapper and Launch Configuration".
+ *  [GEMM] same page, "Relationship to FP8 GEMM Operations" (fp8_gemm(a, a_s,
+ *        b, b_s), scaling fused into the matrix product); "DeepSeek-V3: How
+ *        Selective FP8 Stays Stable", "Learning outcomes" (1x128 activation
+ *        tiles, 128x128 weight blocks, FP32 promotion of partial sums).
+ */
+#ifndef FP8BS_H
+#define FP8BS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(FP8BS_BUILD) && defined(__GNUC__)
+#define FP8BS_API __attribute__((visibility("default")))
+#else
+#define FP8BS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp8bs_status {
+    FP8BS_OK = 0,
+    FP8BS_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or shape; nothing launched */
+    FP8BS_ERR_UNSUPPORTED = 2, /* well-formed but not implemented (e.g. block != 128)    */
+    FP8BS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size()   */
+    FP8BS_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                      */
+    FP8BS_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up (device error word) */
+} fp8bs_status;
+
+typedef enum fp8bs_dtype {
+    FP8BS_DTYPE_BF16 = 0,
+    FP8BS_DTYPE_F32 = 1
+} fp8bs_dtype;
+
+typedef enum fp8bs_scale_fmt {
+    FP8BS_SCALE_FMT_NONE = 0,  /* s = max(amax, 1e-4) / 448 as an fp32 value         */
+    FP8BS_SCALE_FMT_UE8M0 = 1  /* the same s rounded up to a power of two (exactly)   */
+} fp8bs_scale_fmt;
+
+/* Version of this ABI: major * 10000 + minor * 100 + patch. */
+FP8BS_API int fp8bs_version(void);
+
+/* Human-readable name of a status code (static storage). */
+FP8BS_API const char *fp8bs_status_string(fp8bs_status status);
+
+/* Message describing the last non-OK status returned on this host thread
+ * (thread-local storage; empty string if none). */
+FP8BS_API const char *fp8bs_last_error_message(void);
+
+/* Synchronizes `stream`, then reads and clears the device error word of the
+ * current device into *code (FP8BS_OK when no kernel reported a failure).
+ * Returns FP8BS_ERR_CUDA if the synchronization itself failed. */
+FP8BS_API fp8bs_status fp8bs_get_device_error(void *stream, int *code);
+
+/*
+ * act_quant [ACT]: dynamic 1 x block activation quantization.
+ *
+ * For every row r and block b of `block` consecutive elements of the last
+ * dimension:
+ *   amax = max |x[r, b*block + k]|               (in fp32; bf16 widens exactly)
+ *   s[r, b] = max(amax, 1e-4f) / 448.0f          (IEEE fp32 division)
+ *   if fmt == UE8M0: s[r, b] = smallest power of two >= s[r, b]
+ *   q[r, b*block + k] = e4m3fn_rne_satfinite(x / s[r, b])   (IEEE fp32 division)
+ *
+ *   x      device, [rows, cols], bf16 (x_dtype = BF16) or fp32 (F32)
+ *   q      device, [rows, cols], e4m3fn codes (uint8), written
+ *   s      device, [rows, cols / block], fp32, written
+ * cols must be a multiple of block; block must be 128 (others return
+ * FP8BS_ERR_UNSUPPORTED).  rows == 0 is a no-op.  Results are bit-exact with
+ * the definition above.
+ */
+FP8BS_API fp8bs_status fp8bs_act_quant(const void *x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
+                             int64_t block, fp8bs_scale_fmt fmt, uint8_t *q, float *s,
+                             void *stream);
+
+/*
+ * weight_dequant [DEQ]: y[i, j] = round(dec(q[i, j]) * s[i / block, j / block])
+ * with the product taken in fp32 and rounded to the output type
+ * (round-to-nearest-even for bf16).
+ *
+ *   q      device, [M, N] e4m3fn codes (uint8)
+ *   s      device, [cdiv(M, block), cdiv(N, block)] fp32, row-major, so the
+ *          scale of block (bi, bj) sits at bi * cdiv(N, block) + bj
+ *   y      device, [M, N], bf16 (y_dtype = BF16) or fp32 (F32), written
+ * Ragged M and N are allowed (edge blocks are partial).  block must be 128.
+ * M == 0 or N == 0 is a no-op.  Bit-exact with the definition above.
+ */
+FP8BS_API fp8bs_status fp8bs_weight_dequant(const uint8_t *q, const float *s, int64_t M, int64_t N,
+                                  int64_t block, void *y, fp8bs_dtype y_dtype, void *stream);
+
+/*
+ * weight_quant: the inverse of weight_dequant, 128 x 128 block quantization of
+ * a dense weight with the act_quant scale rule applied per tile:
+ *   s[bi, bj] = max(amax_tile, 1e-4f) / 448.0f (optionally rounded up to 2^k)
+ *   q[i, j]   = e4m3fn_rne_satfinite(w[i, j] / s[i / 128, j / 128])
+ *   w      device, [M, N], bf16 or fp32
+ *   q      device, [M, N] uint8, written;  s  device, [cdiv(M,128), cdiv(N,128)] fp32, written
+ * Ragged M and N are allowed.  The pages state the per-tile scale layout that
+ * weight_dequant consumes ([DEQ] "Per-Block Scaling Architecture"); they do
+ * not print the offline quantizer, whose rule is read here as the activation
+ * rule applied per 128 x 128 tile.
+ */
+FP8BS_API fp8bs_status fp8bs_weight_quant(const void *w, fp8bs_dtype w_dtype, int64_t M, int64_t N,
+                                int64_t block, fp8bs_scale_fmt fmt, uint8_t *q, float *s,
+                                void *stream);
+
+/*
+ * fp8_gemm [GEMM]: y = A * W^T on block-scaled FP8 operands, FP32
+ * accumulation, bf16 output:
+ *   y[m, n] = bf16( sum_kb a_s[m, kb] * w_s[n / 128, kb] * P_kb[m, n] ),
+ *   P_kb[m, n] = sum_{k in kb} dec(a[m, k]) * dec(w[n, k]),   kb = k / 128.
+ *
+ *   a      device, [M, K] e4m3fn codes
+ *   a_s    device, [M, K / 128] fp32 (the layout act_quant writes)
+ *   w      device, [N, K] e4m3fn codes (the nn.Linear weight layout)
+ *   w_s    device, [cdiv(N, 128), K / 128] fp32 (the layout weight_dequant reads)
+ *   y      device, [M, N] bf16, written
+ *   workspace / workspace_bytes: device scratch of at least
+ *          fp8bs_gemm_workspace_size(M, N, K) bytes (may be NULL when that is 0);
+ *          its contents on entry do not matter.
+ * K must be a positive multiple of 128.  M and N may be ragged.  M == 0 or
+ * N == 0 is a no-op.  Results are within |dy| <= 4e-3 |y_ref| +
+ * 1e-3 sum_k |a_hat_k w_hat_k| of the exact value y_ref.
+ */
+FP8BS_API size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+FP8BS_API fp8bs_status fp8bs_fp8_gemm(const uint8_t *a, const float *a_s, const uint8_t *w,
+                            const float *w_s, int64_t M, int64_t N, int64_t K, uint16_t *y,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fp8_linear: the FP8 linear layer's forward pass, act_quant followed by
+ * fp8_gemm on one stream ([ACT] notes that the linear wrapper calls act_quant
+ * during the forward pass):
+ *   (q, s) = act_quant(x, 128, fmt);  y = fp8_gemm(q, s, w, w_s)
+ *
+ *   x      device, [M, K] bf16
+ *   w, w_s as for fp8_gemm;  y  device, [M, N] bf16, written
+ *   q      device, [M, K] uint8 and  s  device, [M, K / 128] fp32: caller-
+ *          provided buffers that receive the quantized activations and scales
+ *   workspace as for fp8_gemm (fp8bs_gemm_workspace_size(M, N, K) bytes).
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_linear(const uint16_t *x, int64_t M, int64_t K, fp8bs_scale_fmt fmt,
+                              const uint8_t *w, const float *w_s, int64_t N, uint16_t *y,
+                              uint8_t *q, float *s, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * fp8_gemm_grouped: G independent fp8_gemm problems (experts) that share N
+ * and K, with the rows of A grouped contiguously by problem:
+ *   rows m_offsets[g] .. m_offsets[g+1]-1 of a / a_s / y belong to problem g,
+ *   y[rows of g] = fp8_gemm(a[rows of g], a_s[rows of g], w[g], w_s[g]).
+ *
+ *   m_offsets   DEVICE, G + 1 int64 prefix offsets (m_offsets[0] = 0,
+ *               non-decreasing, m_offsets[G] <= M_total); the host never reads
+ *               them, so routing results need no host synchronization.  A group
+ *               whose end is below its start is empty; rows outside
+ *               [0, M_total) are never read or written.
+ *   a      device, [M_total, K];  a_s  device, [M_total, K / 128]
+ *   w      device, [G, N, K];     w_s  device, [G, cdiv(N, 128), K / 128]
+ *   y      device, [M_total, N] bf16; rows that belong to no group are left
+ *          untouched.
+ * 1 <= G <= 1024.  Same K constraint and tolerance as fp8_gemm.  Needs no
+ * workspace.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t *m_offsets, int64_t M_total,
+                                    const uint8_t *a, const float *a_s, const uint8_t *w,
+                                    const float *w_s, int64_t N, int64_t K, uint16_t *y,
+                                    void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BS_H */

@@ -1,0 +1,81 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/fp8bs.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import subprocess
+
+import pytest
+
+import fp8_block_scaled_10_b200 as fp8bs
+from fp8_block_scaled_10_b200 import build as fbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return fp8bs.lib()
+
+
+def test_header_declares_the_boundary():
+    names = fp8bs.header_symbols()
+    for required in ("fp8bs_act_quant", "fp8bs_weight_dequant", "fp8bs_fp8_gemm",
+                     "fp8bs_fp8_linear", "fp8bs_fp8_gemm_grouped", "fp8bs_weight_quant",
+                     "fp8bs_gemm_workspace_size", "fp8bs_get_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fp8bs.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in fp8bs.header_symbols():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+    # nothing but the declared entry points is exported
+    assert {n for n in exported if n.startswith("fp8bs_")} == set(fp8bs.header_symbols())
+
+
+def test_status_strings(L):
+    assert L.fp8bs_status_string(0) == b"FP8BS_OK"
+    assert L.fp8bs_status_string(3) == b"FP8BS_ERR_WORKSPACE"
+    assert L.fp8bs_version() >= 100
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_host_side_argument_errors_without_gpu(L):
+    dummy = _p(4096)            # never dereferenced: validation fails first
+    # K not a multiple of 128
+    st = L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 8, 256, 100, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    assert b"K=100" in L.fp8bs_last_error_message()
+    # null operand
+    st = L.fp8bs_fp8_gemm(None, dummy, dummy, dummy, 8, 256, 128, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    # misaligned operand
+    st = L.fp8bs_fp8_gemm(_p(4097), dummy, dummy, dummy, 8, 256, 128, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    # block sizes other than 128 are not implemented
+    st = L.fp8bs_act_quant(dummy, 0, 4, 256, 64, 0, dummy, dummy, None)
+    assert st == fp8bs.ERR_UNSUPPORTED
+    # last dimension not a multiple of the block
+    st = L.fp8bs_act_quant(dummy, 0, 4, 200, 128, 0, dummy, dummy, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    # unknown scale format / dtype
+    assert L.fp8bs_act_quant(dummy, 0, 4, 256, 128, 7, dummy, dummy, None) == fp8bs.ERR_INVALID_ARG
+    assert L.fp8bs_weight_dequant(dummy, dummy, 4, 4, 128, dummy, 9, None) == fp8bs.ERR_INVALID_ARG
+    # grouped: G out of range
+    st = L.fp8bs_fp8_gemm_grouped(0, dummy, 8, dummy, dummy, dummy, dummy, 256, 128, dummy, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    # empty problems are successful no-ops
+    assert L.fp8bs_act_quant(None, 0, 0, 256, 128, 0, None, None, None) == fp8bs.OK
+    assert L.fp8bs_weight_dequant(None, None, 0, 16, 128, None, 0, None) == fp8bs.OK
+    assert L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 0, 256, 128, dummy, None, 0, None) == fp8bs.OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        fp8bs.act_quant(torch.zeros(4, 128, dtype=torch.bfloat16))

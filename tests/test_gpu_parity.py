@@ -1,0 +1,324 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle.
+
+Quantization and dequantization are compared byte for byte; the GEMM is held
+to |dy| <= 4e-3 |y_ref| + 1e-3 sum_k |a_k w_k| against the oracle's FP64
+result on the same dequantized operands.  Small cases span several tiles and
+ragged tails; the full-size cases use the workload shapes the benchmark runs
+(compared in full where the oracle is fast enough, else on sampled rows that
+include every tile edge near both ends).
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_block_scaled_10_b200 as fp8bs
+from fp8_block_scaled_10_b200 import workloads as wl
+
+from _util import (assert_gemm_close, cuda_codes, cuda_f32, f32bits, quantized_weight,
+                   sample_rows, u8)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from fp8_block_scaled_10_b200 import build
+    build.build()
+    torch.cuda.init()
+    yield
+    assert fp8bs.device_error() == 0
+
+
+# --------------------------------------------------------------------------
+# act_quant
+# --------------------------------------------------------------------------
+
+def _special_blocks(dtype):
+    """Blocks that stress the scale rule and the e4m3 rounding:
+    zeros, signed zeros, an exact-448 block with ties, tiny values, a single
+    outlier, values that land exactly on e4m3 midpoints after the division."""
+    rows = []
+    z = np.zeros(128, np.float32)
+    rows.append(z.copy())
+    nz = z.copy(); nz[::2] = -0.0; rows.append(nz)
+    t = np.array([448.0] + [1.0625, 1.1875, -3.25, 0.0009765625, -0.0029296875, 464.0 / 2,
+                            2.0 ** -10, 3 * 2.0 ** -10] * 15 + [1.0] * 7, np.float32)[:128]
+    rows.append(t)
+    tiny = np.full(128, 1e-30, np.float32); tiny[5] = -3e-38; rows.append(tiny)
+    out = np.random.default_rng(0).normal(0, 1, 128).astype(np.float32); out[17] = 5000.0
+    rows.append(out)
+    # x = m * s for e4m3 midpoints m, so fl32(x/s) sits on or next to a tie
+    rng = np.random.default_rng(1)
+    for a in (1.0, 3.0, 37.5, 0.1, 7e-3):
+        s = np.float32(a) / np.float32(448.0)
+        e = rng.integers(-6, 8, 128)
+        k = rng.integers(0, 8, 128)
+        m = ((8 + k) + 0.5) * np.exp2(e - 3.0)
+        m = np.minimum(m, 440.0).astype(np.float32) * np.where(rng.random(128) < .5, -1, 1)
+        x = (m * s).astype(np.float32)
+        x[0] = np.float32(a)
+        rows.append(x)
+    x = np.stack(rows).astype(np.float32)
+    if dtype == torch.bfloat16:
+        return torch.from_numpy(x).to(torch.bfloat16)
+    return torch.from_numpy(x)
+
+
+def _oracle_act_quant(x_cpu, fmt):
+    if x_cpu.dtype == torch.bfloat16:
+        arr = wl.bf16_bits(x_cpu)
+    else:
+        arr = x_cpu.numpy()
+    return oracle.act_quant(arr.reshape(-1, arr.shape[-1]), scale_fmt=fmt)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+@pytest.mark.parametrize("shape", [(1, 128), (3, 256), (129, 512), (1000, 1024), (2, 7, 384)])
+def test_act_quant_bit_exact(shape, fmt, dtype):
+    x = wl.normal_with_outliers(int(np.prod(shape[:-1])), shape[-1], seed=sum(shape),
+                                frac=0.01, factor=50.0, dtype=dtype).reshape(shape)
+    q, s = fp8bs.act_quant(x.cuda(), 128, fmt)
+    assert q.dtype == torch.float8_e4m3fn and tuple(s.shape) == shape[:-1] + (shape[-1] // 128,)
+    q_ref, s_ref = _oracle_act_quant(x, fmt)
+    assert np.array_equal(u8(q).reshape(q_ref.shape), q_ref)
+    assert np.array_equal(f32bits(s.cpu().numpy()).reshape(s_ref.shape), f32bits(s_ref))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+def test_act_quant_special_blocks(fmt, dtype):
+    x = _special_blocks(dtype)
+    q, s = fp8bs.act_quant(x.cuda(), 128, fmt)
+    q_ref, s_ref = _oracle_act_quant(x, fmt)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
+    assert np.array_equal(u8(q), q_ref)
+
+
+def test_act_quant_many_midpoints_fp32():
+    """fp32 inputs built as e4m3 midpoint * s: the exact-division fallback runs often."""
+    rng = np.random.default_rng(7)
+    rows, cols = 512, 1024
+    a = np.exp2(rng.uniform(-12, 8, (rows, cols // 128))).astype(np.float32)
+    s = (a / np.float32(448.0)).astype(np.float32)
+    e = rng.integers(-9, 8, (rows, cols))
+    k = rng.integers(0, 16, (rows, cols))
+    m = (k + 0.5) * np.exp2(e - 3.0)
+    m = np.minimum(m, 440.0) * np.where(rng.random((rows, cols)) < .5, -1, 1)
+    x = (m.astype(np.float32) * np.repeat(s, 128, axis=1)).astype(np.float32)
+    x[:, ::128] = a
+    xt = torch.from_numpy(x)
+    q, sg = fp8bs.act_quant(xt.cuda())
+    q_ref, s_ref = oracle.act_quant(x)
+    assert np.array_equal(f32bits(sg.cpu().numpy()), f32bits(s_ref))
+    assert np.array_equal(u8(q), q_ref)
+
+
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+def test_act_quant_full_size(fmt):
+    """act_quant on x bf16 [16384, 7168] ~N(0,1) with 0.1% entries x100, every byte."""
+    x = wl.normal_with_outliers(16384, 7168, seed=20, frac=0.001, factor=100.0)
+    q, s = fp8bs.act_quant(x.cuda(), 128, fmt)
+    q_ref, s_ref = oracle.act_quant(wl.bf16_bits(x), scale_fmt=fmt)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
+    assert np.array_equal(u8(q), q_ref)
+
+
+# --------------------------------------------------------------------------
+# weight_dequant / weight_quant
+# --------------------------------------------------------------------------
+
+def _codes(M, N, seed):
+    return wl.e4m3_codes(M, N, seed=seed).numpy()
+
+
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(128, 128), (256, 576), (129, 130), (300, 1024), (1, 16), (5, 7)])
+def test_weight_dequant_bit_exact(shape, out):
+    M, N = shape
+    q = _codes(M, N, seed=M + N)
+    s = wl.uniform((-(-M // 128), -(-N // 128)), 1e-5, 1e-3, seed=3).numpy()
+    s.flat[0] = -2.5e-4
+    s.flat[-1] = 3.0e4
+    y = fp8bs.weight_dequant(cuda_codes(q), cuda_f32(s), 128,
+                             torch.bfloat16 if out == "bf16" else torch.float32)
+    y_ref = oracle.weight_dequant(q, s, out=out)
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16) if out == "bf16" else y.cpu().numpy()
+    if out == "f32":
+        assert np.array_equal(f32bits(got), f32bits(y_ref))
+    else:
+        assert np.array_equal(got, y_ref)
+
+
+def test_weight_dequant_pages_example_shape():
+    q = _codes(1024, 1024, seed=5)
+    s = wl.uniform((8, 8), 1e-5, 1e-3, seed=6).numpy()
+    y = fp8bs.weight_dequant(cuda_codes(q), cuda_f32(s))
+    assert tuple(y.shape) == (1024, 1024)
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16),
+                          oracle.weight_dequant(q, s))
+
+
+def test_weight_dequant_full_size():
+    """e4m3 W [18432, 7168] (all 254 finite codes), s [144, 56] ~U(1e-5, 1e-3) -> bf16."""
+    q = _codes(18432, 7168, seed=30)
+    s = wl.uniform((144, 56), 1e-5, 1e-3, seed=31).numpy()
+    y = fp8bs.weight_dequant(cuda_codes(q), cuda_f32(s))
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16),
+                          oracle.weight_dequant(q, s))
+
+
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+@pytest.mark.parametrize("shape", [(256, 512), (300, 576), (129, 130), (128, 7168)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_weight_quant_bit_exact(shape, fmt, dtype):
+    w = wl.weight_f32(*shape, seed=shape[0] * 7 + shape[1]).to(dtype)
+    w[0, 0] = 0.5
+    q, s = fp8bs.weight_quant(w.cuda(), 128, fmt)
+    q_ref, s_ref = oracle.weight_quant(w.float().numpy(), scale_fmt=fmt)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
+    assert np.array_equal(u8(q), q_ref)
+
+
+# --------------------------------------------------------------------------
+# fp8_gemm
+# --------------------------------------------------------------------------
+
+def _gemm_case(M, N, K, seed, fmt=None, heavy=False):
+    if heavy:
+        x = wl.heavy_tailed_channels(M, K, seed=seed)
+    else:
+        x = wl.normal_with_outliers(M, K, seed=seed, frac=0.01, factor=50.0)
+    qa, sa = oracle.act_quant(wl.bf16_bits(x), scale_fmt=fmt)
+    qw, sw = quantized_weight(N, K, seed=seed + 1, scale_fmt=fmt)
+    return x, qa, sa, qw, sw
+
+
+def test_gemm_tiny_linear():
+    """x bf16 [128,512] ~N(0,1) with 1% entries x50; W [256,512]; y bf16 [128,256]."""
+    x, qa, sa, qw, sw = _gemm_case(128, 256, 512, seed=0)
+    assert sw.shape == (2, 4)
+    y = fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw))
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "tiny")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 256, 128), (127, 576, 512), (129, 130, 256), (300, 384, 1024), (256, 512, 7168),
+    (513, 1280, 384), (64, 2048, 2048), (2, 18432, 256), (200, 136, 128),
+])
+def test_gemm_shapes(M, N, K):
+    x, qa, sa, qw, sw = _gemm_case(M, N, K, seed=M + N + K)
+    y = fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw))
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "gemm %dx%dx%d" % (M, N, K))
+
+
+def test_gemm_writes_only_its_output():
+    """Canary rows and columns around y stay untouched (raw C-ABI call)."""
+    M, N, K = 130, 200, 256
+    x, qa, sa, qw, sw = _gemm_case(M, N, K, seed=99)
+    a, a_s, w, w_s = cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw)
+    big = torch.full((M + 2, N), -7.0, dtype=torch.bfloat16, device="cuda")
+    y = big[1:M + 1]
+    L = fp8bs.lib()
+    st = L.fp8bs_fp8_gemm(ctypes.c_void_p(a.data_ptr()), ctypes.c_void_p(a_s.data_ptr()),
+                          ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(w_s.data_ptr()),
+                          M, N, K, ctypes.c_void_p(y.data_ptr()), None, 0,
+                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == fp8bs.OK
+    torch.cuda.synchronize()
+    assert torch.all(big[0] == -7.0) and torch.all(big[M + 1] == -7.0)
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "canary")
+
+
+def test_gemm_is_deterministic():
+    x, qa, sa, qw, sw = _gemm_case(64, 7168, 18432 // 4, seed=5, fmt="ue8m0")
+    args = (cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw))
+    y1 = fp8bs.fp8_gemm(*args)
+    y2 = fp8bs.fp8_gemm(*args)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("K,N", wl.DECODE_KN)
+@pytest.mark.parametrize("M", wl.DECODE_M)
+def test_gemm_decode_full(M, K, N):
+    """Decode shapes with ue8m0 scales, every output (split-K path where chosen)."""
+    x, qa, sa, qw, sw = _gemm_case(M, N, K, seed=M * 3 + K, fmt="ue8m0")
+    need = fp8bs.gemm_workspace_size(M, N, K)
+    y = fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw))
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "decode M=%d K=%d N=%d ws=%d" % (M, K, N, need))
+
+
+@pytest.mark.parametrize("K,N", wl.PREFILL_KN)
+def test_fp8_linear_prefill(K, N):
+    """Fused act_quant + GEMM at M=4096 with heavy-tailed channels: q and s on every
+    element, y on sampled rows (all columns)."""
+    M = wl.PREFILL_M
+    x = wl.heavy_tailed_channels(M, K, seed=40 + K)
+    qw, sw = quantized_weight(N, K, seed=41 + N)
+    y, q, s = fp8bs.fp8_linear(x.cuda(), cuda_codes(qw), cuda_f32(sw), return_quant=True)
+    qa, sa = oracle.act_quant(wl.bf16_bits(x))
+    assert np.array_equal(u8(q), qa)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(sa))
+    rows = sample_rows(M, 12, seed=K + N)
+    y_ref, bnd = oracle.gemm(qa[rows], sa[rows], qw, sw)
+    assert_gemm_close(y[torch.from_numpy(rows).cuda()], y_ref, bnd, "prefill K=%d N=%d" % (K, N))
+
+
+def test_fp8_linear_prefill_ue8m0_ragged():
+    M, K, N = 1000, 7168, 576
+    x = wl.heavy_tailed_channels(M, K, seed=50)
+    qw, sw = quantized_weight(N, K, seed=51, scale_fmt="ue8m0")
+    y = fp8bs.fp8_linear(x.cuda(), cuda_codes(qw), cuda_f32(sw), scale_fmt="ue8m0")
+    qa, sa = oracle.act_quant(wl.bf16_bits(x), scale_fmt="ue8m0")
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "ragged ue8m0")
+
+
+# --------------------------------------------------------------------------
+# grouped (expert-batched) GEMM
+# --------------------------------------------------------------------------
+
+def _grouped_case(counts, N, K, seed):
+    G = len(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    Mt = int(offs[-1])
+    x = wl.normal_with_outliers(max(Mt, 1), K, seed=seed, frac=0.001, factor=20.0)[:Mt]
+    qa, sa = oracle.act_quant(wl.bf16_bits(x))
+    qws, sws = zip(*[quantized_weight(N, K, seed=seed + 1 + g) for g in range(G)])
+    return offs, qa, sa, np.stack(qws), np.stack(sws)
+
+
+def test_grouped_small_ragged():
+    counts = [0, 1, 130, 255, 64, 0, 300]
+    N, K = 384, 256
+    offs, qa, sa, qw, sw = _grouped_case(counts, N, K, seed=60)
+    y = fp8bs.fp8_gemm_grouped(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw),
+                               torch.from_numpy(offs).cuda())
+    for g in range(len(counts)):
+        lo, hi = offs[g], offs[g + 1]
+        if hi == lo:
+            continue
+        y_ref, bnd = oracle.gemm(qa[lo:hi], sa[lo:hi], qw[g], sw[g])
+        assert_gemm_close(y[lo:hi], y_ref, bnd, "group %d" % g)
+
+
+def test_grouped_expert_config_sampled():
+    """32 experts, W_e [2048, 7168], 65536 rows split ~Multinomial(65536, 1/32);
+    every expert checked on rows at its tile edges plus random rows."""
+    counts = wl.expert_counts(wl.EXPERT_TOKENS * wl.EXPERT_TOPK, wl.EXPERTS, seed=70).numpy()
+    N, K = wl.EXPERT_FFN, wl.HIDDEN
+    offs, qa, sa, qw, sw = _grouped_case(counts, N, K, seed=71)
+    y = fp8bs.fp8_gemm_grouped(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw),
+                               torch.from_numpy(offs).cuda())
+    for g in range(len(counts)):
+        lo, hi = int(offs[g]), int(offs[g + 1])
+        rows = lo + sample_rows(hi - lo, 2, seed=g)
+        y_ref, bnd = oracle.gemm(qa[rows], sa[rows], qw[g], sw[g])
+        assert_gemm_close(y[torch.from_numpy(rows).cuda()], y_ref, bnd, "expert %d" % g)
