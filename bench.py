@@ -47,6 +47,10 @@ WORKLOAD = "prefill FP8 linear: act_quant x bf16 [4096,7168] + fp8_gemm W e4m3 [
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+# DRAM bytes (read + write) of one prefill GEMM launch from the ncu capture
+# summarised in profiles/fp8_gemm_prefill_M4096_N18432_K7168.md.  It belongs
+# to the kernel as captured; reset it to None whenever the GEMM kernel changes.
+GEMM_TRAFFIC_BYTES = 169.357056e6 + 128.002048e6
 
 
 def parse_args():
@@ -264,7 +268,8 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
             nbytes = nn * kk + 4 * (-(-nn // 128)) * (kk // 128) + mm * kk + 4 * mm * (kk // 128) + 2 * mm * nn
             parts["decode_M%d_K%d_N%d" % (mm, kk, nn)] = {
                 "us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm,
-                "TFLOP/s": 2 * mm * nn * kk / ms / 1e9, "splitk_workspace": lin.nws}
+                "TFLOP/s": 2 * mm * nn * kk / ms / 1e9, "splitk_workspace": lin.nws,
+                "plan": fp8bs.gemm_plan(mm, nn, kk)}
         del lin
     # prefill shapes: fused act_quant + GEMM per call, and the GEMM alone
     for kk, nn in wl.PREFILL_KN:
@@ -276,6 +281,7 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
             ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm(stream)), 10)
             fl = 2 * wl.PREFILL_M * nn * kk
             parts["prefill_K%d_N%d_%s" % (kk, nn, "ue8m0" if fmt else "none")] = {
+                "plan": fp8bs.gemm_plan(wl.PREFILL_M, nn, kk),
                 "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
                 "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
                 "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
@@ -325,7 +331,7 @@ def cpu_baseline(target_s, impl_steps=None):
     import numpy as np
     import oracle
     from fp8_block_scaled_10_b200 import workloads as wl
-    x = wl.heavy_tailed_channels(256, K, seed=0)
+    x = wl.heavy_tailed_channels(4096, K, seed=0)
     xb = wl.bf16_bits(x)
     w = wl.weight_f32(N, K, seed=1).numpy()
     qw, sw = oracle.weight_quant(w)
@@ -338,7 +344,7 @@ def cpu_baseline(target_s, impl_steps=None):
         return time.perf_counter() - t0
 
     t1 = run(2)
-    rows = int(max(1, min(256, round(2 * target_s / max(t1, 1e-3)))))
+    rows = int(max(1, min(4096, round(2 * target_s / max(t1, 1e-3)))))
     times = [run(rows)] if impl_steps is None else None
     return rows, run, times
 
@@ -421,9 +427,11 @@ def ours(args, dist):
         "gpu_launches": lin.launches_per_step * args.steps,
         "roofline": {"bound": "tensor", "kernel": "fp8_gemm_kernel",
                      "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp8_peak, "traffic": None,
+                     "frac": gemm_tflops / fp8_peak, "traffic": GEMM_TRAFFIC_BYTES,
+                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_note": "%s bf16 burst %.1f TFLOP/s x %.1f (nominal FP8/BF16 dense ratio)"
                                   % (peak_kind, bf16, FP8_OVER_BF16)},
+        "gemm_plan": fp8bs.gemm_plan(M, N, K),
         "kernels_us": {"fp8_gemm": gemm_ms * 1e3, "act_quant": aq_ms * 1e3,
                        "act_quant_GB/s": aq_bytes / (aq_ms * 1e-3) / 1e9},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2,

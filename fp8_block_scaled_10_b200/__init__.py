@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "act_quant", "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
-    "fp8_gemm_grouped", "gemm_workspace_size", "device_error", "lib", "Fp8bsError",
+    "fp8_gemm_grouped", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
     "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -68,6 +68,8 @@ def lib():
         "fp8bs_weight_dequant": (i32, [p, p, i64, i64, i64, p, i32, p]),
         "fp8bs_weight_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
         "fp8bs_gemm_workspace_size": (sz, [i64, i64, i64]),
+        "fp8bs_gemm_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
+        "fp8bs_selftest_quotient": (i32, [p, p, p, i64, p]),
         "fp8bs_fp8_gemm": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
         "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
         "fp8bs_fp8_gemm_grouped": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
@@ -182,6 +184,11 @@ def weight_quant(w, block_size=128, scale_fmt=None):
 def gemm_workspace_size(M, N, K):
     """Bytes of scratch fp8_gemm needs for an M x N x K problem on this device."""
     return int(lib().fp8bs_gemm_workspace_size(M, N, K))
+
+
+def gemm_plan(M, N, K):
+    """The launch plan fp8_gemm uses for an M x N x K problem on this device."""
+    return lib().fp8bs_gemm_plan_string(M, N, K).decode()
 
 
 def _workspace(M, N, K, device):

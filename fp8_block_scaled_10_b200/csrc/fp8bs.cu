@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -42,6 +43,10 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
+  int pair_slots = 0;   // CTA pairs (clusters of two) that can be resident at once
+  // CTA-pair GEMM tiles are correct but measured slower than single-CTA tiles
+  // on B200 so far; FP8BS_GEMM_PAIR=1 lets the planner consider them.
+  bool pair_enabled = false;
 };
 
 std::mutex g_mu;
@@ -56,16 +61,33 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G>
-fp8bs_status setup_gemm_kernel() {
-  using C = gemm::Cfg<BN>;
-  cudaError_t e = cudaFuncSetAttribute(gemm::fp8_gemm_kernel<BN, G>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int BN, bool G, bool PAIR>
+fp8bs_status setup_gemm_kernel(DeviceInfo& d) {
+  using C = gemm::Cfg<BN, PAIR>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * d.sms);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::smem_bytes(G);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+    d.pair_slots = d.pair_slots == 0 ? clusters : std::min(d.pair_slots, clusters);
+  }
   if (C::kSplitRegs) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, gemm::fp8_gemm_kernel<BN, G>);
+    e = cudaFuncGetAttributes(&fa, kernel);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
     const long launch_total = static_cast<long>(fa.numRegs) * C::kThreads;
     const long split_total = 128L * C::kCtrlRegs + 32L * C::kEpiWarps * C::kEpiRegs;
@@ -93,13 +115,21 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
     if (major != 10 || minor != 0)
       return fail(FP8BS_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
                   dev, major, minor);
+    {
+      const char* env = getenv("FP8BS_GEMM_PAIR");
+      d.pair_enabled = env != nullptr && env[0] == '1';
+    }
     e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     fp8bs_status r;
-    if ((r = setup_gemm_kernel<128, false>()) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, false>()) != FP8BS_OK ||
-        (r = setup_gemm_kernel<128, true>()) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, true>()) != FP8BS_OK)
+    if ((r = setup_gemm_kernel<128, false, false>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, false>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, true, false>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, true, false>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, true>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, true>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, true, true>(d)) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, true, true>(d)) != FP8BS_OK)
       return r;
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -142,56 +172,98 @@ int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
 // ---------------------------------------------------------------------------
 struct Plan {
   int bn;
+  bool pair;
   int m_tiles, n_tiles;
   int splits, kb_per_split;
   int units;
+  int grid;   // CTAs (twice the clusters in pair mode)
 };
 
-double wave_efficiency(int64_t units, int sms) {
-  const int64_t waves = (units + sms - 1) / sms;
-  return static_cast<double>(units) / static_cast<double>(waves * sms);
+double wave_efficiency(int64_t units, int slots) {
+  const int64_t waves = (units + slots - 1) / slots;
+  return static_cast<double>(units) / static_cast<double>(waves * slots);
 }
 
-Plan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
+// Chooses tile width, CTA pairing and K split.  The score is the fraction of
+// persistent slots (SMs, or CTA pairs) kept busy over the waves of work
+// units, weighted by what each shape costs beyond its MMAs: a 128-wide tile
+// moves more operand bytes per MMA, a CTA pair moves a third fewer, and each
+// extra split adds a reduction pass over the output.
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d) {
   Plan best{};
   double best_score = -1.0;
   const int kbn = static_cast<int>(K / 128);
-  for (int bn : {256, 128}) {
-    const int m_tiles = static_cast<int>((M + 127) / 128);
-    const int n_tiles = static_cast<int>((N + bn - 1) / bn);
-    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
-    // Split K only when the tiles alone cannot fill the GPU.
-    const int max_split = tiles >= sms ? 1 : std::min(16, std::max(1, kbn / 4));
-    for (int s = 1; s <= max_split; ++s) {
-      const int per = (kbn + s - 1) / s;
-      const int splits = (kbn + per - 1) / per;
-      if (splits != s) continue;
-      const int64_t units = tiles * splits;
-      // Work in units of 128x128x128 MMA blocks, per SM, including idle SMs
-      // in the last wave; narrow tiles and extra splits pay a small overhead
-      // (more A re-reads, a reduction pass).
-      const double eff = wave_efficiency(units, sms);
-      const double overhead = (bn == 128 ? 0.97 : 1.0) * (splits > 1 ? 0.95 - 0.002 * splits : 1.0);
-      const double score = eff * overhead;
-      if (score > best_score + 1e-9) {
-        best_score = score;
-        best = Plan{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units)};
+  for (int pair = 0; pair <= 1; ++pair) {
+    if (pair && (!d.pair_enabled || d.pair_slots <= 0 || M <= 128)) continue;
+    const int slots = pair ? d.pair_slots : d.sms;
+    const int rows = pair ? 256 : 128;
+    for (int bn : {256, 128}) {
+      const int m_tiles = static_cast<int>((M + rows - 1) / rows);
+      const int n_tiles = static_cast<int>((N + bn - 1) / bn);
+      const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+      // Split K only when the tiles alone cannot fill the GPU.
+      const int max_split = tiles >= slots ? 1 : std::min(16, std::max(1, kbn / 4));
+      for (int s = 1; s <= max_split; ++s) {
+        const int per = (kbn + s - 1) / s;
+        const int splits = (kbn + per - 1) / per;
+        if (splits != s) continue;
+        const int64_t units = tiles * splits;
+        const double eff = wave_efficiency(units, slots);
+        // Useful rows per unit when M is smaller than the unit.
+        const double fill = static_cast<double>(std::min<int64_t>(M, rows)) / rows;
+        const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? 0.97 : 1.0);
+        const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
+        const double score = eff * feed * split_cost * (M < rows ? fill + 0.5 * (1 - fill) : 1.0);
+        if (score > best_score + 1e-9) {
+          best_score = score;
+          const int grid_units = static_cast<int>(std::min<int64_t>(units, slots));
+          best = Plan{bn, pair != 0, m_tiles, n_tiles, splits, per, static_cast<int>(units),
+                      pair ? 2 * grid_units : grid_units};
+        }
       }
     }
   }
   return best;
 }
 
+// Rows of one W load box: the per-CTA chunk of one sub-MMA's W rows.
+int w_box_rows(int bn, bool pair) {
+  return bn == 256 ? (pair ? gemm::Cfg<256, true>::kBChunkRows : gemm::Cfg<256, false>::kBChunkRows)
+                   : (pair ? gemm::Cfg<128, true>::kBChunkRows : gemm::Cfg<128, false>::kBChunkRows);
+}
+
 size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
-template <int BN, bool G>
+template <int BN, bool G, bool PAIR>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p,
                         int grid, cudaStream_t st) {
-  gemm::fp8_gemm_kernel<BN, G><<<grid, gemm::Cfg<BN>::kThreads, gemm::Cfg<BN>::smem_bytes(G), st>>>(
-      ta, tw, p);
-  return cudaGetLastError();
+  using C = gemm::Cfg<BN, PAIR>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::smem_bytes(G);
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, gemm::fp8_gemm_kernel<BN, G, PAIR>, ta, tw, p);
+}
+
+template <bool G>
+cudaError_t launch_gemm_any(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tw,
+                            const gemm::Params& p, int grid, cudaStream_t st) {
+  if (pair) return bn == 256 ? launch_gemm<256, G, true>(ta, tw, p, grid, st)
+                             : launch_gemm<128, G, true>(ta, tw, p, grid, st);
+  return bn == 256 ? launch_gemm<256, G, false>(ta, tw, p, grid, st)
+                   : launch_gemm<128, G, false>(ta, tw, p, grid, st);
 }
 
 fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
@@ -216,14 +288,14 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const Plan pl = plan_gemm(M, N, K, info->sms);
+  const Plan pl = plan_gemm(M, N, K, *info);
   const size_t need = plan_workspace(pl, M, N);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
 
   CUtensorMap ta, tw;
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
-  if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, w_box_rows(pl.bn, pl.pair))) != FP8BS_OK) return r;
   gemm::Params p{};
   p.sa = a_s;
   p.sw = w_s;
@@ -240,9 +312,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
   p.groups = 1;
-  const int grid = std::min(pl.units, info->sms);
-  cudaError_t e = pl.bn == 256 ? launch_gemm<256, false>(ta, tw, p, grid, st)
-                               : launch_gemm<128, false>(ta, tw, p, grid, st);
+  cudaError_t e = launch_gemm_any<false>(pl.bn, pl.pair, ta, tw, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
@@ -351,11 +421,12 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
   cudaStream_t st = as_stream(stream);
   const int64_t nbn = (N + 127) / 128;
   const bool bf = y_dtype == FP8BS_DTYPE_BF16;
-  if (N % 16 == 0 && N / 16 <= 0xFFFFFFFFll) {
+  if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
     const uint32_t cpr = static_cast<uint32_t>(N / 16);
-    const int grid = grid_for(M * cpr, kDeqThreads * kDeqUnroll, info->sms * 8);
-    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, cpr, nbn);
-    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, cpr, nbn);
+    const uint32_t total = static_cast<uint32_t>(M * (N / 16));
+    const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 8);
+    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
+    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
   } else {
     const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
     if (bf) weight_dequant_any_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);
@@ -396,12 +467,44 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
   return FP8BS_OK;
 }
 
+fp8bs_status fp8bs_selftest_quotient(const float* x, const float* s, float* q, int64_t n,
+                                     void* stream) {
+  if (n < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
+  if (n == 0) return FP8BS_OK;
+  if (!x || !s || !q) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  quotient_selftest_kernel<<<grid_for(n, 256, info->sms * 8), 256, 0, as_stream(stream)>>>(x, s, q, n);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quotient self-test launch");
+  return FP8BS_OK;
+}
+
 size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;
   int dev;
   DeviceInfo* info;
   if (device_setup(&dev, &info) != FP8BS_OK) return 0;
-  return plan_workspace(plan_gemm(M, N, K, info->sms), M, N);
+  return plan_workspace(plan_gemm(M, N, K, *info), M, N);
+}
+
+const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
+  thread_local char buf[256];
+  int dev;
+  DeviceInfo* info;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || device_setup(&dev, &info) != FP8BS_OK) {
+    snprintf(buf, sizeof(buf), "none");
+    return buf;
+  }
+  const Plan pl = plan_gemm(M, N, K, *info);
+  snprintf(buf, sizeof(buf),
+           "bn=%d pair=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d "
+           "sms=%d pair_slots=%d",
+           pl.bn, pl.pair ? 1 : 0, pl.m_tiles, pl.n_tiles, pl.splits, pl.kb_per_split, pl.units,
+           pl.grid, info->sms, info->pair_slots);
+  return buf;
 }
 
 fp8bs_status fp8bs_fp8_gemm(const uint8_t* a, const float* a_s, const uint8_t* w,
@@ -438,9 +541,11 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
   const int bn = N >= 256 ? 256 : 128;
+  // CTA pairs when the groups are large enough on average to fill 256-row units.
+  const bool pair = info->pair_enabled && info->pair_slots > 0 && M_total >= 256 * G;
   CUtensorMap ta, tw;
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
-  if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, G * N, K, w_box_rows(bn, pair))) != FP8BS_OK) return r;
   gemm::Params p{};
   p.sa = a_s;
   p.sw = w_s;
@@ -458,10 +563,12 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   p.num_units = 0;
   p.groups = static_cast<int>(G);
   // Units are only known on the device; an upper bound sizes the grid.
-  const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
-  const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
-  cudaError_t e = bn == 256 ? launch_gemm<256, true>(ta, tw, p, grid, as_stream(stream))
-                            : launch_gemm<128, true>(ta, tw, p, grid, as_stream(stream));
+  const int rows = pair ? 256 : 128;
+  const int64_t max_units = ((M_total + rows - 1) / rows + G) * p.n_tiles;
+  const int slots = pair ? info->pair_slots : info->sms;
+  const int grid_units = static_cast<int>(std::min<int64_t>(max_units, slots));
+  cudaError_t e = launch_gemm_any<true>(bn, pair, ta, tw, p, pair ? 2 * grid_units : grid_units,
+                                        as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
   return FP8BS_OK;
 }

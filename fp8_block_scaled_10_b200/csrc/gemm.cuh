@@ -16,12 +16,22 @@
 // a_s[m, kb] * w_s[nb, kb], while the tensor core fills the other buffer.
 //
 // Roles (persistent CTAs, one per SM, walking work units in a fixed order):
-//   warp 0     TMA producer: A tile [128 x 128] and W tile [BN x 128] per K
-//              block into a ring of shared-memory stages (128B swizzle).
+//   warp 0     TMA producer: A tile [128 x 128] and W tile into a ring of
+//              shared-memory stages (128B swizzle).
 //   warp 1     owns the TMEM allocation; one lane issues the MMAs.
-//   epilogue   warps kFirstEpiWarp..: warp w reads TMEM lanes 32*(w%4)..+31
-//              (one output row per thread) and 128 columns (column group
-//              (w - kFirstEpiWarp) / 4).
+//   epilogue   8 warps from kFirstEpiWarp: warp w reads TMEM lanes
+//              32*(w%4)..+31 (one output row per thread) and BN/2 columns
+//              (column half (w - kFirstEpiWarp) / 4).  Loads of the next
+//              32-column chunk overlap the FMAs of the current one.
+// Pair mode (PAIR): two CTAs of a cluster share one tcgen05.mma.cta_group::2
+// of M = 256.  Each CTA loads its own 128 rows of A and its own half of the W
+// tile (BN/2 rows), so each SM moves a third less operand data per MMA than
+// a single CTA with a 128 x BN tile.  The leader (even) CTA issues the MMAs;
+// both CTAs' loads complete on the leader's full barrier, the leader's commits
+// arrive on both CTAs' barriers, and both CTAs' epilogues release the TMEM
+// buffer on the leader's barrier.  Each CTA holds its own 128 rows of the
+// accumulator in its own TMEM.
+//
 // A work unit is (m tile, n tile, K split).  With one split the epilogue
 // writes bf16; with several it writes FP32 partials that a reduction kernel
 // sums.  Grouped mode (experts) walks (expert, m tile, n tile) units whose
@@ -38,8 +48,8 @@
 namespace fp8bs {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BK = 128;
+constexpr int BM = 128;      // rows of A per CTA
+constexpr int BK = 128;      // one K block per pipeline stage
 constexpr int kMaxGroups = 1024;
 
 struct Params {
@@ -52,7 +62,7 @@ struct Params {
   int N;
   int kbn;                  // K / 128
   int nbn;                  // cdiv(N, 128)
-  int m_tiles;              // dense mode
+  int m_tiles;              // dense mode: tiles of kUnitRows rows
   int n_tiles;
   int splits;
   int kb_per_split;
@@ -60,28 +70,49 @@ struct Params {
   int groups;               // grouped mode
 };
 
-template <int BN>
+template <int BN, bool PAIR>
 struct Cfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
-  static constexpr int kEpiWarps = BN / 32;
+  static constexpr int kUnitRows = PAIR ? 2 * BM : BM;   // rows of one work unit
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;      // W rows loaded per CTA
+  static constexpr int kABytes = BM * BK;
+  static constexpr int kBBytes = kBRows * BK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (6 * 32768) / kStageBytes;
+  // Two epilogue warpgroups: each covers all 128 TMEM lanes (one warp per
+  // 32-lane quadrant) and half of the tile's columns.
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kColsPerWarp = BN / 2;
+  static constexpr int kChunks = kColsPerWarp / 32;
   // BN = 256: warps 0-3 form a control warpgroup that hands registers to the
-  // two epilogue warpgroups (setmaxnreg); BN = 128: warps 0-1 control, 2-5
-  // epilogue, and every thread can hold the 128 accumulators at launch.
+  // two epilogue warpgroups (setmaxnreg); BN = 128: warps 0-1 control, 2-9
+  // epilogue, and every thread can hold its 64 accumulators at launch.
   static constexpr int kFirstEpiWarp = (BN == 256) ? 4 : 2;
   static constexpr bool kSplitRegs = (BN == 256);
-  static constexpr int kCtrlRegs = 40;
-  static constexpr int kEpiRegs = 232;
+  static constexpr int kCtrlRegs = 56;
+  static constexpr int kEpiRegs = 224;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-  static constexpr int kABytes = BM * BK;
-  static constexpr int kBBytes = BN * BK;
-  static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
+  // In pair mode with BN = 256 each K block's MMA is issued as two sub-MMAs of
+  // N = 128, each into its own TMEM sub-buffer with its own full/empty
+  // barrier pair, so the epilogue warps of column half g can drain sub-buffer
+  // g while the tensor core still works on the other half; each sub-MMA takes
+  // 64 rows of W from each CTA, so a CTA loads two chunks of 64 rows per
+  // stage.  (A single CTA keeps one N = BN MMA: two N = 128 MMAs would read
+  // the A tile from shared memory twice.)
+  static constexpr int kSplitN = (PAIR && BN == 256) ? 2 : 1;
+  static constexpr int kSubN = BN / kSplitN;
+  static constexpr int kBChunkRows = PAIR ? kSubN / 2 : kSubN;
+  static constexpr int kBChunkBytes = kBChunkRows * BK;
+  static constexpr int kSubBuffers = 2 * kSplitN;
   static constexpr int kCtrlBytes = 256;
   // grouped mode: per-group m-tile prefix (int) and clamped [lo, hi) rows (int64)
   static constexpr int kGroupBytes = 8 * 2 * kMaxGroups + 4 * (kMaxGroups + 1);
   static constexpr int smem_bytes(bool grouped) {
     return kStages * kStageBytes + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1024;
   }
+  // Arrivals that release one TMEM sub-buffer: the epilogue warps that read
+  // it, in both CTAs in pair mode.
+  static constexpr int kTmemReleaseCount = (kEpiWarps / kSplitN) * (PAIR ? 2 : 1);
 };
 
 // Control block at the end of the tile ring.
@@ -89,8 +120,8 @@ template <int kStages>
 struct Ctrl {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[4];     // [buffer * kSplitN + half]
+  uint64_t tempty[4];
   uint64_t flush;
   uint32_t tmem_base;
   int abort_flag;
@@ -98,7 +129,7 @@ struct Ctrl {
 };
 
 struct Unit {
-  int64_t row0;      // first A/y row of the tile
+  int64_t row0;      // first A/y row of the unit (of the pair in pair mode)
   int64_t row_end;   // rows >= row_end are not stored
   int64_t w_row0;    // first W row (grouped: expert * N + n0)
   int group;
@@ -109,6 +140,7 @@ struct Unit {
 
 // Dense units: m tile fastest, so the CTAs running at the same time share W
 // tiles (and sweep all of A, which stays in L2).
+template <int kUnitRows>
 __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   Unit t;
   const int m_tile = u % p.m_tiles;
@@ -116,7 +148,7 @@ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   t.split = rest % p.splits;
   t.n_tile = rest / p.splits;
   t.group = 0;
-  t.row0 = static_cast<int64_t>(m_tile) * BM;
+  t.row0 = static_cast<int64_t>(m_tile) * kUnitRows;
   t.row_end = p.M;
   t.kb0 = t.split * p.kb_per_split;
   t.kb1 = min(p.kbn, t.kb0 + p.kb_per_split);
@@ -127,6 +159,7 @@ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
 // at the same time work on one or two experts and read each W_e once.
 // tile_prefix[g] is the number of m tiles of groups < g; rows[2g], rows[2g+1]
 // are group g's clamped row range [lo, hi).
+template <int kUnitRows>
 __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix,
                                              const int64_t* rows, int u) {
   Unit t;
@@ -138,7 +171,7 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
     if (tile_prefix[mid] <= gm) a = mid; else b = mid;
   }
   t.group = a;
-  t.row0 = rows[2 * a] + static_cast<int64_t>(gm - tile_prefix[a]) * BM;
+  t.row0 = rows[2 * a] + static_cast<int64_t>(gm - tile_prefix[a]) * kUnitRows;
   t.row_end = rows[2 * a + 1];
   t.split = 0;
   t.kb0 = 0;
@@ -146,11 +179,11 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   return t;
 }
 
-template <int BN, bool GROUPED>
-__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
+template <int BN, bool GROUPED, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w, const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -169,15 +202,18 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;   // 0 = leader
+  const int unit_start = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kSubBuffers; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::kEpiWarps);
+      mbar_init(&tempty[b], C::kTmemReleaseCount);
     }
     mbar_init(flush, 1);
     *abort_flag = 0;
@@ -188,8 +224,13 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     tma_prefetch_descriptor(&tmap_w);
   }
   if (warp == 1) {
-    tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(&ctrl->tmem_base, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (GROUPED) {
     // Clamp the device offsets to [0, M], count each group's m tiles and form
@@ -203,7 +244,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
           int64_t lo = p.m_offsets[g], hi = p.m_offsets[g + 1];
           lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
           hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
-          tiles = static_cast<int>((hi - lo + BM - 1) / BM);
+          tiles = static_cast<int>((hi - lo + C::kUnitRows - 1) / C::kUnitRows);
           group_rows[2 * g] = lo;
           group_rows[2 * g + 1] = hi;
         }
@@ -225,7 +266,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     ctrl->num_units = p.num_units;
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctrl->tmem_base;
   const int num_units = ctrl->num_units;
@@ -233,10 +274,10 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   auto unit_of = [&](int u) -> Unit {
     Unit t;
     if (GROUPED) {
-      t = grouped_unit(p, tile_prefix, group_rows, u);
+      t = grouped_unit<C::kUnitRows>(p, tile_prefix, group_rows, u);
       t.w_row0 = static_cast<int64_t>(t.group) * p.N + static_cast<int64_t>(t.n_tile) * BN;
     } else {
-      t = dense_unit(p, u);
+      t = dense_unit<C::kUnitRows>(p, u);
       t.w_row0 = static_cast<int64_t>(t.n_tile) * BN;
     }
     return t;
@@ -251,15 +292,32 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0;       // stages with a TMA load issued
       uint32_t armed_phase = 0; // parity each armed stage completes
-      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      for (int u = unit_start; u < num_units; u += unit_step) {
         const Unit t = unit_of(u);
+        const int32_t a_row = static_cast<int32_t>(t.row0 + rank * BM);
+        // W rows of chunk h: sub-tile h (kSubN rows) and, in pair mode, this
+        // CTA's half of it.
+        const int32_t b_row = static_cast<int32_t>(t.w_row0 + rank * C::kBChunkRows);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.row0));
-          tma_load_2d(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.w_row0));
+          if (PAIR) {
+            // Both CTAs' bytes complete on the leader's full barrier, which the
+            // leader alone arms.
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+            const uint32_t bar = map_to_rank(&full[stage], 0);
+            tma_load_2d_pair(a_tiles + stage * C::kABytes, &tmap_a, bar, kb * BK, a_row);
+#pragma unroll
+            for (int h = 0; h < C::kSplitN; ++h)
+              tma_load_2d_pair(b_tiles + stage * C::kBBytes + h * C::kBChunkBytes, &tmap_w, bar,
+                               kb * BK, b_row + h * C::kSubN);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK, a_row);
+#pragma unroll
+            for (int h = 0; h < C::kSplitN; ++h)
+              tma_load_2d(b_tiles + stage * C::kBBytes + h * C::kBChunkBytes, &tmap_w,
+                          &full[stage], kb * BK, b_row + h * C::kSubN);
+          }
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) {
@@ -269,37 +327,47 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         }
       }
     producer_done:
-      if (*abort_flag) {
-        // Let every load in flight land before the CTA exits.
+      if (*abort_flag && (!PAIR || rank == 0)) {
+        // Let every load in flight land before the CTA exits (in pair mode the
+        // leader's full barriers count the peer's loads too).
         for (int s = 0; s < C::kStages; ++s)
-          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
+          if (armed & (1u << s)) mbar_wait<PAIR>(&full[s], (armed_phase >> s) & 1u, nullptr);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+    if (lane == 0 && (!PAIR || rank == 0)) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(PAIR ? 2 * BM : BM, C::kSubN);
       int stage = 0;
       uint32_t phase = 0;
       int tb = 0;
       uint32_t tphase = 0;
-      for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      for (int u = unit_start; u < num_units; u += unit_step) {
         const Unit t = unit_of(u);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
-          tc_fence_after();
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto mma_done;
+          if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) goto mma_done;
           tc_fence_after();
           const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
           const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            mma_f8f6f4(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
-                       smem_desc_k_sw128(b_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
-          mma_commit(&empty[stage]);
-          mma_commit(&tfull[tb]);
+          for (int h = 0; h < C::kSplitN; ++h) {
+            const int sb = tb * C::kSplitN + h;
+            if (!mbar_wait<PAIR>(&tempty[sb], tphase ^ 1u, abort_flag)) goto mma_done;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN + h * C::kSubN);
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k) {
+              const uint64_t ad = smem_desc_k_sw128(a_addr + 32 * k);
+              const uint64_t bd = smem_desc_k_sw128(b_addr + h * C::kBChunkBytes + 32 * k);
+              if (PAIR) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+              else mma_f8f6f4(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+            }
+            if (PAIR) mma_commit_pair_mask(&tfull[sb], 0x3);
+            else mma_commit(&tfull[sb]);
+          }
+          if (PAIR) mma_commit_pair_mask(&empty[stage], 0x3);
+          else mma_commit(&empty[stage]);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -310,7 +378,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       }
     mma_done:
       // Every MMA issued must finish before the TMEM columns are released.
-      mma_commit(flush);
+      if (PAIR) mma_commit_pair(flush); else mma_commit(flush);
       mbar_wait(flush, 0, nullptr);
     }
     __syncwarp();
@@ -320,86 +388,109 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int e = warp - C::kFirstEpiWarp;
     const int quad = warp & 3;
-    const int g = e >> 2;
-    const int row_in_tile = quad * 32 + lane;
+    const int g = e >> 2;                       // column half
+    constexpr int CPW = C::kColsPerWarp;
+    constexpr int NCH = C::kChunks;
+    const int row_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const bool vec_store = (p.N % 8) == 0;
+    // This warp's sub-buffer within each TMEM buffer (both halves are the same
+    // sub-buffer when the MMA is not split).
+    const int half = (g * C::kSplitN) >> 1;
+    const uint32_t tempty_leader0 = PAIR ? map_to_rank(&tempty[half], 0) : 0u;
+    const uint32_t tempty_leader1 = PAIR ? map_to_rank(&tempty[C::kSplitN + half], 0) : 0u;
     int tb = 0;
     uint32_t tphase = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+    for (int u = unit_start; u < num_units; u += unit_step) {
       const Unit t = unit_of(u);
       const int64_t row = t.row0 + row_in_tile;
       const bool row_ok = row < t.row_end;
-      const int nb = (t.n_tile * BN) / 128 + g;
+      const int nb = (t.n_tile * BN + g * CPW) / 128;
       const bool nb_ok = nb < p.nbn;
       const float* sa_row = p.sa + (row_ok ? row : 0) * static_cast<int64_t>(p.kbn);
       const float* sw_row =
           p.sw + (static_cast<int64_t>(t.group) * p.nbn + (nb_ok ? nb : 0)) * p.kbn;
-      float acc[128];
+      float2 acc[CPW / 2];
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < CPW / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
       float sa_next = row_ok ? __ldg(sa_row + t.kb0) : 0.0f;
       float sw_next = nb_ok ? __ldg(sw_row + t.kb0) : 0.0f;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         const float scale = sa_next * sw_next;
+        const float2 scale2 = make_float2(scale, scale);
         if (kb + 1 < t.kb1) {
           sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
           sw_next = nb_ok ? __ldg(sw_row + kb + 1) : 0.0f;
         }
-        const bool ok = mbar_wait(&tfull[tb], tphase, abort_flag);
+        const bool ok = mbar_wait<PAIR>(&tfull[tb * C::kSplitN + half], tphase, abort_flag);
         if (!__all_sync(0xFFFFFFFFu, ok)) goto epilogue_done;
         tc_fence_after();
+        const uint32_t col_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
+        // Two register buffers: the load of chunk c+1 is in flight while the
+        // FMAs of chunk c run.
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(col_addr, va);
+        tmem_ld_wait(va);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(tb * BN + g * 128 + c * 32), v);
-          tmem_ld_wait();
-          if (c == 3) {
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t(&cur)[32] = (c & 1) ? vb : va;
+          uint32_t(&nxt)[32] = (c & 1) ? va : vb;
+          if (c + 1 < NCH) tmem_ld_32x32b_x32(col_addr + 32 * (c + 1), nxt);
+          if (c + 1 == NCH) {
+            // Every load of this buffer has completed: hand it back to the MMA.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[tb]);
+            if (lane == 0) {
+              if (PAIR) mbar_arrive_cluster(tb ? tempty_leader1 : tempty_leader0);
+              else mbar_arrive(&tempty[tb * C::kSplitN + half]);
+            }
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[c * 32 + j] = fmaf(__uint_as_float(v[j]), scale, acc[c * 32 + j]);
+          for (int j = 0; j < 16; ++j)
+            acc[c * 16 + j] = __ffma2_rn(
+                make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), scale2,
+                acc[c * 16 + j]);
+          if (c + 1 < NCH) tmem_ld_wait(nxt);
         }
         tb ^= 1;
         if (tb == 0) tphase ^= 1u;
       }
       if (row_ok) {
-        const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * 128;
+        const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
         if (p.splits == 1) {
           __nv_bfloat16* yrow = p.y + row * p.N;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < CPW / 8; ++c) {
             const int64_t col = col0 + c * 8;
             if (vec_store && col + 8 <= p.N) {
               uint32_t h[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 b2 =
-                    __floats2bfloat162_rn(acc[c * 8 + 2 * j], acc[c * 8 + 2 * j + 1]);
+                __nv_bfloat162 b2 = __float22bfloat162_rn(acc[c * 4 + j]);
                 h[j] = *reinterpret_cast<uint32_t*>(&b2);
               }
               *reinterpret_cast<uint4*>(yrow + col) = make_uint4(h[0], h[1], h[2], h[3]);
             } else {
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                if (col + j < p.N) yrow[col + j] = __float2bfloat16_rn(acc[c * 8 + j]);
+              for (int j = 0; j < 8; ++j) {
+                const float v = (j & 1) ? acc[c * 4 + j / 2].y : acc[c * 4 + j / 2].x;
+                if (col + j < p.N) yrow[col + j] = __float2bfloat16_rn(v);
+              }
             }
           }
         } else {
           float* wrow = p.ws + (static_cast<int64_t>(t.split) * p.M + row) * p.N;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < CPW / 4; ++c) {
             const int64_t col = col0 + c * 4;
+            const float2 lo = acc[2 * c], hi = acc[2 * c + 1];
             if ((p.N % 4) == 0 && col + 4 <= p.N) {
-              *reinterpret_cast<float4*>(wrow + col) =
-                  make_float4(acc[c * 4], acc[c * 4 + 1], acc[c * 4 + 2], acc[c * 4 + 3]);
+              *reinterpret_cast<float4*>(wrow + col) = make_float4(lo.x, lo.y, hi.x, hi.y);
             } else {
+              const float v4[4] = {lo.x, lo.y, hi.x, hi.y};
 #pragma unroll
               for (int j = 0; j < 4; ++j)
-                if (col + j < p.N) wrow[col + j] = acc[c * 4 + j];
+                if (col + j < p.N) wrow[col + j] = v4[j];
             }
           }
         }
@@ -410,9 +501,13 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // In pair mode neither CTA may release TMEM or exit while the other can
+  // still touch its shared memory, barriers or TMEM.
+  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

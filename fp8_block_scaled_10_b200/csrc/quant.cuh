@@ -16,6 +16,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -46,41 +47,59 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
       __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// True when fl32(x/s) might round to a different e4m3 code than t = x * r,
-// r = RN(1/s).  t is within 1.5 * 2^-23 |x/s| of x/s (two roundings of
-// relative size <= 2^-24), and fl32(x/s) within half an ulp of it, so the two
-// fp32 values are at most 3 ulps apart.  e4m3 rounding decisions for
-// 2^-6 <= |t| < 512 sit where the 20 bits below e4m3's 3-bit fraction equal
-// 0x80000 (the halfway point); any t within 4 ulps of such a pattern, and
-// any 0 < |t| < 2^-6 (the e4m3 subnormal range), takes the exact division
-// instead.  t == 0 needs nothing: then x == 0 and x / s is that same zero.
-__device__ __forceinline__ bool near_e4m3_midpoint(float t) {
-  const uint32_t u = __float_as_uint(t) & 0x7FFFFFFFu;
-  return (u - 1u < 0x3C7FFFFFu) || (((u & 0x000FFFFFu) - 0x0007FFFCu) < 9u);
+// Correctly rounded fp32 quotient x / s of two pairs sharing one divisor,
+// from r = RN(1/s) by Markstein's division correction (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with r within half an ulp of
+// 1/s and q within one ulp of x/s, the residual e = x - q*s is exact under an
+// FMA and RN(q + e*r) is the correctly rounded quotient.  The first estimate
+// q0 = RN(x*r) can be up to two ulps off, so one correction step brings it
+// within an ulp and a second one applies the theorem.  ns = -s.  Zeros keep
+// their sign through a final copysign; quotients small enough to underflow
+// fp32 all encode to a signed e4m3 zero, so the no-underflow premise does not
+// matter for the codes.
+__device__ __forceinline__ float2 quotient2(float2 x, float2 r, float2 ns) {
+  float2 q = __fmul2_rn(x, r);
+  q = __ffma2_rn(__ffma2_rn(q, ns, x), r, q);
+  q = __ffma2_rn(__ffma2_rn(q, ns, x), r, q);
+  q.x = __uint_as_float((__float_as_uint(q.x) & 0x7FFFFFFFu) | (__float_as_uint(x.x) & 0x80000000u));
+  q.y = __uint_as_float((__float_as_uint(q.y) & 0x7FFFFFFFu) | (__float_as_uint(x.y) & 0x80000000u));
+  return q;
 }
 
 // Quantizes 8 values of one block and packs the codes (element 0 in the low
 // byte).  For ue8m0, r = 1/s is an exact power of two, so x * r is exactly
-// the correctly rounded x / s.
+// the correctly rounded x / s; otherwise the quotient comes from quotient2.
 template <bool UE8M0>
 __device__ __forceinline__ uint2 quantize8(const float (&v)[8], float s, float r) {
   float t[8];
+  if (UE8M0) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) t[j] = v[j] * r;
-  if (!UE8M0) {
-    uint32_t mask = 0;
+    for (int j = 0; j < 8; ++j) t[j] = v[j] * r;
+  } else {
+    const float2 r2 = make_float2(r, r), ns2 = make_float2(-s, -s);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) mask |= static_cast<uint32_t>(near_e4m3_midpoint(t[j])) << j;
-    if (mask) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (mask & (1u << j)) t[j] = __fdiv_rn(v[j], s);
+    for (int j = 0; j < 4; ++j) {
+      const float2 q = quotient2(make_float2(v[2 * j], v[2 * j + 1]), r2, ns2);
+      t[2 * j] = q.x;
+      t[2 * j + 1] = q.y;
     }
   }
   uint2 out;
   out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
   out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
   return out;
+}
+
+// Self-test kernel: q[i] = x[i] / s[i] through quotient2.
+__global__ void quotient_selftest_kernel(const float* __restrict__ x, const float* __restrict__ s,
+                                         float* __restrict__ q, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    const float sc = s[i];
+    const float2 r = make_float2(__frcp_rn(sc), 0.0f);
+    q[i] = quotient2(make_float2(x[i], 0.0f), r, make_float2(-sc, -1.0f)).x;
+  }
 }
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
@@ -176,26 +195,26 @@ constexpr int kDeqThreads = 256;
 constexpr int kDeqUnroll = 2;
 
 // Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row;
-// all 16 share one block scale because 16 divides 128.
+// all 16 share one block scale because 16 divides 128.  Chunk indices fit in
+// 32 bits (the host checks M * N / 16 < 2^32).
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
-                          void* __restrict__ y, int64_t M, uint32_t chunks_per_row,
+                          void* __restrict__ y, uint32_t total_chunks, uint32_t chunks_per_row,
                           int64_t nbn) {
-  const int64_t total = M * static_cast<int64_t>(chunks_per_row);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kDeqThreads * kDeqUnroll;
-  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDeqThreads * kDeqUnroll + threadIdx.x;
-       c0 < total; c0 += stride) {
+  const uint32_t stride = gridDim.x * kDeqThreads * kDeqUnroll;
+  for (uint32_t c0 = blockIdx.x * kDeqThreads * kDeqUnroll + threadIdx.x; c0 < total_chunks;
+       c0 += stride) {
     uint4 raw[kDeqUnroll];
     float sc[kDeqUnroll];
     int64_t off[kDeqUnroll];
 #pragma unroll
     for (int u = 0; u < kDeqUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(u) * kDeqThreads;
-      if (c < total) {
-        const int64_t row = c / chunks_per_row;
-        const int64_t col = (c - row * chunks_per_row) * 16;
-        off[u] = row * static_cast<int64_t>(chunks_per_row) * 16 + col;
+      const uint32_t c = c0 + u * kDeqThreads;
+      if (c < total_chunks) {
+        const uint32_t row = c / chunks_per_row;
+        const uint32_t col = (c - row * chunks_per_row) * 16;
+        off[u] = static_cast<int64_t>(c) * 16;
         raw[u] = __ldcs(reinterpret_cast<const uint4*>(q + off[u]));
         sc[u] = __ldg(s + (row >> 7) * nbn + (col >> 7));
       } else {
@@ -206,14 +225,17 @@ __global__ void __launch_bounds__(kDeqThreads)
     for (int u = 0; u < kDeqUnroll; ++u) {
       if (off[u] < 0) continue;
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      float v[16];
+      float2 v[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = e4m3_value((w[j >> 2] >> (8 * (j & 3))) & 0xFFu) * sc[u];
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t pair = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        v[j] = make_float2(e4m3_value(pair & 0xFFu) * sc[u], e4m3_value(pair >> 8) * sc[u]);
+      }
       if (OUT_BF16) {
         uint32_t h[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          __nv_bfloat162 b2 = __float22bfloat162_rn(v[j]);
           h[j] = *reinterpret_cast<uint32_t*>(&b2);
         }
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + off[u]);
@@ -223,7 +245,7 @@ __global__ void __launch_bounds__(kDeqThreads)
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + off[u]);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          __stcs(dst + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          __stcs(dst + j, make_float4(v[2 * j].x, v[2 * j].y, v[2 * j + 1].x, v[2 * j + 1].y));
       }
     }
   }

@@ -17,6 +17,9 @@
  * scratch space take it from a caller-provided workspace whose size the
  * matching *_workspace_size() function returns.
  *
+ * Environment: FP8BS_GEMM_PAIR=1 lets the GEMM planner use CTA-pair tiles
+ * (tcgen05.mma.cta_group::2); they are off by default.
+ *
  * Sources of the operations (page title, then section):
  *  [ACT] "Understanding Dynamic and Static Activation Quantization Schemes in
  *        DeepSeek-V3", "How Dynamic Activation Quantization Works";
@@ -152,6 +155,23 @@ FP8BS_API fp8bs_status fp8bs_weight_quant(const void *w, fp8bs_dtype w_dtype, in
  * 1e-3 sum_k |a_hat_k w_hat_k| of the exact value y_ref.
  */
 FP8BS_API size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Self-test of the division act_quant uses for scale_fmt NONE: q[i] =
+ * x[i] / s[i] by Markstein's division correction from RN(1/s).  q[i] is the
+ * correctly rounded fp32 quotient whenever |x[i]| and |x[i]/s[i]| are at
+ * least 2^-100 (nothing in the correction underflows); below that it may be
+ * off by ulps of a value far under the smallest e4m3 step, which rounds to
+ * the same e4m3 code.  x, s, q are device fp32 arrays of n elements, s[i] a
+ * positive normal number.  For verification only.
+ */
+FP8BS_API fp8bs_status fp8bs_selftest_quotient(const float *x, const float *s, float *q, int64_t n,
+                                               void *stream);
+
+/* Launch plan fp8_gemm would use for an M x N x K problem on the current
+ * device (tile width, CTA pairing, K split, work units, grid), as a
+ * NUL-terminated string in thread-local storage; for logs and benchmarks. */
+FP8BS_API const char *fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K);
 
 FP8BS_API fp8bs_status fp8bs_fp8_gemm(const uint8_t *a, const float *a_s, const uint8_t *w,
                             const float *w_s, int64_t M, int64_t N, int64_t K, uint16_t *y,

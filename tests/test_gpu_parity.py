@@ -322,3 +322,50 @@ def test_grouped_expert_config_sampled():
         rows = lo + sample_rows(hi - lo, 2, seed=g)
         y_ref, bnd = oracle.gemm(qa[rows], sa[rows], qw[g], sw[g])
         assert_gemm_close(y[torch.from_numpy(rows).cuda()], y_ref, bnd, "expert %d" % g)
+
+
+# --------------------------------------------------------------------------
+# the division act_quant uses (scale_fmt None) against IEEE fp32 division
+# --------------------------------------------------------------------------
+
+def _adversarial_quotient_inputs(n, seed):
+    rng = np.random.default_rng(seed)
+    # x: bf16-like (8 significant bits), full fp32, near binade edges, tiny, zeros
+    xb = rng.normal(0, 1, n).astype(np.float32)
+    xb = (xb.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    xf = (rng.normal(0, 1, n) * np.exp2(rng.uniform(-40, 40, n))).astype(np.float32)
+    edge = np.exp2(rng.integers(-30, 30, n)).astype(np.float32)
+    edge = (edge.view(np.uint32) + rng.integers(-3, 4, n).astype(np.uint32)).view(np.float32)
+    tiny = (rng.normal(0, 1, n) * 1e-38).astype(np.float32)
+    x = np.concatenate([xb, xf, edge, tiny, np.float32([0.0, -0.0, 1.0, -1.0])])
+    # s: a/448 for bf16 a (what act_quant divides by), random, all-ones significands, powers of 2
+    a = np.abs(rng.normal(0, 10, len(x))).astype(np.float32) + np.float32(1e-4)
+    a = (a.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    s1 = (a / np.float32(448.0)).astype(np.float32)
+    s2 = np.exp2(rng.uniform(-22, 20, len(x))).astype(np.float32)
+    s3 = ((rng.integers(100, 150, len(x)).astype(np.uint32) << 23) | np.uint32(0x7FFFFF)).view(np.float32)
+    s4 = np.exp2(rng.integers(-22, 20, len(x)).astype(np.float32))
+    pick = rng.integers(0, 4, len(x))
+    s = np.choose(pick, [s1, s2, s3, s4]).astype(np.float32)
+    return x, s
+
+
+def test_quotient_matches_ieee_division():
+    x, s = _adversarial_quotient_inputs(10_000_000, seed=90)
+    ref = (x / s).astype(np.float32)            # numpy: IEEE fp32 division on the CPU
+    xt, st = cuda_f32(x), cuda_f32(s)
+    q = torch.empty_like(xt)
+    L = fp8bs.lib()
+    st_code = L.fp8bs_selftest_quotient(ctypes.c_void_p(xt.data_ptr()), ctypes.c_void_p(st.data_ptr()),
+                                        ctypes.c_void_p(q.data_ptr()), x.size,
+                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st_code == fp8bs.OK
+    got = q.cpu().numpy()
+    # Markstein's correction is exact while nothing underflows: compare the
+    # fp32 quotient bitwise wherever numerator and quotient are >= 2^-100 ...
+    big = (np.abs(x) >= np.float32(2.0 ** -100)) & (np.abs(ref) >= np.float32(2.0 ** -100))
+    bad = big & (f32bits(got) != f32bits(ref))
+    assert not bad.any(), (x[bad][:5], s[bad][:5], got[bad][:5], ref[bad][:5])
+    assert big.mean() > 0.7
+    # ... and everywhere, the e4m3 code act_quant derives from it
+    assert np.array_equal(oracle.e4m3_encode_array(got), oracle.e4m3_encode_array(ref))
