@@ -513,6 +513,59 @@ fp8bs_status fp8bs_fp8_gemm(const uint8_t* a, const float* a_s, const uint8_t* w
   return run_gemm(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream));
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fp8_gemm without a caller workspace: the split-K partials live in this
+// file-scope device array, which every GPU that loads the library holds
+// until the process exits.  Host code must not pass the array's name to a
+// kernel (on the host it is only a stand-in symbol); the device address is
+// looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+namespace {
+static __device__ __align__(256) float g_static_scratch[FP8BS_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[fp8bs::kMaxDevices] = {};
+
+fp8bs_status static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fp8bs::cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= fp8bs::kMaxDevices)
+    return fp8bs::fail(FP8BS_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fp8bs::cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                              "cudaGetSymbolAddress(static scratch)");
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return FP8BS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                           const float* w_s, int64_t M, int64_t N, int64_t K,
+                                           uint16_t* y, void* stream) {
+  const size_t need = fp8bs_gemm_workspace_size(M, N, K);
+  if (need > FP8BS_STATIC_SCRATCH_BYTES)
+    return fp8bs::fail(FP8BS_ERR_WORKSPACE,
+                       "M=%lld N=%lld K=%lld needs %zu bytes of split-K scratch; the static "
+                       "scratch holds %zu bytes (use fp8bs_fp8_gemm with a workspace)",
+                       (long long)M, (long long)N, (long long)K, need,
+                       (size_t)FP8BS_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  const fp8bs_status r = static_scratch_address(&scratch);
+  if (r != FP8BS_OK) return r;
+  return fp8bs_fp8_gemm(a, a_s, w, w_s, M, N, K, y, scratch, FP8BS_STATIC_SCRATCH_BYTES, stream);
+}
+
 fp8bs_status fp8bs_fp8_linear(const uint16_t* x, int64_t M, int64_t K, fp8bs_scale_fmt fmt,
                               const uint8_t* w, const float* w_s, int64_t N, uint16_t* y,
                               uint8_t* q, float* s, void* workspace, size_t workspace_bytes,

@@ -178,6 +178,41 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm(const uint8_t *a, const float *a_s, const 
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * fp8_gemm for callers that cannot allocate device memory.  (The pages have
+ * no counterpart: this entry point is an addition for deployment.)
+ *
+ * Some callers cannot call cudaMalloc at the time of the call, or cannot own
+ * a scratch buffer at all: for example an inference server that reserves its
+ * whole device memory budget at start-up and forbids later allocations, a
+ * plugin inside a host framework that owns the allocator, or a plain C caller
+ * that has no allocator for a workspace.  This entry point computes exactly
+ * what fp8bs_fp8_gemm computes, and allocates nothing: the split-K partials
+ * that fp8bs_fp8_gemm would keep in the caller's workspace go to a scratch
+ * array of FP8BS_STATIC_SCRATCH_BYTES that the library holds in device
+ * memory on every GPU that loads it, until the process exits.
+ *
+ *   a, a_s, w, w_s, y, M, N, K: as for fp8bs_fp8_gemm (caller-owned device
+ *   buffers; inputs and output are still the caller's).
+ *
+ * Problems whose plan needs more split-K scratch than
+ * FP8BS_STATIC_SCRATCH_BYTES (fp8bs_gemm_workspace_size(M, N, K) is larger)
+ * are rejected with FP8BS_ERR_WORKSPACE before anything is launched.
+ *
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, once per device, on the current device); make that
+ * first call before any stream capture.  All calls share the one array and
+ * every call writes the partials it reads, so nothing needs clearing between
+ * calls, but calls that overlap on the GPU (other streams, other threads)
+ * race on the array: serialise them.
+ */
+#define FP8BS_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t *a, const float *a_s,
+                                                     const uint8_t *w, const float *w_s,
+                                                     int64_t M, int64_t N, int64_t K,
+                                                     uint16_t *y, void *stream);
+
+/*
  * fp8_linear: the FP8 linear layer's forward pass, act_quant followed by
  * fp8_gemm on one stream ([ACT] notes that the linear wrapper calls act_quant
  * during the forward pass):
