@@ -201,6 +201,12 @@ class Linear:
                                    self.n, self.k, vp(self.y), vp(self.ws), self.nws, stream)
         assert st == 0, self.L.fp8bs_last_error_message()
 
+    def gemm_bs(self, stream):
+        """The block-scaled (ue8m0) GEMM; needs fmt=1 (power-of-two scales)."""
+        st = self.L.fp8bs_fp8_gemm_ue8m0(vp(self.q), vp(self.s), vp(self.qw), vp(self.sw), self.m,
+                                         self.n, self.k, vp(self.y), vp(self.ws), self.nws, stream)
+        assert st == 0, self.L.fp8bs_last_error_message()
+
 
 def time_events(fn, iters, flush=None):
     """Mean device time (ms) of fn() over iters launches, each bracketed by events
@@ -261,15 +267,16 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
             lin = Linear(fp8bs, wl, mm, kk, nn, fmt=1, seed=100 + kk) if lin is None or lin.n != nn \
                 else _resize(lin, fp8bs, wl, mm)
             lin.act_quant(stream)
-            f = lambda: lin.gemm(stream)
-            for _ in range(3):
-                f()
-            ms = time_events(f, 10, flush)
             nbytes = nn * kk + 4 * (-(-nn // 128)) * (kk // 128) + mm * kk + 4 * mm * (kk // 128) + 2 * mm * nn
-            parts["decode_M%d_K%d_N%d" % (mm, kk, nn)] = {
-                "us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm,
-                "TFLOP/s": 2 * mm * nn * kk / ms / 1e9, "splitk_workspace": lin.nws,
-                "plan": fp8bs.gemm_plan(mm, nn, kk)}
+            for tag, f in (("", lambda: lin.gemm(stream)), ("_bs", lambda: lin.gemm_bs(stream))):
+                for _ in range(3):
+                    f()
+                ms = time_events(f, 10, flush)
+                parts["decode_M%d_K%d_N%d%s" % (mm, kk, nn, tag)] = {
+                    "us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm,
+                    "TFLOP/s": 2 * mm * nn * kk / ms / 1e9, "splitk_workspace": lin.nws,
+                    "plan": fp8bs.gemm_plan(mm, nn, kk),
+                    "kernel": "block-scaled MMA" if tag else "promotion"}
         del lin
     # prefill shapes: fused act_quant + GEMM per call, and the GEMM alone
     for kk, nn in wl.PREFILL_KN:
@@ -285,6 +292,16 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
                 "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
                 "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
                 "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
+            if fmt:
+                for _ in range(3):
+                    lin.gemm_bs(stream)
+                ms_g = time_events(lambda: lin.gemm_bs(stream), 10)
+                ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm_bs(stream)), 10)
+                parts["prefill_K%d_N%d_ue8m0_bs" % (kk, nn)] = {
+                    "kernel": "block-scaled MMA",
+                    "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
+                    "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
+                    "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
             del lin
     # expert-batched grouped GEMM: 32 x W [2048, 7168], 65536 routed rows
     counts = wl.expert_counts(wl.EXPERT_TOKENS * wl.EXPERT_TOPK, wl.EXPERTS, seed=70)
@@ -308,6 +325,23 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
     fl = 2 * Mt * wl.EXPERT_FFN * wl.HIDDEN
     parts["experts_grouped"] = {"rows": Mt, "us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
                                 "frac_fp8": fl / ms / 1e9 / fp8_peak}
+    # the same experts with ue8m0 scales on the block-scaled MMA
+    xg = wl.normal_with_outliers(Mt, wl.HIDDEN, seed=71, frac=0.001, factor=20.0, device="cuda")
+    qa, sa = fp8bs.act_quant(xg, 128, "ue8m0")
+    del xg
+    for e in range(wl.EXPERTS):
+        qe, se = fp8bs.weight_quant(wl.weight_f32(wl.EXPERT_FFN, wl.HIDDEN, seed=72 + e, device="cuda"),
+                                    128, "ue8m0")
+        wg[e].copy_(qe.view(torch.uint8))
+        sg[e].copy_(se)
+    f = lambda: L.fp8bs_fp8_gemm_grouped_ue8m0(wl.EXPERTS, vp(offs), Mt, vp(qa), vp(sa), vp(wg),
+                                               vp(sg), wl.EXPERT_FFN, wl.HIDDEN, vp(yg), stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10)
+    parts["experts_grouped_ue8m0_bs"] = {"rows": Mt, "us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
+                                         "frac_fp8": fl / ms / 1e9 / fp8_peak,
+                                         "kernel": "block-scaled MMA"}
     return parts
 
 

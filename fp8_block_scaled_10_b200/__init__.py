@@ -32,7 +32,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp8bs.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp8bs.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_SCALE = range(7)
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SCALE_FMT_NONE, SCALE_FMT_UE8M0 = 0, 1
 
@@ -45,7 +45,8 @@ class Fp8bsError(RuntimeError):
 
 _STATUS_NAMES = {OK: "FP8BS_OK", ERR_INVALID_ARG: "FP8BS_ERR_INVALID_ARG",
                  ERR_UNSUPPORTED: "FP8BS_ERR_UNSUPPORTED", ERR_WORKSPACE: "FP8BS_ERR_WORKSPACE",
-                 ERR_CUDA: "FP8BS_ERR_CUDA", ERR_TIMEOUT: "FP8BS_ERR_TIMEOUT"}
+                 ERR_CUDA: "FP8BS_ERR_CUDA", ERR_TIMEOUT: "FP8BS_ERR_TIMEOUT",
+                 ERR_SCALE: "FP8BS_ERR_SCALE"}
 
 _lib = None
 
@@ -73,6 +74,9 @@ def lib():
         "fp8bs_fp8_gemm": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
         "fp8bs_fp8_gemm_static_scratch": (i32, [p, p, p, p, i64, i64, i64, p, p]),
         "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
+        "fp8bs_fp8_gemm_ue8m0": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
+        "fp8bs_fp8_linear_ue8m0": (i32, [p, i64, i64, p, p, i64, p, p, p, p, sz, p]),
+        "fp8bs_fp8_gemm_grouped_ue8m0": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
         "fp8bs_fp8_gemm_grouped": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
     }
     for name, (res, args) in sig.items():
@@ -199,11 +203,13 @@ def _workspace(M, N, K, device):
     return torch.empty(n, dtype=torch.uint8, device=device), n
 
 
-def fp8_gemm(a, a_s, b, b_s):
+def fp8_gemm(a, a_s, b, b_s, scale_fmt=None):
     """y = a @ b^T on block-scaled FP8 operands, bf16 output.
 
     a: [..., K] e4m3fn, a_s: [..., K/128] float32, b: [N, K] e4m3fn,
-    b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] bfloat16."""
+    b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] bfloat16.
+    scale_fmt="ue8m0" promises that every scale is a power of two and uses
+    the tensor core's block-scaled MMA."""
     a, b = _codes(a), _codes(b)
     _need_cuda(a, a_s, b, b_s)
     K = a.shape[-1]
@@ -211,15 +217,19 @@ def fp8_gemm(a, a_s, b, b_s):
     N = b.shape[0]
     y = torch.empty(*a.shape[:-1], N, dtype=torch.bfloat16, device=a.device)
     ws, nws = _workspace(M, N, K, a.device)
-    _check(lib().fp8bs_fp8_gemm(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, _ptr(y),
-                                _ptr(ws), nws, _stream(a.device)))
+    fn = lib().fp8bs_fp8_gemm_ue8m0 if _scale_fmt(scale_fmt) else lib().fp8bs_fp8_gemm
+    _check(fn(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, _ptr(y), _ptr(ws), nws,
+              _stream(a.device)))
     return y
 
 
-def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False):
+def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,
+               weight_scale_fmt=None):
     """FP8 linear forward: act_quant(x) then fp8_gemm with the block-scaled weight.
 
-    x: [..., K] bfloat16, weight: [N, K] e4m3fn, weight_scale: [cdiv(N,128), K/128]."""
+    x: [..., K] bfloat16, weight: [N, K] e4m3fn, weight_scale: [cdiv(N,128), K/128].
+    With scale_fmt="ue8m0" and weight_scale_fmt="ue8m0" (power-of-two weight
+    scales) the GEMM runs on the block-scaled MMA."""
     w = _codes(weight)
     _need_cuda(x, w, weight_scale)
     if x.dtype != torch.bfloat16:
@@ -231,13 +241,18 @@ def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False):
     q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
     s = torch.empty(*x.shape[:-1], K // 128, dtype=torch.float32, device=x.device)
     ws, nws = _workspace(M, N, K, x.device)
-    _check(lib().fp8bs_fp8_linear(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
-                                  _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s), _ptr(ws), nws,
-                                  _stream(x.device)))
+    if _scale_fmt(scale_fmt) and _scale_fmt(weight_scale_fmt):
+        _check(lib().fp8bs_fp8_linear_ue8m0(_ptr(x), M, K, _ptr(w), _ptr(weight_scale), N,
+                                            _ptr(y), _ptr(q), _ptr(s), _ptr(ws), nws,
+                                            _stream(x.device)))
+    else:
+        _check(lib().fp8bs_fp8_linear(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
+                                      _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s), _ptr(ws),
+                                      nws, _stream(x.device)))
     return (y, q, s) if return_quant else y
 
 
-def fp8_gemm_grouped(a, a_s, w, w_s, m_offsets):
+def fp8_gemm_grouped(a, a_s, w, w_s, m_offsets, scale_fmt=None):
     """Per-expert FP8 GEMMs over rows grouped contiguously by expert.
 
     a: [M_total, K] e4m3fn, a_s: [M_total, K/128], w: [G, N, K] e4m3fn,
@@ -249,8 +264,9 @@ def fp8_gemm_grouped(a, a_s, w, w_s, m_offsets):
     G, N, K = w.shape
     M = a.shape[0]
     y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
-    _check(lib().fp8bs_fp8_gemm_grouped(G, _ptr(m_offsets), M, _ptr(a), _ptr(a_s), _ptr(w),
-                                        _ptr(w_s), N, K, _ptr(y), _stream(a.device)))
+    fn = lib().fp8bs_fp8_gemm_grouped_ue8m0 if _scale_fmt(scale_fmt) else lib().fp8bs_fp8_gemm_grouped
+    _check(fn(G, _ptr(m_offsets), M, _ptr(a), _ptr(a_s), _ptr(w), _ptr(w_s), N, K, _ptr(y),
+              _stream(a.device)))
     return y
 
 

@@ -14,6 +14,7 @@
 
 #include "fp8bs.h"
 #include "gemm.cuh"
+#include "gemm_bs.cuh"
 #include "quant.cuh"
 #include "sm100.cuh"
 
@@ -99,6 +100,16 @@ fp8bs_status setup_gemm_kernel(DeviceInfo& d) {
   return FP8BS_OK;
 }
 
+template <int BN, bool G>
+fp8bs_status setup_gemm_bs_kernel() {
+  const cudaError_t e =
+      cudaFuncSetAttribute(gemm::fp8_gemm_bs_kernel<BN, G>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemm::BsCfg<BN>::smem_bytes(G));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return FP8BS_OK;
+}
+
 // One-time per-device setup: SM count, shared-memory opt-in of the GEMM
 // kernels, and the driver's tensor-map encoder.
 fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
@@ -129,7 +140,11 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_kernel<128, false, true>(d)) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, false, true>(d)) != FP8BS_OK ||
         (r = setup_gemm_kernel<128, true, true>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, true, true>(d)) != FP8BS_OK)
+        (r = setup_gemm_kernel<256, true, true>(d)) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<128, false>()) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<256, false>()) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<256, true>()) != FP8BS_OK)
       return r;
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -189,12 +204,12 @@ double wave_efficiency(int64_t units, int slots) {
 // units, weighted by what each shape costs beyond its MMAs: a 128-wide tile
 // moves more operand bytes per MMA, a CTA pair moves a third fewer, and each
 // extra split adds a reduction pass over the output.
-Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d) {
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_pair = true) {
   Plan best{};
   double best_score = -1.0;
   const int kbn = static_cast<int>(K / 128);
   for (int pair = 0; pair <= 1; ++pair) {
-    if (pair && (!d.pair_enabled || d.pair_slots <= 0 || M <= 128)) continue;
+    if (pair && (!allow_pair || !d.pair_enabled || d.pair_slots <= 0 || M <= 128)) continue;
     const int slots = pair ? d.pair_slots : d.sms;
     const int rows = pair ? 256 : 128;
     for (int bn : {256, 128}) {
@@ -323,6 +338,61 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   return FP8BS_OK;
 }
 
+template <int BN, bool G>
+cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p,
+                           int grid, cudaStream_t st) {
+  using C = gemm::BsCfg<BN>;
+  gemm::fp8_gemm_bs_kernel<BN, G><<<grid, C::kThreads, C::smem_bytes(G), st>>>(ta, tw, p);
+  return cudaGetLastError();
+}
+
+// Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel, without
+// CTA pairs.
+fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
+                         int64_t M, int64_t N, int64_t K, uint16_t* y, void* ws, size_t ws_bytes,
+                         cudaStream_t st) {
+  fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (M == 0) return FP8BS_OK;
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  const Plan pl = plan_gemm(M, N, K, *info, false);
+  const size_t need = plan_workspace(pl, M, N);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+  CUtensorMap ta, tw;
+  if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
+  gemm::Params p{};
+  p.sa = a_s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ws = static_cast<float*>(ws);
+  p.m_offsets = nullptr;
+  p.M = M;
+  p.N = static_cast<int>(N);
+  p.kbn = static_cast<int>(K / 128);
+  p.nbn = static_cast<int>((N + 127) / 128);
+  p.m_tiles = pl.m_tiles;
+  p.n_tiles = pl.n_tiles;
+  p.splits = pl.splits;
+  p.kb_per_split = pl.kb_per_split;
+  p.num_units = pl.units;
+  p.groups = 1;
+  cudaError_t e = pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, p, pl.grid, st)
+                               : launch_gemm_bs<128, false>(ta, tw, p, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
+  if (pl.splits > 1) {
+    const int64_t MN = M * N;
+    splitk_reduce_kernel<<<grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st>>>(
+        static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+  }
+  return FP8BS_OK;
+}
+
 fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
                            int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
                            cudaStream_t st) {
@@ -376,6 +446,7 @@ const char* fp8bs_status_string(fp8bs_status status) {
     case FP8BS_ERR_WORKSPACE: return "FP8BS_ERR_WORKSPACE";
     case FP8BS_ERR_CUDA: return "FP8BS_ERR_CUDA";
     case FP8BS_ERR_TIMEOUT: return "FP8BS_ERR_TIMEOUT";
+    case FP8BS_ERR_SCALE: return "FP8BS_ERR_SCALE";
   }
   return "FP8BS_UNKNOWN_STATUS";
 }
@@ -564,6 +635,71 @@ fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t* a, const float* a_s, c
   const fp8bs_status r = static_scratch_address(&scratch);
   if (r != FP8BS_OK) return r;
   return fp8bs_fp8_gemm(a, a_s, w, w_s, M, N, K, y, scratch, FP8BS_STATIC_SCRATCH_BYTES, stream);
+}
+
+fp8bs_status fp8bs_fp8_gemm_ue8m0(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                  const float* w_s, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return run_gemm_bs(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream));
+}
+
+fp8bs_status fp8bs_fp8_linear_ue8m0(const uint16_t* x, int64_t M, int64_t K, const uint8_t* w,
+                                    const float* w_s, int64_t N, uint16_t* y, uint8_t* q,
+                                    float* s, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  fp8bs_status r = check_gemm_operands(q, s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M == 0) return FP8BS_OK;
+  cudaStream_t st = as_stream(stream);
+  if ((r = run_act_quant(x, FP8BS_DTYPE_BF16, M, K, 128, FP8BS_SCALE_FMT_UE8M0, q, s, st)) !=
+      FP8BS_OK)
+    return r;
+  return run_gemm_bs(q, s, w, w_s, M, N, K, y, workspace, workspace_bytes, st);
+}
+
+fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, int64_t M_total,
+                                          const uint8_t* a, const float* a_s, const uint8_t* w,
+                                          const float* w_s, int64_t N, int64_t K, uint16_t* y,
+                                          void* stream) {
+  if (G < 1 || G > gemm::kMaxGroups)
+    return fail(FP8BS_ERR_INVALID_ARG, "G=%lld out of [1, %d]", (long long)G, gemm::kMaxGroups);
+  if (!m_offsets || (reinterpret_cast<uintptr_t>(m_offsets) & 7u))
+    return fail(FP8BS_ERR_INVALID_ARG, "m_offsets must be an 8-byte aligned device pointer");
+  fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (M_total < 0 || M_total > (int64_t(1) << 31))
+    return fail(FP8BS_ERR_INVALID_ARG, "M_total out of range");
+  if (M_total == 0) return FP8BS_OK;
+  if (G * N > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "G*N too large");
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  const int bn = N >= 256 ? 256 : 128;
+  CUtensorMap ta, tw;
+  if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
+  gemm::Params p{};
+  p.sa = a_s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ws = nullptr;
+  p.m_offsets = m_offsets;
+  p.M = M_total;
+  p.N = static_cast<int>(N);
+  p.kbn = static_cast<int>(K / 128);
+  p.nbn = static_cast<int>((N + 127) / 128);
+  p.m_tiles = 0;
+  p.n_tiles = static_cast<int>((N + bn - 1) / bn);
+  p.splits = 1;
+  p.kb_per_split = p.kbn;
+  p.num_units = 0;
+  p.groups = static_cast<int>(G);
+  const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
+  cudaError_t e = bn == 256 ? launch_gemm_bs<256, true>(ta, tw, p, grid, as_stream(stream))
+                            : launch_gemm_bs<128, true>(ta, tw, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped_ue8m0 launch");
+  return FP8BS_OK;
 }
 
 fp8bs_status fp8bs_fp8_linear(const uint16_t* x, int64_t M, int64_t K, fp8bs_scale_fmt fmt,

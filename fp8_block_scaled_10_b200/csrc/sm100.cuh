@@ -303,6 +303,58 @@ __device__ __forceinline__ void reg_acquire() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// ---------------------------------------------------------------------------
+// Block-scaled MMA (kind::mxf8f6f4.block_scale): e4m3 operands with one ue8m0
+// scale factor per 32 K elements for every row of A and of B, read from TMEM.
+// ---------------------------------------------------------------------------
+// D (+)= (SFA x A) * (SFB x B)^T; sfa/sfb are TMEM addresses whose top two
+// bits select the scale byte (the 32-K sub-block) within each 32-bit cell.
+__device__ __forceinline__ void mma_mxf8_block_scaled(uint32_t tmem_d, uint64_t adesc,
+                                                      uint64_t bdesc, uint32_t idesc,
+                                                      uint32_t sfa, uint32_t sfb,
+                                                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copies a 32-row x 16-byte block from shared memory into TMEM lanes 0-31 and
+// replicates it into the other three 32-lane quadrants.
+__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Shared-memory descriptor of a contiguous block of 16-byte rows (no
+// swizzle): 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the
+// async proxy (tcgen05.cp / tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: A and B e4m3,
+// K-major, ue8m0 scale factors, shape M x N; sub-block ids are or-ed in per MMA
+// (A at bit 29, B at bit 4).
+__host__ __device__ constexpr uint32_t idesc_e4m3_block_scaled(int M, int N) {
+  return (0u << 7) | (0u << 10)                     // A, B format: e4m3
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (1u << 23)                               // scale factors: ue8m0
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
 // 128 bytes long and stored with the 128-byte swizzle that TMA's
 // CU_TENSOR_MAP_SWIZZLE_128B writes: 8-row groups 1024 bytes apart (stride

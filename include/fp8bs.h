@@ -56,7 +56,9 @@ typedef enum fp8bs_status {
     FP8BS_ERR_UNSUPPORTED = 2, /* well-formed but not implemented (e.g. block != 128)    */
     FP8BS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size()   */
     FP8BS_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                      */
-    FP8BS_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up (device error word) */
+    FP8BS_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up (device error word) */
+    FP8BS_ERR_SCALE = 6        /* a *_ue8m0 GEMM met a scale that is not a positive normal
+                                  power of two (device error word)                        */
 } fp8bs_status;
 
 typedef enum fp8bs_dtype {
@@ -213,6 +215,31 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t *a, const flo
                                                      uint16_t *y, void *stream);
 
 /*
+ * fp8_gemm_ue8m0: fp8_gemm for power-of-two scales ([ACT]: scale_fmt "ue8m0"
+ * rounds scales to powers of two for hardware compatibility).  Same
+ * arguments, layouts, workspace and result as fp8bs_fp8_gemm, but every a_s
+ * and w_s entry must be a positive normal power of two, which the tensor core
+ * then applies itself (tcgen05.mma kind::mxf8f6f4.block_scale with ue8m0
+ * scale factors, one FP32 accumulation over all of K).  A scale that is not
+ * such a power of two is reported through the device error word
+ * (FP8BS_ERR_SCALE) and makes the output meaningless.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_ue8m0(const uint8_t *a, const float *a_s, const uint8_t *w,
+                                            const float *w_s, int64_t M, int64_t N, int64_t K,
+                                            uint16_t *y, void *workspace, size_t workspace_bytes,
+                                            void *stream);
+
+/*
+ * fp8_linear_ue8m0: act_quant(x, 128, UE8M0) followed by fp8_gemm_ue8m0 on
+ * one stream.  Arguments as for fp8bs_fp8_linear; w_s must hold powers of
+ * two (weights quantized with the ue8m0 scale format).
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_linear_ue8m0(const uint16_t *x, int64_t M, int64_t K,
+                                              const uint8_t *w, const float *w_s, int64_t N,
+                                              uint16_t *y, uint8_t *q, float *s, void *workspace,
+                                              size_t workspace_bytes, void *stream);
+
+/*
  * fp8_linear: the FP8 linear layer's forward pass, act_quant followed by
  * fp8_gemm on one stream ([ACT] notes that the linear wrapper calls act_quant
  * during the forward pass):
@@ -251,6 +278,16 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t *m_offset
                                     const uint8_t *a, const float *a_s, const uint8_t *w,
                                     const float *w_s, int64_t N, int64_t K, uint16_t *y,
                                     void *stream);
+
+/*
+ * fp8_gemm_grouped_ue8m0: fp8_gemm_grouped with the power-of-two scale
+ * requirement and the block-scaled MMA of fp8_gemm_ue8m0.  Same arguments.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t *m_offsets,
+                                                    int64_t M_total, const uint8_t *a,
+                                                    const float *a_s, const uint8_t *w,
+                                                    const float *w_s, int64_t N, int64_t K,
+                                                    uint16_t *y, void *stream);
 
 #ifdef __cplusplus
 }
