@@ -495,7 +495,7 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
   if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
     const uint32_t cpr = static_cast<uint32_t>(N / 16);
     const uint32_t total = static_cast<uint32_t>(M * (N / 16));
-    const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 8);
+    const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
     if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
     else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
   } else {
@@ -550,6 +550,24 @@ fp8bs_status fp8bs_selftest_quotient(const float* x, const float* s, float* q, i
   quotient_selftest_kernel<<<grid_for(n, 256, info->sms * 8), 256, 0, as_stream(stream)>>>(x, s, q, n);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quotient self-test launch");
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_selftest_block_scale(const float* amax, float* s, int64_t n, int scale_fmt,
+                                        void* stream) {
+  if (n < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
+  if (scale_fmt != FP8BS_SCALE_FMT_NONE && scale_fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "unknown scale_fmt");
+  if (n == 0) return FP8BS_OK;
+  if (!amax || !s) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  scale_selftest_kernel<<<grid_for(n, 256, info->sms * 8), 256, 0, as_stream(stream)>>>(
+      amax, s, n, scale_fmt == FP8BS_SCALE_FMT_UE8M0);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block-scale self-test launch");
   return FP8BS_OK;
 }
 

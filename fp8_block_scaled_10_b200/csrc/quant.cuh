@@ -26,12 +26,26 @@ namespace fp8bs {
 // Scalar pieces
 // ---------------------------------------------------------------------------
 
-// s = max(amax, 1e-4f) / 448 with IEEE division; for ue8m0 the smallest power
-// of two >= s, taken on the bit pattern (s is a positive normal number here:
-// s >= 1e-4/448): a nonzero fraction bumps the exponent and clears the
-// fraction.
+// Correctly rounded fp32 quotient x / d from r = RN(1/d) by Markstein's
+// division correction (see quotient2 below for the method and its premises).
+__device__ __forceinline__ float quotient1(float x, float r, float nd) {
+  float q = x * r;
+  q = fmaf(fmaf(q, nd, x), r, q);
+  q = fmaf(fmaf(q, nd, x), r, q);
+  return q;
+}
+
+// s = max(amax, 1e-4f) / 448, correctly rounded (the division by the
+// constant 448 through quotient1 with r = RN(1/448), a compile-time constant;
+// a >= 1e-4 keeps every step far from underflow, and an infinite amax, where
+// the correction would produce inf - inf, is passed through as the quotient
+// inf / 448 = inf); for ue8m0 the smallest power of two >= s, taken on the
+// bit pattern (s is a positive normal number): a nonzero fraction bumps the
+// exponent and clears the fraction.
 __device__ __forceinline__ float block_scale(float amax, bool ue8m0) {
-  float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+  const float a = fmaxf(amax, 1e-4f);
+  float s = quotient1(a, 1.0f / 448.0f, -448.0f);
+  if (isinf(a)) s = a;
   if (ue8m0) {
     uint32_t u = __float_as_uint(s);
     if (u & 0x007FFFFFu) u = (u & 0x7F800000u) + 0x00800000u;
@@ -100,6 +114,14 @@ __global__ void quotient_selftest_kernel(const float* __restrict__ x, const floa
     const float2 r = make_float2(__frcp_rn(sc), 0.0f);
     q[i] = quotient2(make_float2(x[i], 0.0f), r, make_float2(-sc, -1.0f)).x;
   }
+}
+
+// s[i] = block_scale(amax[i]) for the self-test of the scale rule.
+__global__ void scale_selftest_kernel(const float* __restrict__ amax, float* __restrict__ s,
+                                      int64_t n, bool ue8m0) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * 256)
+    s[i] = block_scale(amax[i], ue8m0);
 }
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
@@ -191,7 +213,7 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __uint_as_float(__float_as_uint(v) | ((code & 0x80u) << 24));
 }
 
-constexpr int kDeqThreads = 256;
+constexpr int kDeqThreads = 512;
 constexpr int kDeqUnroll = 2;
 
 // Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row;

@@ -170,6 +170,18 @@ FP8BS_API size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 FP8BS_API fp8bs_status fp8bs_selftest_quotient(const float *x, const float *s, float *q, int64_t n,
                                                void *stream);
 
+/*
+ * Self-test of the per-block scale rule that act_quant and weight_quant
+ * apply to a block's absolute maximum ([ACT]; scale_fmt as in act_quant):
+ * s[i] = max(amax[i], 1e-4) / 448 as the correctly rounded fp32 quotient,
+ * then for FP8BS_SCALE_FMT_UE8M0 the smallest power of two >= that.  amax and s
+ * are device fp32 arrays of n elements; amax[i] is a non-negative number or
+ * +inf.  Errors: FP8BS_ERR_INVALID_ARG for n < 0, a null pointer with n > 0
+ * or an unknown scale_fmt.  For verification only.
+ */
+FP8BS_API fp8bs_status fp8bs_selftest_block_scale(const float *amax, float *s, int64_t n,
+                                                  int scale_fmt, void *stream);
+
 /* Launch plan fp8_gemm would use for an M x N x K problem on the current
  * device (tile width, CTA pairing, K split, work units, grid), as a
  * NUL-terminated string in thread-local storage; for logs and benchmarks. */

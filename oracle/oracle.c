@@ -160,7 +160,10 @@ uint16_t oracle_bf16_from_f32(float f)
 float oracle_ue8m0_round_up(float s)
 {
     int e;
-    double f = frexp((double)s, &e);              /* s = f * 2^e, f in [0.5, 1) */
+    double f;
+    if (!isfinite(s))                             /* +inf: no larger power of two */
+        return s;
+    f = frexp((double)s, &e);                     /* s = f * 2^e, f in [0.5, 1) */
     if (f == 0.5)
         return s;
     return (float)ldexp(1.0, e);

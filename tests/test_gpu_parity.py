@@ -369,3 +369,51 @@ def test_quotient_matches_ieee_division():
     assert big.mean() > 0.7
     # ... and everywhere, the e4m3 code act_quant derives from it
     assert np.array_equal(oracle.e4m3_encode_array(got), oracle.e4m3_encode_array(ref))
+
+
+def _scale_selftest(amax, scale_fmt):
+    s = torch.empty_like(amax)
+    st_code = fp8bs.lib().fp8bs_selftest_block_scale(
+        ctypes.c_void_p(amax.data_ptr()), ctypes.c_void_p(s.data_ptr()), amax.numel(),
+        fp8bs.SCALE_FMT_UE8M0 if scale_fmt == "ue8m0" else fp8bs.SCALE_FMT_NONE,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st_code == fp8bs.OK
+    return s
+
+
+def test_block_scale_rule_every_float():
+    """The kernels' scale max(amax, 1e-4) / 448 equals the correctly rounded
+    fp32 quotient for every fp32 amax from 0 to +inf (checked against CUDA's
+    IEEE division in torch, chunk by chunk), and ue8m0 rounds it up to a power
+    of two; a sample is checked against the oracle's scale rule as well."""
+    top = 0x7F800000                                   # +inf, included
+    chunk = 1 << 27
+    floor = torch.tensor(1e-4, dtype=torch.float32, device="cuda")
+    for start in range(0, top + 1, chunk):
+        bits = torch.arange(start, min(start + chunk, top + 1), dtype=torch.int32, device="cuda")
+        amax = bits.view(torch.float32)
+        # a tensor divisor: torch turns division by a Python scalar into a
+        # multiplication by its reciprocal, which is not correctly rounded
+        want = torch.maximum(amax, floor) / torch.full_like(amax, 448.0)
+        got = _scale_selftest(amax, "none")
+        bad = (got.view(torch.int32) != want.view(torch.int32))
+        assert not bool(bad.any()), (amax[bad][:4].tolist(), got[bad][:4].tolist())
+        up = _scale_selftest(amax, "ue8m0")
+        m, e = torch.frexp(want)                        # want = m 2^e, m in [0.5, 1)
+        want_up = torch.where((m == 0.5) | torch.isinf(want), want,
+                              torch.ldexp(torch.ones_like(want), e))
+        assert torch.equal(up.view(torch.int32), want_up.view(torch.int32))
+        del bits, amax, want, got, up, m, e, want_up
+    # zero, subnormals and values under the floor all give the floor's scale
+    small = torch.tensor([0.0, 1e-45, 1e-38, 5e-5, 9.9999e-5], device="cuda")
+    assert torch.equal(_scale_selftest(small, "none"),
+                       torch.full_like(small, float(np.float32(1e-4) / np.float32(448))))
+    # against the oracle on a sample spanning many binades
+    rng = np.random.default_rng(5)
+    sample = (10.0 ** rng.uniform(-6, 38, 4096)).astype(np.float32)
+    sample[:3] = [np.float32(1e-4), np.float32(448.0), np.float32(np.inf)]
+    for fmt in ("none", "ue8m0"):
+        got = _scale_selftest(torch.from_numpy(sample).cuda(), fmt).cpu().numpy()
+        ref = np.array([oracle.block_scale(float(a), fmt == "ue8m0") for a in sample],
+                       dtype=np.float32)
+        assert np.array_equal(f32bits(got), f32bits(ref)), fmt

@@ -163,6 +163,9 @@ def test_ue8m0_round_up_is_exact_power_of_two_ceiling():
                                              np.nextafter(f32(1), f32(0))])])
     for v in vals:
         assert oracle.ue8m0_round_up(v) == _exact_pow2_ceil(v), v
+    # an infinite scale (a block holding inf) has no larger power of two
+    assert oracle.ue8m0_round_up(np.inf) == np.inf
+    assert oracle.block_scale(np.inf, True) == np.inf
 
 
 def test_block_scale_pages_constants():
