@@ -177,6 +177,37 @@ fp8bs_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
   return FP8BS_OK;
 }
 
+// Every GEMM configuration fits the 227 KB of shared memory a CTA can opt into.
+constexpr int kMaxSmemOptin = 227 * 1024;
+static_assert(gemm::Cfg<256, false>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<128, false>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<256, true>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<128, true>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::BsCfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::BsCfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+
+// bf16 y [rows, cols] for the GEMM epilogue's TMA stores: boxes of 32 rows x
+// 32 columns in the 64-byte swizzle the epilogue stages them in.  Usable when
+// the row pitch is a multiple of 16 bytes (cols % 8 == 0); otherwise *map is
+// zeroed and the kernel stores directly (y_tma = 0).
+fp8bs_status make_tmap_y(CUtensorMap* map, const void* y, int64_t rows, int64_t cols,
+                         bool enable, int* y_tma) {
+  memset(map, 0, sizeof(*map));
+  *y_tma = 0;
+  if (!enable || cols % 8 != 0) return FP8BS_OK;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+  const cuuint32_t box[2] = {32u, 32u};
+  const cuuint32_t elem[2] = {1u, 1u};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(y), dims,
+                              strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (y) failed (%d)", (int)r);
+  *y_tma = 1;
+  return FP8BS_OK;
+}
+
 int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
   const int64_t need = (work_items + per_cta - 1) / per_cta;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, max_ctas)));
@@ -201,9 +232,14 @@ double wave_efficiency(int64_t units, int slots) {
 
 // Chooses tile width, CTA pairing and K split.  The score is the fraction of
 // persistent slots (SMs, or CTA pairs) kept busy over the waves of work
-// units, weighted by what each shape costs beyond its MMAs: a 128-wide tile
-// moves more operand bytes per MMA, a CTA pair moves a third fewer, and each
-// extra split adds a reduction pass over the output.
+// units, weighted by what each shape costs beyond its MMAs: a CTA pair moves
+// a third fewer operand bytes, and each extra split adds a reduction pass
+// over the output.  When several 128-row tiles share each W tile (M >= 256)
+// the kernel is bound by the shared-memory operand feed (about 70 B per SM
+// clock from L2): one K block of a 128 x 256 tile moves 48 KB in ~690 clocks,
+// of a 128 x 128 tile 32 KB in ~470 clocks for half the MMA work, so a
+// 128-wide tile runs at ~0.75 of the 256-wide rate.  Below that, the weight
+// stream from HBM bounds both widths alike.
 Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_pair = true) {
   Plan best{};
   double best_score = -1.0;
@@ -226,7 +262,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_
         const double eff = wave_efficiency(units, slots);
         // Useful rows per unit when M is smaller than the unit.
         const double fill = static_cast<double>(std::min<int64_t>(M, rows)) / rows;
-        const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? 0.97 : 1.0);
+        const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? (M >= 256 ? 0.75 : 0.97) : 1.0);
         const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
         const double score = eff * feed * split_cost * (M < rows ? fill + 0.5 * (1 - fill) : 1.0);
         if (score > best_score + 1e-9) {
@@ -252,8 +288,8 @@ size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
 }
 
 template <int BN, bool G, bool PAIR>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p,
-                        int grid, cudaStream_t st) {
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
+                        const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::Cfg<BN, PAIR>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -269,16 +305,17 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const gemm
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, gemm::fp8_gemm_kernel<BN, G, PAIR>, ta, tw, p);
+  return cudaLaunchKernelEx(&cfg, gemm::fp8_gemm_kernel<BN, G, PAIR>, ta, tw, ty, p);
 }
 
 template <bool G>
 cudaError_t launch_gemm_any(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tw,
-                            const gemm::Params& p, int grid, cudaStream_t st) {
-  if (pair) return bn == 256 ? launch_gemm<256, G, true>(ta, tw, p, grid, st)
-                             : launch_gemm<128, G, true>(ta, tw, p, grid, st);
-  return bn == 256 ? launch_gemm<256, G, false>(ta, tw, p, grid, st)
-                   : launch_gemm<128, G, false>(ta, tw, p, grid, st);
+                            const CUtensorMap& ty, const gemm::Params& p, int grid,
+                            cudaStream_t st) {
+  if (pair) return bn == 256 ? launch_gemm<256, G, true>(ta, tw, ty, p, grid, st)
+                             : launch_gemm<128, G, true>(ta, tw, ty, p, grid, st);
+  return bn == 256 ? launch_gemm<256, G, false>(ta, tw, ty, p, grid, st)
+                   : launch_gemm<128, G, false>(ta, tw, ty, p, grid, st);
 }
 
 fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
@@ -308,10 +345,11 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
 
-  CUtensorMap ta, tw;
+  CUtensorMap ta, tw, ty;
+  gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, w_box_rows(pl.bn, pl.pair))) != FP8BS_OK) return r;
-  gemm::Params p{};
+  if ((r = make_tmap_y(&ty, y, M, N, pl.splits == 1, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -327,7 +365,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
   p.groups = 1;
-  cudaError_t e = launch_gemm_any<false>(pl.bn, pl.pair, ta, tw, p, pl.grid, st);
+  cudaError_t e = launch_gemm_any<false>(pl.bn, pl.pair, ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
@@ -339,10 +377,10 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
 }
 
 template <int BN, bool G>
-cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p,
-                           int grid, cudaStream_t st) {
+cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
+                           const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::BsCfg<BN>;
-  gemm::fp8_gemm_bs_kernel<BN, G><<<grid, C::kThreads, C::smem_bytes(G), st>>>(ta, tw, p);
+  gemm::fp8_gemm_bs_kernel<BN, G><<<grid, C::kThreads, C::smem_bytes(G), st>>>(ta, tw, ty, p);
   return cudaGetLastError();
 }
 
@@ -362,10 +400,11 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   const size_t need = plan_workspace(pl, M, N);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
-  CUtensorMap ta, tw;
+  CUtensorMap ta, tw, ty;
+  gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
-  gemm::Params p{};
+  if ((r = make_tmap_y(&ty, y, M, N, pl.splits == 1, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -381,8 +420,8 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
   p.groups = 1;
-  cudaError_t e = pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, p, pl.grid, st)
-                               : launch_gemm_bs<128, false>(ta, tw, p, pl.grid, st);
+  cudaError_t e = pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, ty, p, pl.grid, st)
+                               : launch_gemm_bs<128, false>(ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
@@ -693,10 +732,11 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
   const int bn = N >= 256 ? 256 : 128;
-  CUtensorMap ta, tw;
+  CUtensorMap ta, tw, ty;
+  gemm::Params p{};
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
-  gemm::Params p{};
+  if ((r = make_tmap_y(&ty, y, M_total, N, true, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -714,8 +754,8 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
   p.groups = static_cast<int>(G);
   const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
   const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
-  cudaError_t e = bn == 256 ? launch_gemm_bs<256, true>(ta, tw, p, grid, as_stream(stream))
-                            : launch_gemm_bs<128, true>(ta, tw, p, grid, as_stream(stream));
+  cudaError_t e = bn == 256 ? launch_gemm_bs<256, true>(ta, tw, ty, p, grid, as_stream(stream))
+                            : launch_gemm_bs<128, true>(ta, tw, ty, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped_ue8m0 launch");
   return FP8BS_OK;
 }
@@ -750,10 +790,11 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   const int bn = N >= 256 ? 256 : 128;
   // CTA pairs when the groups are large enough on average to fill 256-row units.
   const bool pair = info->pair_enabled && info->pair_slots > 0 && M_total >= 256 * G;
-  CUtensorMap ta, tw;
+  CUtensorMap ta, tw, ty;
+  gemm::Params p{};
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, G * N, K, w_box_rows(bn, pair))) != FP8BS_OK) return r;
-  gemm::Params p{};
+  if ((r = make_tmap_y(&ty, y, M_total, N, true, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -774,7 +815,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   const int64_t max_units = ((M_total + rows - 1) / rows + G) * p.n_tiles;
   const int slots = pair ? info->pair_slots : info->sms;
   const int grid_units = static_cast<int>(std::min<int64_t>(max_units, slots));
-  cudaError_t e = launch_gemm_any<true>(bn, pair, ta, tw, p, pair ? 2 * grid_units : grid_units,
+  cudaError_t e = launch_gemm_any<true>(bn, pair, ta, tw, ty, p, pair ? 2 * grid_units : grid_units,
                                         as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
   return FP8BS_OK;

@@ -68,7 +68,40 @@ struct Params {
   int kb_per_split;
   int num_units;            // dense mode; grouped mode derives it on the device
   int groups;               // grouped mode
+  int y_tma;                // 1: bf16 y written by TMA stores through staging boxes
 };
+
+// Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
+// 32 rows x 32 columns (2 KB) in shared memory, laid out in the 64-byte
+// swizzle of the y tensor map (16-byte chunk q of row r at chunk
+// q ^ ((r >> 1) & 3)), so the 32 lanes writing one row each hit distinct
+// banks.  One TMA store then writes 32 rows x 64 B of y; the warps' direct
+// stores would write 16 B into 32 different rows per instruction.
+constexpr int kOutBoxBytes = 32 * 32 * 2;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b2);
+}
+
+// Stages this lane's 32 packed bf16 values as row `lane` of the warp's box and
+// stores the box at column x, row y of y.  Lane 0 first waits until the
+// box's previous store has read it.
+__device__ __forceinline__ void store_out_box(const CUtensorMap* tmap_y, uint8_t* box, int lane,
+                                              const uint32_t (&h)[16], int32_t x, int32_t y) {
+  if (lane == 0) tma_store_wait_read();
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmap_y, box, x, y);
+    tma_store_commit();
+  }
+}
 
 template <int BN, bool PAIR>
 struct Cfg {
@@ -105,10 +138,14 @@ struct Cfg {
   static constexpr int kBChunkBytes = kBChunkRows * BK;
   static constexpr int kSubBuffers = 2 * kSplitN;
   static constexpr int kCtrlBytes = 256;
-  // grouped mode: per-group m-tile prefix (int) and clamped [lo, hi) rows (int64)
-  static constexpr int kGroupBytes = 8 * 2 * kMaxGroups + 4 * (kMaxGroups + 1);
-  static constexpr int smem_bytes(bool grouped) {
-    return kStages * kStageBytes + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1024;
+  // grouped mode: per-group m-tile prefix (int)
+  static constexpr int kGroupBytes = 4 * (kMaxGroups + 1);
+  // output staging boxes (one per epilogue warp), 1024-byte aligned
+  __host__ __device__ static constexpr int out_offset(bool grouped) {
+    return (kStages * kStageBytes + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1023) & ~1023;
+  }
+  __host__ __device__ static constexpr int smem_bytes(bool grouped) {
+    return out_offset(grouped) + kEpiWarps * kOutBoxBytes + 1024;
   }
   // Arrivals that release one TMEM sub-buffer: the epilogue warps that read
   // it, in both CTAs in pair mode.
@@ -155,13 +192,20 @@ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   return t;
 }
 
+// Row range [lo, hi) of group g: the device offsets clamped to [0, M] and
+// made non-decreasing.
+__device__ __forceinline__ void group_rows(const Params& p, int g, int64_t& lo, int64_t& hi) {
+  lo = __ldg(p.m_offsets + g);
+  hi = __ldg(p.m_offsets + g + 1);
+  lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
+  hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
+}
+
 // Grouped units: n tile fastest inside one global m tile, so the CTAs running
 // at the same time work on one or two experts and read each W_e once.
-// tile_prefix[g] is the number of m tiles of groups < g; rows[2g], rows[2g+1]
-// are group g's clamped row range [lo, hi).
+// tile_prefix[g] is the number of m tiles of groups < g.
 template <int kUnitRows>
-__device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix,
-                                             const int64_t* rows, int u) {
+__device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix, int u) {
   Unit t;
   const int gm = u / p.n_tiles;
   t.n_tile = u % p.n_tiles;
@@ -171,8 +215,10 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
     if (tile_prefix[mid] <= gm) a = mid; else b = mid;
   }
   t.group = a;
-  t.row0 = rows[2 * a] + static_cast<int64_t>(gm - tile_prefix[a]) * kUnitRows;
-  t.row_end = rows[2 * a + 1];
+  int64_t lo, hi;
+  group_rows(p, a, lo, hi);
+  t.row0 = lo + static_cast<int64_t>(gm - tile_prefix[a]) * kUnitRows;
+  t.row_end = hi;
   t.split = 0;
   t.kb0 = 0;
   t.kb1 = p.kbn;
@@ -182,7 +228,8 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
 template <int BN, bool GROUPED, bool PAIR>
 __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+                    const __grid_constant__ CUtensorMap tmap_w,
+                    const __grid_constant__ CUtensorMap tmap_y, const Params p) {
   using C = Cfg<BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -197,8 +244,8 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
   uint64_t* tempty = ctrl->tempty;
   uint64_t* flush = &ctrl->flush;
   volatile int* abort_flag = &ctrl->abort_flag;
-  int64_t* group_rows = reinterpret_cast<int64_t*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
-  int* tile_prefix = reinterpret_cast<int*>(group_rows + 2 * kMaxGroups);
+  int* tile_prefix = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
+  uint8_t* out_boxes = smem + C::out_offset(GROUPED);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -222,6 +269,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_descriptor(&tmap_a);
     tma_prefetch_descriptor(&tmap_w);
+    if (p.y_tma) tma_prefetch_descriptor(&tmap_y);
   }
   if (warp == 1) {
     if (PAIR) {
@@ -241,12 +289,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
         const int g = g0 + lane;
         int tiles = 0;
         if (g < p.groups) {
-          int64_t lo = p.m_offsets[g], hi = p.m_offsets[g + 1];
-          lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
-          hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
+          int64_t lo, hi;
+          group_rows(p, g, lo, hi);
           tiles = static_cast<int>((hi - lo + C::kUnitRows - 1) / C::kUnitRows);
-          group_rows[2 * g] = lo;
-          group_rows[2 * g + 1] = hi;
         }
         int incl = tiles;
 #pragma unroll
@@ -274,7 +319,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
   auto unit_of = [&](int u) -> Unit {
     Unit t;
     if (GROUPED) {
-      t = grouped_unit<C::kUnitRows>(p, tile_prefix, group_rows, u);
+      t = grouped_unit<C::kUnitRows>(p, tile_prefix, u);
       t.w_row0 = static_cast<int64_t>(t.group) * p.N + static_cast<int64_t>(t.n_tile) * BN;
     } else {
       t = dense_unit<C::kUnitRows>(p, u);
@@ -455,8 +500,21 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
         tb ^= 1;
         if (tb == 0) tphase ^= 1u;
       }
-      if (row_ok) {
-        const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
+      const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
+      const int64_t slab0 = t.row0 + static_cast<int64_t>(rank) * BM + quad * 32;
+      if (p.y_tma && slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end)) {
+        // Staged TMA stores; rows past M and columns past N are clipped.
+        uint8_t* box = out_boxes + e * kOutBoxBytes;
+#pragma unroll
+        for (int c = 0; c < CPW / 32; ++c) {
+          if (col0 + 32 * c >= p.N) break;
+          uint32_t h[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) h[j] = pack_bf16x2(acc[c * 16 + j].x, acc[c * 16 + j].y);
+          store_out_box(&tmap_y, box, lane, h, static_cast<int32_t>(col0 + 32 * c),
+                        static_cast<int32_t>(slab0));
+        }
+      } else if (row_ok) {
         if (p.splits == 1) {
           __nv_bfloat16* yrow = p.y + row * p.N;
 #pragma unroll
@@ -496,7 +554,8 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
         }
       }
     }
-  epilogue_done:;
+  epilogue_done:
+    if (lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();

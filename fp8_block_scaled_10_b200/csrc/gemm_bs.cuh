@@ -26,8 +26,9 @@
 //               ahead), writes the exponent atoms into the stage's shared
 //               memory and checks that each scale is a positive normal power
 //               of two (else device error FP8BS_ERR_SCALE = 6).
-//   warps 4-11  epilogue: per tile, each thread converts one row of BN/2
-//               accumulator columns to bf16 (or writes FP32 split-K partials).
+//   warps 4-11  epilogue: per tile, each thread reads one row of BN/2
+//               accumulator columns into registers as bf16, releases the
+//               accumulator, then stores (or writes FP32 split-K partials).
 #pragma once
 
 #include "gemm.cuh"
@@ -53,9 +54,13 @@ struct BsCfg {
   static constexpr int kFirstEpiWarp = 4;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
   static constexpr int kCtrlBytes = 256;
-  static constexpr int kGroupBytes = 8 * 2 * kMaxGroups + 4 * (kMaxGroups + 1);
-  static constexpr int smem_bytes(bool grouped) {
-    return kStages * (kStageBytes + kSFBytes) + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1024;
+  static constexpr int kGroupBytes = 4 * (kMaxGroups + 1);
+  __host__ __device__ static constexpr int out_offset(bool grouped) {
+    return (kStages * (kStageBytes + kSFBytes) + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1023) &
+           ~1023;
+  }
+  __host__ __device__ static constexpr int smem_bytes(bool grouped) {
+    return out_offset(grouped) + kEpiWarps * kOutBoxBytes + 1024;
   }
 };
 
@@ -83,7 +88,8 @@ __device__ __forceinline__ uint32_t ue8m0_byte(float v, bool* bad) {
 template <int BN, bool GROUPED>
 __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     fp8_gemm_bs_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                       const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+                       const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_y, const Params p) {
   using C = BsCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -100,8 +106,8 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
   uint64_t* tempty = ctrl->tempty;
   uint64_t* flush = &ctrl->flush;
   volatile int* abort_flag = &ctrl->abort_flag;
-  int64_t* group_rows = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(ctrl) + C::kCtrlBytes);
-  int* tile_prefix = reinterpret_cast<int*>(group_rows + 2 * kMaxGroups);
+  int* tile_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ctrl) + C::kCtrlBytes);
+  uint8_t* out_boxes = smem + C::out_offset(GROUPED);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -124,6 +130,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_descriptor(&tmap_a);
     tma_prefetch_descriptor(&tmap_w);
+    if (p.y_tma) tma_prefetch_descriptor(&tmap_y);
   }
   if (warp == 1) {
     tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
@@ -136,12 +143,9 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
         const int g = g0 + lane;
         int tiles = 0;
         if (g < p.groups) {
-          int64_t lo = p.m_offsets[g], hi = p.m_offsets[g + 1];
-          lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
-          hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
+          int64_t lo, hi;
+          group_rows(p, g, lo, hi);
           tiles = static_cast<int>((hi - lo + BM - 1) / BM);
-          group_rows[2 * g] = lo;
-          group_rows[2 * g + 1] = hi;
         }
         int incl = tiles;
 #pragma unroll
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
   auto unit_of = [&](int u) -> Unit {
     Unit t;
     if (GROUPED) {
-      t = grouped_unit<BM>(p, tile_prefix, group_rows, u);
+      t = grouped_unit<BM>(p, tile_prefix, u);
       t.w_row0 = static_cast<int64_t>(t.group) * p.N + static_cast<int64_t>(t.n_tile) * BN;
     } else {
       t = dense_unit<BM>(p, u);
@@ -362,39 +366,70 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
       const int64_t row = t.row0 + row_in_tile;
       const bool row_ok = row < t.row_end;
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
+      const uint32_t acc_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
+      if (p.splits == 1) {
+        // Read all of this warp's columns as packed bf16 first and hand the
+        // accumulator back, so the next tile's MMAs start before the stores.
+        uint32_t h[NCH][16];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_addr + static_cast<uint32_t>(tb * BN + g * CPW + 32 * c), v);
-        tmem_ld_wait(v);
-        if (c + 1 == NCH) {
-          // All of this warp's accumulator columns are in registers.
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[tb]);
-        }
-        if (!row_ok) continue;
-        const int64_t col = col0 + 32 * c;
-        if (p.splits == 1) {
-          __nv_bfloat16* yrow = p.y + row * p.N;
-          if (vec_store && col + 32 <= p.N) {
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(acc_addr + 32 * c, v);
+          tmem_ld_wait(v);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t h[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * j]),
-                                                          __uint_as_float(v[8 * q + 2 * j + 1]));
-                h[j] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              *reinterpret_cast<uint4*>(yrow + col + 8 * q) = make_uint4(h[0], h[1], h[2], h[3]);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col + j < p.N) yrow[col + j] = __float2bfloat16_rn(__uint_as_float(v[j]));
+          for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]),
+                                                      __uint_as_float(v[2 * j + 1]));
+            h[c][j] = *reinterpret_cast<uint32_t*>(&b2);
           }
-        } else {
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        const int64_t slab0 = t.row0 + quad * 32;
+        if (p.y_tma && slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end)) {
+          // Staged TMA stores; rows past M and columns past N are clipped.
+          uint8_t* box = out_boxes + e * kOutBoxBytes;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            if (col0 + 32 * c >= p.N) break;
+            store_out_box(&tmap_y, box, lane, h[c], static_cast<int32_t>(col0 + 32 * c),
+                          static_cast<int32_t>(slab0));
+          }
+        } else if (row_ok) {
+          __nv_bfloat16* yrow = p.y + row * p.N;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            const int64_t col = col0 + 32 * c;
+            if (vec_store && col + 32 <= p.N) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(yrow + col + 8 * q) =
+                    make_uint4(h[c][4 * q], h[c][4 * q + 1], h[c][4 * q + 2], h[c][4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const uint32_t pair = h[c][j >> 1];
+                const uint16_t bits = static_cast<uint16_t>((j & 1) ? (pair >> 16) : (pair & 0xFFFFu));
+                if (col + j < p.N) yrow[col + j] = __ushort_as_bfloat16(bits);
+              }
+            }
+          }
+        }
+      } else {
+        // FP32 split-K partials, chunk by chunk.
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(acc_addr + 32 * c, v);
+          tmem_ld_wait(v);
+          if (c + 1 == NCH) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tb]);
+          }
+          if (!row_ok) continue;
+          const int64_t col = col0 + 32 * c;
           float* wrow = p.ws + (static_cast<int64_t>(t.split) * p.M + row) * p.N;
           if ((p.N % 4) == 0 && col + 32 <= p.N) {
 #pragma unroll
@@ -414,7 +449,8 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
         tphase ^= 1u;
       }
     }
-  epilogue_done:;
+  epilogue_done:
+    if (lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
