@@ -208,6 +208,14 @@ fp8bs_status make_tmap_y(CUtensorMap* map, const void* y, int64_t rows, int64_t 
   return FP8BS_OK;
 }
 
+// Multiplier and shifts of div_invariant for a divisor d >= 1.
+InvariantDiv invariant_div(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (uint64_t(1) << l) < d) ++l;
+  const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
+  return InvariantDiv{static_cast<uint32_t>(m), l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
+}
+
 int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
   const int64_t need = (work_items + per_cta - 1) / per_cta;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, max_ctas)));
@@ -451,8 +459,8 @@ fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
   const int64_t nblocks = rows * (cols / 128);
-  // 16 half-warps per CTA, kActUnroll blocks each per iteration; up to 8 CTAs per SM.
-  const int grid = grid_for(nblocks, 16 * kActUnroll, info->sms * 8);
+  // (kActThreads / kActLanes) blocks per CTA per unroll step; up to 8 CTAs per SM.
+  const int grid = grid_for(nblocks, (kActThreads / kActLanes) * kActUnroll, info->sms * 8);
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   if (x_dtype == FP8BS_DTYPE_BF16) {
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
@@ -535,8 +543,9 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
     const uint32_t cpr = static_cast<uint32_t>(N / 16);
     const uint32_t total = static_cast<uint32_t>(M * (N / 16));
     const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
-    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
-    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, nbn);
+    const InvariantDiv row_div = invariant_div(cpr);
+    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, row_div, nbn);
+    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, row_div, nbn);
   } else {
     const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
     if (bf) weight_dequant_any_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);

@@ -146,51 +146,64 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 // ---------------------------------------------------------------------------
 // The input is a flat run of nblocks blocks of 128 elements (the last
 // dimension is a multiple of 128, so blocks never straddle rows) and block b's
-// scale is s[b].  A half-warp owns one block: each of its 16 lanes holds 8
-// consecutive elements (16 bytes of bf16), the amax is a 4-step xor shuffle
-// inside the half-warp, and each lane writes 8 code bytes.  Every warp
-// handles kUnroll block pairs per iteration with all loads issued first.
+// scale is s[b].  kActLanes lanes own one block, each holding 128 / kActLanes
+// consecutive elements; the amax is a log2(kActLanes)-step xor shuffle among
+// them, each thread computes one scale per block and writes its code bytes.
+// A warp covers (32 / kActLanes) * kActUnroll consecutive blocks per
+// iteration with all loads issued first.
 constexpr int kActThreads = 256;
-constexpr int kActUnroll = 4;
+constexpr int kActLanes = 4;
+constexpr int kActUnroll = 1;
+constexpr int kActElems = 128 / kActLanes;
+constexpr int kActBlocksPerWarp = 32 / kActLanes;
 
 template <typename T, bool UE8M0>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const T* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
                      int64_t nblocks) {
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;
-  const int l16 = lane & 15;
+  const int group = lane / kActLanes;
+  const int li = lane % kActLanes;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kActThreads) >> 5;
-  const int64_t step = nwarps * 2 * kActUnroll;
+  const int64_t step = nwarps * kActBlocksPerWarp * kActUnroll;
 
-  for (int64_t base = warp * 2 * kActUnroll; base < nblocks; base += step) {
-    float v[kActUnroll][8];
+  for (int64_t base = warp * kActBlocksPerWarp * kActUnroll; base < nblocks; base += step) {
+    float v[kActUnroll][kActElems];
 #pragma unroll
     for (int u = 0; u < kActUnroll; ++u) {
-      const int64_t b = base + 2 * u + half;
+      const int64_t b = base + kActBlocksPerWarp * u + group;
       if (b < nblocks) {
-        load8(x + b * 128 + l16 * 8, v[u]);
+        const T* p = x + b * 128 + li * kActElems;
+#pragma unroll
+        for (int h = 0; h < kActElems / 8; ++h)
+          load8(p + 8 * h, *reinterpret_cast<float(*)[8]>(&v[u][8 * h]));
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+        for (int j = 0; j < kActElems; ++j) v[u][j] = 0.0f;
       }
     }
 #pragma unroll
     for (int u = 0; u < kActUnroll; ++u) {
-      const int64_t b = base + 2 * u + half;
+      const int64_t b = base + kActBlocksPerWarp * u + group;
       float amax = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[u][j]));
+      for (int j = 0; j < kActElems; ++j) amax = fmaxf(amax, fabsf(v[u][j]));
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1)
+      for (int off = kActLanes / 2; off >= 1; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
       const float sc = block_scale(amax, UE8M0);
       const float r = __frcp_rn(sc);
       if (b < nblocks) {
-        const uint2 codes = quantize8<UE8M0>(v[u], sc, r);
-        __stcs(reinterpret_cast<uint2*>(q + b * 128 + l16 * 8), codes);
-        if (l16 == 0) __stcs(s + b, sc);
+        uint8_t* qp = q + b * 128 + li * kActElems;
+#pragma unroll
+        for (int h = 0; h < kActElems / 16; ++h) {
+          const uint2 lo = quantize8<UE8M0>(*reinterpret_cast<const float(*)[8]>(&v[u][16 * h]), sc, r);
+          const uint2 hi =
+              quantize8<UE8M0>(*reinterpret_cast<const float(*)[8]>(&v[u][16 * h + 8]), sc, r);
+          __stcs(reinterpret_cast<uint4*>(qp + 16 * h), make_uint4(lo.x, lo.y, hi.x, hi.y));
+        }
+        if (li == 0) __stcs(s + b, sc);
       }
     }
   }
@@ -219,11 +232,44 @@ constexpr int kDeqUnroll = 2;
 // Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row;
 // all 16 share one block scale because 16 divides 128.  Chunk indices fit in
 // 32 bits (the host checks M * N / 16 < 2^32).
+// Quotient n / d for a divisor fixed per launch, by multiplication
+// (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", 1994, the round-up method): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, t = mulhi(m, n) and
+// n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0).
+struct InvariantDiv {
+  uint32_t m, sh1, sh2;
+};
+
+__device__ __forceinline__ uint32_t div_invariant(uint32_t n, const InvariantDiv& d) {
+  const uint32_t t = __umulhi(n, d.m);
+  return (t + ((n - t) >> d.sh1)) >> d.sh2;
+}
+
+// fp32 bits of (e4m3 value of the byte in bits 24..31 of c) * 2^-120: an
+// arithmetic shift by 4 moves the 7 magnitude bits to 26..20 (exponent field
+// e, mantissa m of e4m3 become the low exponent bits and top mantissa bits of
+// fp32, which re-biases 7 -> 127) and the clear removes the sign's copies.
+// Exact for normal and subnormal codes; the NaN codes are handled apart.
+__device__ __forceinline__ float e4m3_times_2m120(uint32_t c_top) {
+  return __uint_as_float(static_cast<uint32_t>(static_cast<int32_t>(c_top) >> 4) & 0x87FFFFFFu);
+}
+
+// Nonzero when one of the four code bytes of w is a NaN code (0x7F or 0xFF).
+__device__ __forceinline__ uint32_t has_nan_code(uint32_t w) {
+  return ((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
+}
+
+// Contiguous weights: thread-chunks of 16 codes (one 16-byte load).  The fast
+// path multiplies the shifted decode by s * 2^120, which is exact while
+// |s| < 2^7 (the product of the real factors is q * s, rounded once, as in
+// fl32(decode(q) * s)); chunks with a larger or non-finite scale, or with a
+// NaN code, take the integer decode of e4m3_value.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
                           void* __restrict__ y, uint32_t total_chunks, uint32_t chunks_per_row,
-                          int64_t nbn) {
+                          InvariantDiv row_div, int64_t nbn) {
   const uint32_t stride = gridDim.x * kDeqThreads * kDeqUnroll;
   for (uint32_t c0 = blockIdx.x * kDeqThreads * kDeqUnroll + threadIdx.x; c0 < total_chunks;
        c0 += stride) {
@@ -234,7 +280,7 @@ __global__ void __launch_bounds__(kDeqThreads)
     for (int u = 0; u < kDeqUnroll; ++u) {
       const uint32_t c = c0 + u * kDeqThreads;
       if (c < total_chunks) {
-        const uint32_t row = c / chunks_per_row;
+        const uint32_t row = div_invariant(c, row_div);
         const uint32_t col = (c - row * chunks_per_row) * 16;
         off[u] = static_cast<int64_t>(c) * 16;
         raw[u] = __ldcs(reinterpret_cast<const uint4*>(q + off[u]));
@@ -247,17 +293,28 @@ __global__ void __launch_bounds__(kDeqThreads)
     for (int u = 0; u < kDeqUnroll; ++u) {
       if (off[u] < 0) continue;
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      float2 v[8];
+      float v[16];
+      const bool fast = fabsf(sc[u]) < 128.0f &&
+                        (has_nan_code(w[0]) | has_nan_code(w[1]) | has_nan_code(w[2]) |
+                         has_nan_code(w[3])) == 0u;
+      if (fast) {
+        const float sc_up = sc[u] * 0x1p120f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t pair = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-        v[j] = make_float2(e4m3_value(pair & 0xFFu) * sc[u], e4m3_value(pair >> 8) * sc[u]);
+        for (int j = 0; j < 4; ++j) {
+          v[4 * j + 0] = e4m3_times_2m120(w[j] << 24) * sc_up;
+          v[4 * j + 1] = e4m3_times_2m120(__byte_perm(w[j], 0u, 0x1444u)) * sc_up;
+          v[4 * j + 2] = e4m3_times_2m120(__byte_perm(w[j], 0u, 0x2444u)) * sc_up;
+          v[4 * j + 3] = e4m3_times_2m120(w[j] & 0xFF000000u) * sc_up;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = e4m3_value((w[j >> 2] >> (8 * (j & 3))) & 0xFFu) * sc[u];
       }
       if (OUT_BF16) {
         uint32_t h[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 b2 = __float22bfloat162_rn(v[j]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
           h[j] = *reinterpret_cast<uint32_t*>(&b2);
         }
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + off[u]);
@@ -267,7 +324,7 @@ __global__ void __launch_bounds__(kDeqThreads)
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + off[u]);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          __stcs(dst + j, make_float4(v[2 * j].x, v[2 * j].y, v[2 * j + 1].x, v[2 * j + 1].y));
+          __stcs(dst + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
       }
     }
   }

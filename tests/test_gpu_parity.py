@@ -153,6 +153,34 @@ def test_weight_dequant_bit_exact(shape, out):
         assert np.array_equal(got, y_ref)
 
 
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_weight_dequant_every_code_and_scale_range(out):
+    """All 256 codes (NaN codes 0x7F/0xFF included) against scales that span
+    the kernel's two decode routes: |s| < 128 (shifted decode times s * 2^120),
+    |s| >= 128 (integer decode), and a subnormal and a negative scale.
+    Non-NaN outputs bit-exact; NaN exactly where the oracle has NaN."""
+    M, N = 256, 1024
+    q = (np.arange(M * N, dtype=np.int64) % 256).astype(np.uint8).reshape(M, N)
+    q[1::2] = q[1::2, ::-1]
+    s = np.array([[1.0, -3.5e-3, 127.99, 128.0, 3.0e30, 1e-40, 2.0 ** -20, 448.0],
+                  [448.0, 2.0 ** -20, 1e-40, 3.0e30, 128.0, 127.99, -3.5e-3, 1.0]],
+                 dtype=np.float32)
+    y = fp8bs.weight_dequant(cuda_codes(q), cuda_f32(s), 128,
+                             torch.bfloat16 if out == "bf16" else torch.float32)
+    y_ref = oracle.weight_dequant(q, s, out=out)
+    if out == "bf16":
+        got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+        as_f = lambda b: (b.astype(np.uint32) << 16).view(np.float32)
+        g, r = as_f(got), as_f(y_ref)
+    else:
+        got = y.cpu().numpy()
+        g, r = got, y_ref
+    assert np.array_equal(np.isnan(g), np.isnan(r))
+    fin = ~np.isnan(r)
+    assert fin.mean() > 0.99
+    assert np.array_equal(f32bits(g[fin]), f32bits(r[fin]))
+
+
 def test_weight_dequant_pages_example_shape():
     q = _codes(1024, 1024, seed=5)
     s = wl.uniform((8, 8), 1e-5, 1e-3, seed=6).numpy()
