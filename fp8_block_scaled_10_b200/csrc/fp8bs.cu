@@ -208,6 +208,37 @@ fp8bs_status make_tmap_y(CUtensorMap* map, const void* y, int64_t rows, int64_t 
   return FP8BS_OK;
 }
 
+// Launches a library kernel with programmatic stream serialization: it may
+// start while the previous kernel of the stream finishes (every kernel here
+// waits for that kernel before touching global memory, and lets the next one
+// start early), which overlaps launch latency and prologues across the
+// act_quant -> GEMM -> split-K reduction chain.  `cluster` > 1 adds a
+// cluster dimension (CTA pairs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
+                   int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(n);
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Multiplier and shifts of div_invariant for a divisor d >= 1.
 InvariantDiv invariant_div(uint32_t d) {
   uint32_t l = 0;
@@ -299,21 +330,8 @@ template <int BN, bool G, bool PAIR>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                         const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::Cfg<BN, PAIR>;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(C::kThreads);
-  cfg.dynamicSmemBytes = C::smem_bytes(G);
-  cfg.stream = st;
-  if (PAIR) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  return cudaLaunchKernelEx(&cfg, gemm::fp8_gemm_kernel<BN, G, PAIR>, ta, tw, ty, p);
+  return launch(gemm::fp8_gemm_kernel<BN, G, PAIR>, grid, C::kThreads, C::smem_bytes(G), st,
+                PAIR ? 2 : 1, ta, tw, ty, p);
 }
 
 template <bool G>
@@ -377,9 +395,9 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    splitk_reduce_kernel<<<grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st>>>(
+    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st, 1,
         static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+    if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
   return FP8BS_OK;
 }
@@ -388,8 +406,8 @@ template <int BN, bool G>
 cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                            const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::BsCfg<BN>;
-  gemm::fp8_gemm_bs_kernel<BN, G><<<grid, C::kThreads, C::smem_bytes(G), st>>>(ta, tw, ty, p);
-  return cudaGetLastError();
+  return launch(gemm::fp8_gemm_bs_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, 1, ta,
+                tw, ty, p);
 }
 
 // Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel, without
@@ -433,9 +451,9 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    splitk_reduce_kernel<<<grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st>>>(
+    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st, 1,
         static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+    if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
   return FP8BS_OK;
 }
@@ -462,16 +480,16 @@ fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int
   // (kActThreads / kActLanes) blocks per CTA per unroll step; up to 8 CTAs per SM.
   const int grid = grid_for(nblocks, (kActThreads / kActLanes) * kActUnroll, info->sms * 8);
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
+  cudaError_t e;
   if (x_dtype == FP8BS_DTYPE_BF16) {
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
-    if (ue) act_quant_kernel<__nv_bfloat16, true><<<grid, kActThreads, 0, st>>>(xb, q, s, nblocks);
-    else act_quant_kernel<__nv_bfloat16, false><<<grid, kActThreads, 0, st>>>(xb, q, s, nblocks);
+    e = ue ? launch(act_quant_kernel<__nv_bfloat16, true>, grid, kActThreads, 0, st, 1, xb, q, s, nblocks)
+           : launch(act_quant_kernel<__nv_bfloat16, false>, grid, kActThreads, 0, st, 1, xb, q, s, nblocks);
   } else {
     const auto* xf = static_cast<const float*>(x);
-    if (ue) act_quant_kernel<float, true><<<grid, kActThreads, 0, st>>>(xf, q, s, nblocks);
-    else act_quant_kernel<float, false><<<grid, kActThreads, 0, st>>>(xf, q, s, nblocks);
+    e = ue ? launch(act_quant_kernel<float, true>, grid, kActThreads, 0, st, 1, xf, q, s, nblocks)
+           : launch(act_quant_kernel<float, false>, grid, kActThreads, 0, st, 1, xf, q, s, nblocks);
   }
-  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return FP8BS_OK;
 }
@@ -539,19 +557,21 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
   cudaStream_t st = as_stream(stream);
   const int64_t nbn = (N + 127) / 128;
   const bool bf = y_dtype == FP8BS_DTYPE_BF16;
+  cudaError_t e;
   if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
     const uint32_t cpr = static_cast<uint32_t>(N / 16);
     const uint32_t total = static_cast<uint32_t>(M * (N / 16));
     const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
     const InvariantDiv row_div = invariant_div(cpr);
-    if (bf) weight_dequant_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, row_div, nbn);
-    else weight_dequant_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, total, cpr, row_div, nbn);
+    e = bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, 1, q, s, y, total, cpr,
+                    row_div, nbn)
+           : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, 1, q, s, y, total, cpr,
+                    row_div, nbn);
   } else {
     const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
-    if (bf) weight_dequant_any_kernel<true><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);
-    else weight_dequant_any_kernel<false><<<grid, kDeqThreads, 0, st>>>(q, s, y, M, N, nbn);
+    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, 1, q, s, y, M, N, nbn)
+           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, 1, q, s, y, M, N, nbn);
   }
-  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "weight_dequant launch");
   return FP8BS_OK;
 }
@@ -576,12 +596,13 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
   const dim3 grid(static_cast<unsigned>(cb), static_cast<unsigned>(rb));
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   cudaStream_t st = as_stream(stream);
+  cudaError_t e;
   if (w_dtype == FP8BS_DTYPE_F32)
-    weight_quant_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(w), q, s, M, N, cb, ue);
+    e = launch(weight_quant_kernel<float>, grid, 256, 0, st, 1, static_cast<const float*>(w), q, s,
+               M, N, cb, ue);
   else
-    weight_quant_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue);
-  const cudaError_t e = cudaGetLastError();
+    e = launch(weight_quant_kernel<__nv_bfloat16>, grid, 256, 0, st, 1,
+               static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue);
   if (e != cudaSuccess) return cuda_fail(e, "weight_quant launch");
   return FP8BS_OK;
 }

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
   const uint32_t rank = PAIR ? cluster_rank() : 0u;   // 0 = leader
   const int unit_start = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
@@ -280,6 +281,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
       tmem_relinquish();
     }
   }
+  // Inputs may come from the previous kernel of the stream (launched with
+  // programmatic serialization): wait for it before any global access.
+  pdl_wait();
   if (GROUPED) {
     // Clamp the device offsets to [0, M], count each group's m tiles and form
     // their exclusive prefix sum (warp 2, 32 groups per step).

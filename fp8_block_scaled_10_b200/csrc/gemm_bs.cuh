@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
   const int unit_start = static_cast<int>(blockIdx.x);
   const int unit_step = static_cast<int>(gridDim.x);
 
@@ -136,6 +137,9 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
+  // Inputs may come from the previous kernel of the stream (launched with
+  // programmatic serialization): wait for it before any global access.
+  pdl_wait();
   if (GROUPED) {
     if (warp == 2) {
       int carry = 0;

@@ -20,6 +20,8 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include "sm100.cuh"
+
 namespace fp8bs {
 
 // ---------------------------------------------------------------------------
@@ -161,6 +163,8 @@ template <typename T, bool UE8M0>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const T* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
                      int64_t nblocks) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int group = lane / kActLanes;
   const int li = lane % kActLanes;
@@ -270,6 +274,8 @@ __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
                           void* __restrict__ y, uint32_t total_chunks, uint32_t chunks_per_row,
                           InvariantDiv row_div, int64_t nbn) {
+  pdl_trigger();
+  pdl_wait();
   const uint32_t stride = gridDim.x * kDeqThreads * kDeqUnroll;
   for (uint32_t c0 = blockIdx.x * kDeqThreads * kDeqUnroll + threadIdx.x; c0 < total_chunks;
        c0 += stride) {
@@ -335,6 +341,8 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_any_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
                               void* __restrict__ y, int64_t M, int64_t N, int64_t nbn) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t total = M * N;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDeqThreads + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * kDeqThreads) {
@@ -365,6 +373,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
     weight_quant_kernel(const T* __restrict__ w, uint8_t* __restrict__ q, float* __restrict__ s,
                         int64_t M, int64_t N, int64_t nbn, bool ue8m0) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[8];
   const int64_t bi = blockIdx.y, bj = blockIdx.x;
   const int64_t r0 = bi * 128, c0 = bj * 128;
@@ -398,6 +408,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     splitk_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ y,
                          int64_t MN, int splits) {
+  pdl_trigger();
+  pdl_wait();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < MN;
        i += static_cast<int64_t>(gridDim.x) * 256) {
     float acc = 0.0f;

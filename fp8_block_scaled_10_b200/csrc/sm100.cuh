@@ -29,6 +29,20 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before the previous kernel of the stream has
+// finished; pdl_wait() blocks until that kernel has completed and its writes
+// are visible, so it precedes every read of inputs another kernel may write.
+// pdl_trigger() lets the next such kernel start its own prologue early.
+// Without a programmatic dependency both return at once.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
