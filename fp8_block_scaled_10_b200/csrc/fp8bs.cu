@@ -186,25 +186,43 @@ static_assert(gemm::Cfg<128, true>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 
-// bf16 y [rows, cols] for the GEMM epilogue's TMA stores: boxes of 32 rows x
-// 32 columns in the 64-byte swizzle the epilogue stages them in.  Usable when
-// the row pitch is a multiple of 16 bytes (cols % 8 == 0); otherwise *map is
-// zeroed and the kernel stores directly (y_tma = 0).
-fp8bs_status make_tmap_y(CUtensorMap* map, const void* y, int64_t rows, int64_t cols,
-                         bool enable, int* y_tma) {
+// Output map of the GEMM epilogue's TMA stores.  One split: bf16 y [rows,
+// cols] in boxes of 32 rows x 32 columns (needs cols % 8 == 0, a 16-byte row
+// pitch).  Several: the FP32 workspace [splits][rows][cols] in boxes of 32
+// rows x 16 columns of one split (needs cols % 4 == 0), so rows past M are
+// clipped inside each split.  Both in the 64-byte swizzle the epilogue stages
+// them in.  Otherwise *map is zeroed and the kernel stores directly
+// (y_tma = 0).
+fp8bs_status make_tmap_out(CUtensorMap* map, const void* y, const void* ws, int64_t rows,
+                           int64_t cols, int splits, int* y_tma) {
   memset(map, 0, sizeof(*map));
   *y_tma = 0;
-  if (!enable || cols % 8 != 0) return FP8BS_OK;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
-  const cuuint32_t box[2] = {32u, 32u};
-  const cuuint32_t elem[2] = {1u, 1u};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(y), dims,
-                              strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (y) failed (%d)", (int)r);
-  *y_tma = 1;
+  CUresult r;
+  if (splits == 1) {
+    if (cols % 8 != 0) return FP8BS_OK;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+    const cuuint32_t box[2] = {32u, 32u};
+    const cuuint32_t elem[2] = {1u, 1u};
+    r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(y), dims, strides, box,
+                 elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (y) failed (%d)", (int)r);
+    *y_tma = 1;
+    return FP8BS_OK;
+  }
+  if (cols % 4 != 0) return FP8BS_OK;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(splits)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4u,
+                                 static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * 4u};
+  const cuuint32_t box[3] = {16u, 32u, 1u};
+  const cuuint32_t elem[3] = {1u, 1u, 1u};
+  r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ws), dims, strides, box,
+               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (ws) failed (%d)", (int)r);
+  *y_tma = 2;
   return FP8BS_OK;
 }
 
@@ -269,20 +287,25 @@ double wave_efficiency(int64_t units, int slots) {
   return static_cast<double>(units) / static_cast<double>(waves * slots);
 }
 
-// Chooses tile width, CTA pairing and K split.  The score is the fraction of
-// persistent slots (SMs, or CTA pairs) kept busy over the waves of work
-// units, weighted by what each shape costs beyond its MMAs: a CTA pair moves
-// a third fewer operand bytes, and each extra split adds a reduction pass
-// over the output.  When several 128-row tiles share each W tile (M >= 256)
-// the kernel is bound by the shared-memory operand feed (about 70 B per SM
-// clock from L2): one K block of a 128 x 256 tile moves 48 KB in ~690 clocks,
-// of a 128 x 128 tile 32 KB in ~470 clocks for half the MMA work, so a
-// 128-wide tile runs at ~0.75 of the 256-wide rate.  Below that, the weight
-// stream from HBM bounds both widths alike.
+// Chooses tile width, CTA pairing and K split.
+//
+// M > 128 (several 128-row tiles share each W tile): the kernel is bound by
+// its operand feed from L2 (about 70 B per SM clock), so a K block of a
+// 128 x 256 tile (48 KB) takes ~0.5 us and one of a 128 x 128 tile (32 KB,
+// half the MMA work) ~2/3 of that.  The plan minimises the estimated time:
+// waves of work units x K blocks per unit x time per K block, plus, for a K
+// split, the FP32 partials' round trip through HBM and the reduction launch.
+//
+// M <= 128 (decode): the weight stream from HBM bounds every tile width
+// alike; the score is the fraction of persistent slots kept busy, with a
+// small cost per split, preferring wider tiles, and CTA pairs weighted by the
+// third fewer operand bytes they move.
 Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_pair = true) {
   Plan best{};
   double best_score = -1.0;
+  double best_time = 1e30;
   const int kbn = static_cast<int>(K / 128);
+  const bool compute_bound = M > 128;
   for (int pair = 0; pair <= 1; ++pair) {
     if (pair && (!allow_pair || !d.pair_enabled || d.pair_slots <= 0 || M <= 128)) continue;
     const int slots = pair ? d.pair_slots : d.sms;
@@ -298,14 +321,25 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_
         const int splits = (kbn + per - 1) / per;
         if (splits != s) continue;
         const int64_t units = tiles * splits;
-        const double eff = wave_efficiency(units, slots);
-        // Useful rows per unit when M is smaller than the unit.
-        const double fill = static_cast<double>(std::min<int64_t>(M, rows)) / rows;
-        const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? (M >= 256 ? 0.75 : 0.97) : 1.0);
-        const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
-        const double score = eff * feed * split_cost * (M < rows ? fill + 0.5 * (1 - fill) : 1.0);
-        if (score > best_score + 1e-9) {
-          best_score = score;
+        bool better;
+        if (compute_bound) {
+          const double kb_us = (bn == 256 ? 0.5 : 1.0 / 3.0) * (rows / 128.0) / (pair ? 1.15 : 1.0);
+          const double waves = static_cast<double>((units + slots - 1) / slots);
+          double t = waves * per * kb_us;
+          if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
+            t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
+          better = t < best_time - 1e-9;
+          if (better) best_time = t;
+        } else {
+          const double eff = wave_efficiency(units, slots);
+          const double fill = static_cast<double>(std::min<int64_t>(M, rows)) / rows;
+          const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? 0.97 : 1.0);
+          const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
+          const double score = eff * feed * split_cost * (fill + 0.5 * (1 - fill));
+          better = score > best_score + 1e-9;
+          if (better) best_score = score;
+        }
+        if (better) {
           const int grid_units = static_cast<int>(std::min<int64_t>(units, slots));
           best = Plan{bn, pair != 0, m_tiles, n_tiles, splits, per, static_cast<int>(units),
                       pair ? 2 * grid_units : grid_units};
@@ -375,7 +409,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, w_box_rows(pl.bn, pl.pair))) != FP8BS_OK) return r;
-  if ((r = make_tmap_y(&ty, y, M, N, pl.splits == 1, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -430,7 +464,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
-  if ((r = make_tmap_y(&ty, y, M, N, pl.splits == 1, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -766,7 +800,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
-  if ((r = make_tmap_y(&ty, y, M_total, N, true, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, nullptr, M_total, N, 1, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
@@ -824,7 +858,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, G * N, K, w_box_rows(bn, pair))) != FP8BS_OK) return r;
-  if ((r = make_tmap_y(&ty, y, M_total, N, true, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, nullptr, M_total, N, 1, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);

@@ -68,7 +68,8 @@ struct Params {
   int kb_per_split;
   int num_units;            // dense mode; grouped mode derives it on the device
   int groups;               // grouped mode
-  int y_tma;                // 1: bf16 y written by TMA stores through staging boxes
+  int y_tma;                // 1: bf16 y written by TMA stores through staging boxes;
+                            // 2: FP32 split-K partials written by TMA stores (3-D map)
 };
 
 // Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
@@ -84,11 +85,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&b2);
 }
 
-// Stages this lane's 32 packed bf16 values as row `lane` of the warp's box and
-// stores the box at column x, row y of y.  Lane 0 first waits until the
-// box's previous store has read it.
-__device__ __forceinline__ void store_out_box(const CUtensorMap* tmap_y, uint8_t* box, int lane,
-                                              const uint32_t (&h)[16], int32_t x, int32_t y) {
+// Stages this lane's 64 bytes (32 packed bf16, or 16 FP32 split-K partials)
+// as row `lane` of the warp's box and stores the box at column x, row y of y
+// (2-D map), or of split z of the FP32 workspace (3-D map, z >= 0).  Lane 0
+// first waits until the box's previous store has read it.
+__device__ __forceinline__ void store_out_box(const CUtensorMap* tmap, uint8_t* box, int lane,
+                                              const uint32_t (&h)[16], int32_t x, int32_t y,
+                                              int32_t z = -1) {
   if (lane == 0) tma_store_wait_read();
   __syncwarp();
 #pragma unroll
@@ -98,7 +101,8 @@ __device__ __forceinline__ void store_out_box(const CUtensorMap* tmap_y, uint8_t
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(tmap_y, box, x, y);
+    if (z < 0) tma_store_2d(tmap, box, x, y);
+    else tma_store_3d(tmap, box, x, y, z);
     tma_store_commit();
   }
 }
@@ -506,7 +510,23 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
       }
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
       const int64_t slab0 = t.row0 + static_cast<int64_t>(rank) * BM + quad * 32;
-      if (p.y_tma && slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end)) {
+      const bool slab_tma = slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end);
+      if (p.y_tma == 2 && slab_tma) {
+        // FP32 split-K partials of split t.split, 16 columns per box.
+        uint8_t* box = out_boxes + e * kOutBoxBytes;
+#pragma unroll
+        for (int c = 0; c < CPW / 16; ++c) {
+          if (col0 + 16 * c >= p.N) break;
+          uint32_t w16[16];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            w16[2 * j] = __float_as_uint(acc[c * 8 + j].x);
+            w16[2 * j + 1] = __float_as_uint(acc[c * 8 + j].y);
+          }
+          store_out_box(&tmap_y, box, lane, w16, static_cast<int32_t>(col0 + 16 * c),
+                        static_cast<int32_t>(slab0), t.split);
+        }
+      } else if (p.y_tma == 1 && slab_tma) {
         // Staged TMA stores; rows past M and columns past N are clipped.
         uint8_t* box = out_boxes + e * kOutBoxBytes;
 #pragma unroll

@@ -421,7 +421,11 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
           }
         }
       } else {
-        // FP32 split-K partials, chunk by chunk.
+        // FP32 split-K partials, chunk by chunk: staged TMA stores into split
+        // t.split of the workspace (rows past M clipped), else direct stores.
+        const int64_t slab0 = t.row0 + quad * 32;
+        const bool slab_tma = p.y_tma == 2 && slab0 < t.row_end;
+        uint8_t* box = out_boxes + e * kOutBoxBytes;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           uint32_t v[32];
@@ -432,8 +436,20 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[tb]);
           }
-          if (!row_ok) continue;
           const int64_t col = col0 + 32 * c;
+          if (slab_tma) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if (col + 16 * hh >= p.N) break;
+              uint32_t w16[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) w16[j] = v[16 * hh + j];
+              store_out_box(&tmap_y, box, lane, w16, static_cast<int32_t>(col + 16 * hh),
+                            static_cast<int32_t>(slab0), t.split);
+            }
+            continue;
+          }
+          if (!row_ok) continue;
           float* wrow = p.ws + (static_cast<int64_t>(t.split) * p.M + row) * p.N;
           if ((p.N % 4) == 0 && col + 32 <= p.N) {
 #pragma unroll
