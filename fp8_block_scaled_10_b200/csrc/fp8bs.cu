@@ -44,10 +44,6 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
-  int pair_slots = 0;   // CTA pairs (clusters of two) that can be resident at once
-  // CTA-pair GEMM tiles are correct but measured slower than single-CTA tiles
-  // on B200 so far; FP8BS_GEMM_PAIR=1 lets the planner consider them.
-  bool pair_enabled = false;
 };
 
 std::mutex g_mu;
@@ -62,30 +58,13 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G, bool PAIR>
-fp8bs_status setup_gemm_kernel(DeviceInfo& d) {
-  using C = gemm::Cfg<BN, PAIR>;
-  auto kernel = gemm::fp8_gemm_kernel<BN, G, PAIR>;
+template <int BN, bool G>
+fp8bs_status setup_gemm_kernel() {
+  using C = gemm::Cfg<BN>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-  if (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * d.sms);
-    cfg.blockDim = dim3(C::kThreads);
-    cfg.dynamicSmemBytes = C::smem_bytes(G);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-    d.pair_slots = d.pair_slots == 0 ? clusters : std::min(d.pair_slots, clusters);
-  }
   if (C::kSplitRegs) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, kernel);
@@ -126,21 +105,15 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
     if (major != 10 || minor != 0)
       return fail(FP8BS_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
                   dev, major, minor);
-    {
-      const char* env = getenv("FP8BS_GEMM_PAIR");
-      d.pair_enabled = env != nullptr && env[0] == '1';
-    }
     e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     fp8bs_status r;
-    if ((r = setup_gemm_kernel<128, false, false>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, false, false>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<128, true, false>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, true, false>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<128, false, true>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, false, true>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<128, true, true>(d)) != FP8BS_OK ||
-        (r = setup_gemm_kernel<256, true, true>(d)) != FP8BS_OK ||
+    if ((r = setup_gemm_kernel<128, false>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<192, false>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<192, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, true>()) != FP8BS_OK ||
@@ -179,10 +152,9 @@ fp8bs_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
 
 // Every GEMM configuration fits the 227 KB of shared memory a CTA can opt into.
 constexpr int kMaxSmemOptin = 227 * 1024;
-static_assert(gemm::Cfg<256, false>::smem_bytes(true) <= kMaxSmemOptin, "smem");
-static_assert(gemm::Cfg<128, false>::smem_bytes(true) <= kMaxSmemOptin, "smem");
-static_assert(gemm::Cfg<256, true>::smem_bytes(true) <= kMaxSmemOptin, "smem");
-static_assert(gemm::Cfg<128, true>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<192>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 
@@ -230,24 +202,16 @@ fp8bs_status make_tmap_out(CUtensorMap* map, const void* y, const void* ws, int6
 // start while the previous kernel of the stream finishes (every kernel here
 // waits for that kernel before touching global memory, and lets the next one
 // start early), which overlaps launch latency and prologues across the
-// act_quant -> GEMM -> split-K reduction chain.  `cluster` > 1 adds a
-// cluster dimension (CTA pairs).
+// act_quant -> GEMM -> split-K reduction chain.
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
-                   int cluster, Args&&... args) {
+                   Args&&... args) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   int n = 0;
   attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[n].val.programmaticStreamSerializationAllowed = 1;
   ++n;
-  if (cluster > 1) {
-    attr[n].id = cudaLaunchAttributeClusterDimension;
-    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
-    attr[n].val.clusterDim.y = 1;
-    attr[n].val.clusterDim.z = 1;
-    ++n;
-  }
   cfg.gridDim = grid;
   cfg.blockDim = dim3(static_cast<unsigned>(block));
   cfg.dynamicSmemBytes = smem;
@@ -275,11 +239,10 @@ int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
 // ---------------------------------------------------------------------------
 struct Plan {
   int bn;
-  bool pair;
   int m_tiles, n_tiles;
   int splits, kb_per_split;
   int units;
-  int grid;   // CTAs (twice the clusters in pair mode)
+  int grid;   // persistent CTAs
 };
 
 double wave_efficiency(int64_t units, int slots) {
@@ -287,95 +250,94 @@ double wave_efficiency(int64_t units, int slots) {
   return static_cast<double>(units) / static_cast<double>(waves * slots);
 }
 
-// Chooses tile width, CTA pairing and K split.
+// The two GEMM kernels the planner serves.
+enum class GemmKind { kPromotion, kBlockScaled };
+
+// Time per K block of one 128-row work unit, in microseconds, measured on
+// B200 at M = 4096 with every SM busy.
+//   promotion kernel: 128 x 256 tile ~0.55, 128 x 192 ~0.48, 128 x 128
+//     ~0.36 (the tensor core and the epilogue's FP32 promotion overlap; the
+//     wider tile moves fewer operand bytes per FLOP);
+//   block-scaled kernel: 128 x 256 ~0.5, 128 x 128 ~1/3 (operand feed).
+double kb_time_us(GemmKind kind, int bn) {
+  if (kind == GemmKind::kPromotion) return bn == 256 ? 0.55 : (bn == 192 ? 0.48 : 0.36);
+  return bn == 256 ? 0.5 : 1.0 / 3.0;
+}
+
+// Chooses tile width and K split.
 //
-// M > 128 (several 128-row tiles share each W tile): the kernel is bound by
-// its operand feed from L2 (about 70 B per SM clock), so a K block of a
-// 128 x 256 tile (48 KB) takes ~0.5 us and one of a 128 x 128 tile (32 KB,
-// half the MMA work) ~2/3 of that.  The plan minimises the estimated time:
-// waves of work units x K blocks per unit x time per K block, plus, for a K
-// split, the FP32 partials' round trip through HBM and the reduction launch.
+// M > 128 (several 128-row tiles share each W tile): the estimated time is
+// waves of work units x K blocks per unit x kb_time_us, plus, for a K split,
+// the FP32 partials' round trip through HBM and the reduction launch.
 //
 // M <= 128 (decode): the weight stream from HBM bounds every tile width
 // alike; the score is the fraction of persistent slots kept busy, with a
-// small cost per split, preferring wider tiles, and CTA pairs weighted by the
-// third fewer operand bytes they move.
-Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d, bool allow_pair = true) {
+// small cost per split, preferring wider tiles.
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
+               GemmKind kind = GemmKind::kPromotion) {
   Plan best{};
   double best_score = -1.0;
   double best_time = 1e30;
   const int kbn = static_cast<int>(K / 128);
   const bool compute_bound = M > 128;
-  for (int pair = 0; pair <= 1; ++pair) {
-    if (pair && (!allow_pair || !d.pair_enabled || d.pair_slots <= 0 || M <= 128)) continue;
-    const int slots = pair ? d.pair_slots : d.sms;
-    const int rows = pair ? 256 : 128;
-    for (int bn : {256, 128}) {
-      const int m_tiles = static_cast<int>((M + rows - 1) / rows);
-      const int n_tiles = static_cast<int>((N + bn - 1) / bn);
-      const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
-      // Split K only when the tiles alone cannot fill the GPU.
-      const int max_split = tiles >= slots ? 1 : std::min(16, std::max(1, kbn / 4));
-      for (int s = 1; s <= max_split; ++s) {
-        const int per = (kbn + s - 1) / s;
-        const int splits = (kbn + per - 1) / per;
-        if (splits != s) continue;
-        const int64_t units = tiles * splits;
-        bool better;
-        if (compute_bound) {
-          const double kb_us = (bn == 256 ? 0.5 : 1.0 / 3.0) * (rows / 128.0) / (pair ? 1.15 : 1.0);
-          const double waves = static_cast<double>((units + slots - 1) / slots);
-          double t = waves * per * kb_us;
-          if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
-            t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
-          better = t < best_time - 1e-9;
-          if (better) best_time = t;
-        } else {
-          const double eff = wave_efficiency(units, slots);
-          const double fill = static_cast<double>(std::min<int64_t>(M, rows)) / rows;
-          const double feed = (pair ? 1.15 : 1.0) * (bn == 128 ? 0.97 : 1.0);
-          const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
-          const double score = eff * feed * split_cost * (fill + 0.5 * (1 - fill));
-          better = score > best_score + 1e-9;
-          if (better) best_score = score;
-        }
-        if (better) {
-          const int grid_units = static_cast<int>(std::min<int64_t>(units, slots));
-          best = Plan{bn, pair != 0, m_tiles, n_tiles, splits, per, static_cast<int>(units),
-                      pair ? 2 * grid_units : grid_units};
-        }
+  const int slots = d.sms;
+  for (int bn : {256, 192, 128}) {
+    if (bn == 192 && (kind != GemmKind::kPromotion || !compute_bound)) continue;
+    const int m_tiles = static_cast<int>((M + 127) / 128);
+    const int n_tiles = static_cast<int>((N + bn - 1) / bn);
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    // Split K only when the tiles alone cannot fill the GPU.
+    const int max_split = tiles >= slots ? 1 : std::min(16, std::max(1, kbn / 4));
+    for (int s = 1; s <= max_split; ++s) {
+      const int per = (kbn + s - 1) / s;
+      const int splits = (kbn + per - 1) / per;
+      if (splits != s) continue;
+      const int64_t units = tiles * splits;
+      bool better;
+      if (compute_bound) {
+        const double kb_us = kb_time_us(kind, bn);
+        const double waves = static_cast<double>((units + slots - 1) / slots);
+        double t = waves * per * kb_us;
+        if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
+          t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
+        better = t < best_time - 1e-9;
+        if (better) best_time = t;
+      } else {
+        const double eff = wave_efficiency(units, slots);
+        const double fill = static_cast<double>(std::min<int64_t>(M, 128)) / 128;
+        const double feed = bn == 128 ? 0.97 : 1.0;
+        const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
+        const double score = eff * feed * split_cost * (fill + 0.5 * (1 - fill));
+        better = score > best_score + 1e-9;
+        if (better) best_score = score;
       }
+      if (better)
+        best = Plan{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units),
+                    static_cast<int>(std::min<int64_t>(units, slots))};
     }
   }
   return best;
-}
-
-// Rows of one W load box: the per-CTA chunk of one sub-MMA's W rows.
-int w_box_rows(int bn, bool pair) {
-  return bn == 256 ? (pair ? gemm::Cfg<256, true>::kBChunkRows : gemm::Cfg<256, false>::kBChunkRows)
-                   : (pair ? gemm::Cfg<128, true>::kBChunkRows : gemm::Cfg<128, false>::kBChunkRows);
 }
 
 size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
-template <int BN, bool G, bool PAIR>
+template <int BN, bool G>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                         const gemm::Params& p, int grid, cudaStream_t st) {
-  using C = gemm::Cfg<BN, PAIR>;
-  return launch(gemm::fp8_gemm_kernel<BN, G, PAIR>, grid, C::kThreads, C::smem_bytes(G), st,
-                PAIR ? 2 : 1, ta, tw, ty, p);
+  using C = gemm::Cfg<BN>;
+  return launch(gemm::fp8_gemm_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, ta, tw,
+                ty, p);
 }
 
 template <bool G>
-cudaError_t launch_gemm_any(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tw,
+cudaError_t launch_gemm_any(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
                             const CUtensorMap& ty, const gemm::Params& p, int grid,
                             cudaStream_t st) {
-  if (pair) return bn == 256 ? launch_gemm<256, G, true>(ta, tw, ty, p, grid, st)
-                             : launch_gemm<128, G, true>(ta, tw, ty, p, grid, st);
-  return bn == 256 ? launch_gemm<256, G, false>(ta, tw, ty, p, grid, st)
-                   : launch_gemm<128, G, false>(ta, tw, ty, p, grid, st);
+  return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
+         : bn == 192 ? launch_gemm<192, G>(ta, tw, ty, p, grid, st)
+                     : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
 }
 
 fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
@@ -408,7 +370,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   CUtensorMap ta, tw, ty;
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
-  if ((r = make_tmap(&tw, w, N, K, w_box_rows(pl.bn, pl.pair))) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
   if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
@@ -425,11 +387,11 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
   p.groups = 1;
-  cudaError_t e = launch_gemm_any<false>(pl.bn, pl.pair, ta, tw, ty, p, pl.grid, st);
+  cudaError_t e = launch_gemm_any<false>(pl.bn, ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st, 1,
+    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,
         static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
     if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
@@ -440,12 +402,11 @@ template <int BN, bool G>
 cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                            const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::BsCfg<BN>;
-  return launch(gemm::fp8_gemm_bs_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, 1, ta,
+  return launch(gemm::fp8_gemm_bs_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, ta,
                 tw, ty, p);
 }
 
-// Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel, without
-// CTA pairs.
+// Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel.
 fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
                          int64_t M, int64_t N, int64_t K, uint16_t* y, void* ws, size_t ws_bytes,
                          cudaStream_t st) {
@@ -456,7 +417,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const Plan pl = plan_gemm(M, N, K, *info, false);
+  const Plan pl = plan_gemm(M, N, K, *info, GemmKind::kBlockScaled);
   const size_t need = plan_workspace(pl, M, N);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
@@ -485,7 +446,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st, 1,
+    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,
         static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
     if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
@@ -517,12 +478,12 @@ fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int
   cudaError_t e;
   if (x_dtype == FP8BS_DTYPE_BF16) {
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
-    e = ue ? launch(act_quant_kernel<__nv_bfloat16, true>, grid, kActThreads, 0, st, 1, xb, q, s, nblocks)
-           : launch(act_quant_kernel<__nv_bfloat16, false>, grid, kActThreads, 0, st, 1, xb, q, s, nblocks);
+    e = ue ? launch(act_quant_kernel<__nv_bfloat16, true>, grid, kActThreads, 0, st, xb, q, s, nblocks)
+           : launch(act_quant_kernel<__nv_bfloat16, false>, grid, kActThreads, 0, st, xb, q, s, nblocks);
   } else {
     const auto* xf = static_cast<const float*>(x);
-    e = ue ? launch(act_quant_kernel<float, true>, grid, kActThreads, 0, st, 1, xf, q, s, nblocks)
-           : launch(act_quant_kernel<float, false>, grid, kActThreads, 0, st, 1, xf, q, s, nblocks);
+    e = ue ? launch(act_quant_kernel<float, true>, grid, kActThreads, 0, st, xf, q, s, nblocks)
+           : launch(act_quant_kernel<float, false>, grid, kActThreads, 0, st, xf, q, s, nblocks);
   }
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return FP8BS_OK;
@@ -597,14 +558,14 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
     const uint32_t total = static_cast<uint32_t>(M * (N / 16));
     const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
     const InvariantDiv row_div = invariant_div(cpr);
-    e = bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, 1, q, s, y, total, cpr,
+    e = bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
                     row_div, nbn)
-           : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, 1, q, s, y, total, cpr,
+           : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
                     row_div, nbn);
   } else {
     const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
-    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, 1, q, s, y, M, N, nbn)
-           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, 1, q, s, y, M, N, nbn);
+    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn)
+           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn);
   }
   if (e != cudaSuccess) return cuda_fail(e, "weight_dequant launch");
   return FP8BS_OK;
@@ -632,10 +593,10 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
   if (w_dtype == FP8BS_DTYPE_F32)
-    e = launch(weight_quant_kernel<float>, grid, 256, 0, st, 1, static_cast<const float*>(w), q, s,
+    e = launch(weight_quant_kernel<float>, grid, 256, 0, st, static_cast<const float*>(w), q, s,
                M, N, cb, ue);
   else
-    e = launch(weight_quant_kernel<__nv_bfloat16>, grid, 256, 0, st, 1,
+    e = launch(weight_quant_kernel<__nv_bfloat16>, grid, 256, 0, st,
                static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue);
   if (e != cudaSuccess) return cuda_fail(e, "weight_quant launch");
   return FP8BS_OK;
@@ -679,7 +640,9 @@ size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   int dev;
   DeviceInfo* info;
   if (device_setup(&dev, &info) != FP8BS_OK) return 0;
-  return plan_workspace(plan_gemm(M, N, K, *info), M, N);
+  // One size serves both GEMM entry points (their plans may differ).
+  return std::max(plan_workspace(plan_gemm(M, N, K, *info), M, N),
+                  plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N));
 }
 
 const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
@@ -692,10 +655,9 @@ const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
   }
   const Plan pl = plan_gemm(M, N, K, *info);
   snprintf(buf, sizeof(buf),
-           "bn=%d pair=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d "
-           "sms=%d pair_slots=%d",
-           pl.bn, pl.pair ? 1 : 0, pl.m_tiles, pl.n_tiles, pl.splits, pl.kb_per_split, pl.units,
-           pl.grid, info->sms, info->pair_slots);
+           "bn=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d sms=%d",
+           pl.bn, pl.m_tiles, pl.n_tiles, pl.splits, pl.kb_per_split, pl.units, pl.grid,
+           info->sms);
   return buf;
 }
 
@@ -851,13 +813,17 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const int bn = N >= 256 ? 256 : 128;
-  // CTA pairs when the groups are large enough on average to fill 256-row units.
-  const bool pair = info->pair_enabled && info->pair_slots > 0 && M_total >= 256 * G;
+  // The tile width with the least estimated time per 128-row tile of a group.
+  int bn = 128;
+  for (int cand : {256, 192}) {
+    if (N < cand) continue;
+    const auto cost = [&](int b) { return ((N + b - 1) / b) * kb_time_us(GemmKind::kPromotion, b); };
+    if (cost(cand) < cost(bn) - 1e-9) bn = cand;
+  }
   CUtensorMap ta, tw, ty;
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M_total, K, 128)) != FP8BS_OK) return r;
-  if ((r = make_tmap(&tw, w, G * N, K, w_box_rows(bn, pair))) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, G * N, K, bn)) != FP8BS_OK) return r;
   if ((r = make_tmap_out(&ty, y, nullptr, M_total, N, 1, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
@@ -875,12 +841,9 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   p.num_units = 0;
   p.groups = static_cast<int>(G);
   // Units are only known on the device; an upper bound sizes the grid.
-  const int rows = pair ? 256 : 128;
-  const int64_t max_units = ((M_total + rows - 1) / rows + G) * p.n_tiles;
-  const int slots = pair ? info->pair_slots : info->sms;
-  const int grid_units = static_cast<int>(std::min<int64_t>(max_units, slots));
-  cudaError_t e = launch_gemm_any<true>(bn, pair, ta, tw, ty, p, pair ? 2 * grid_units : grid_units,
-                                        as_stream(stream));
+  const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
+  cudaError_t e = launch_gemm_any<true>(bn, ta, tw, ty, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
   return FP8BS_OK;
 }

@@ -18,19 +18,19 @@
 // Roles (persistent CTAs, one per SM, walking work units in a fixed order):
 //   warp 0     TMA producer: A tile [128 x 128] and W tile into a ring of
 //              shared-memory stages (128B swizzle).
-//   warp 1     owns the TMEM allocation; one lane issues the MMAs.
+//   warps 1, 3 one lane each issues the MMAs of alternate K blocks; warp 1
+//              owns the TMEM allocation.
+//   warp 2     scale producer: for every K block of every unit it loads the
+//              128 activation scales a_s[rows, kb] and the weight scales
+//              w_s[nb, kb] of the tile (four K blocks ahead, in registers)
+//              into a small shared-memory ring that the epilogue reads.  The
+//              epilogue threads would otherwise each wait on a scattered
+//              global load per K block, which measured slower than the drain
+//              of the TMEM partial itself.
 //   epilogue   8 warps from kFirstEpiWarp: warp w reads TMEM lanes
 //              32*(w%4)..+31 (one output row per thread) and BN/2 columns
 //              (column half (w - kFirstEpiWarp) / 4).  Loads of the next
 //              32-column chunk overlap the FMAs of the current one.
-// Pair mode (PAIR): two CTAs of a cluster share one tcgen05.mma.cta_group::2
-// of M = 256.  Each CTA loads its own 128 rows of A and its own half of the W
-// tile (BN/2 rows), so each SM moves a third less operand data per MMA than
-// a single CTA with a 128 x BN tile.  The leader (even) CTA issues the MMAs;
-// both CTAs' loads complete on the leader's full barrier, the leader's commits
-// arrive on both CTAs' barriers, and both CTAs' epilogues release the TMEM
-// buffer on the leader's barrier.  Each CTA holds its own 128 rows of the
-// accumulator in its own TMEM.
 //
 // A work unit is (m tile, n tile, K split).  With one split the epilogue
 // writes bf16; with several it writes FP32 partials that a reduction kernel
@@ -51,6 +51,10 @@ namespace gemm {
 constexpr int BM = 128;      // rows of A per CTA
 constexpr int BK = 128;      // one K block per pipeline stage
 constexpr int kMaxGroups = 1024;
+#ifndef FP8BS_SPIN_WAITS
+#define FP8BS_SPIN_WAITS 0
+#endif
+constexpr bool kSpinWaits = FP8BS_SPIN_WAITS != 0;
 
 struct Params {
   const float* sa;          // [M_total, kbn]
@@ -107,53 +111,56 @@ __device__ __forceinline__ void store_out_box(const CUtensorMap* tmap, uint8_t* 
   }
 }
 
-template <int BN, bool PAIR>
+template <int BN>
 struct Cfg {
-  static constexpr int kUnitRows = PAIR ? 2 * BM : BM;   // rows of one work unit
-  static constexpr int kBRows = PAIR ? BN / 2 : BN;      // W rows loaded per CTA
+  static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
   static constexpr int kABytes = BM * BK;
-  static constexpr int kBBytes = kBRows * BK;
+  static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (6 * 32768) / kStageBytes;
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
   // Two epilogue warpgroups: each covers all 128 TMEM lanes (one warp per
   // 32-lane quadrant) and half of the tile's columns.
   static constexpr int kEpiWarps = 8;
   static constexpr int kColsPerWarp = BN / 2;
   static constexpr int kChunks = kColsPerWarp / 32;
-  // BN = 256: warps 0-3 form a control warpgroup that hands registers to the
-  // two epilogue warpgroups (setmaxnreg); BN = 128: warps 0-1 control, 2-9
-  // epilogue, and every thread can hold its 64 accumulators at launch.
-  static constexpr int kFirstEpiWarp = (BN == 256) ? 4 : 2;
-  static constexpr bool kSplitRegs = (BN == 256);
+  // Warps 0-3 form the control warpgroup (TMA, MMA, scales); for BN >= 192
+  // it hands registers to the two epilogue warpgroups (setmaxnreg), for
+  // BN = 128 every thread can hold its 64 accumulators at launch.
+  // Weight blocks a tile's columns can touch: tiles start at multiples of BN,
+  // so a 128- or 256-wide tile covers whole blocks and a 192-wide tile
+  // straddles at most one block boundary.
+  static constexpr int kNbSpan = BN == 128 ? 1 : 2;
+  // The epilogue releases a TMEM buffer once its columns are in registers.
+  // With at most 96 columns per thread (BN <= 192) all of them are loaded in
+  // one batch, so the release comes one load latency after the MMA finishes;
+  // with 128 (BN = 256) the registers only allow a two-deep chunk pipeline
+  // whose FMAs delay the release.
+  static constexpr bool kOneBatch = BN <= 192;
+  static constexpr int kFirstEpiWarp = 4;
+  static constexpr bool kSplitRegs = (BN >= 192);
   static constexpr int kCtrlRegs = 56;
   static constexpr int kEpiRegs = 224;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-  static constexpr int kTmemCols = 2 * BN;
-  // In pair mode with BN = 256 each K block's MMA is issued as two sub-MMAs of
-  // N = 128, each into its own TMEM sub-buffer with its own full/empty
-  // barrier pair, so the epilogue warps of column half g can drain sub-buffer
-  // g while the tensor core still works on the other half; each sub-MMA takes
-  // 64 rows of W from each CTA, so a CTA loads two chunks of 64 rows per
-  // stage.  (A single CTA keeps one N = BN MMA: two N = 128 MMAs would read
-  // the A tile from shared memory twice.)
-  static constexpr int kSplitN = (PAIR && BN == 256) ? 2 : 1;
-  static constexpr int kSubN = BN / kSplitN;
-  static constexpr int kBChunkRows = PAIR ? kSubN / 2 : kSubN;
-  static constexpr int kBChunkBytes = kBChunkRows * BK;
-  static constexpr int kSubBuffers = 2 * kSplitN;
-  static constexpr int kCtrlBytes = 256;
+  // TMEM partial buffers: as many as the 512 columns hold (2 of 256 columns,
+  // 4 of 128), so the epilogue can lag the tensor core by kAccBufs - 1 K blocks.
+  static constexpr int kAccBufs = 512 / BN;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kCtrlBytes = 512;
+  // Scale ring: per K block the tile's 128 activation scales and its
+  // (BN / 128) weight scales.
+  static constexpr int kScaleSlots = 4;   // >= kAccBufs; slot b goes with TMEM buffer b
+  static constexpr int kScaleSlotBytes = 4 * (BM + 4);
+  static constexpr int kScaleBytes = kScaleSlots * kScaleSlotBytes;
   // grouped mode: per-group m-tile prefix (int)
   static constexpr int kGroupBytes = 4 * (kMaxGroups + 1);
   // output staging boxes (one per epilogue warp), 1024-byte aligned
   __host__ __device__ static constexpr int out_offset(bool grouped) {
-    return (kStages * kStageBytes + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1023) & ~1023;
+    return (kStages * kStageBytes + kCtrlBytes + kScaleBytes + (grouped ? kGroupBytes : 0) +
+            1023) & ~1023;
   }
   __host__ __device__ static constexpr int smem_bytes(bool grouped) {
     return out_offset(grouped) + kEpiWarps * kOutBoxBytes + 1024;
   }
-  // Arrivals that release one TMEM sub-buffer: the epilogue warps that read
-  // it, in both CTAs in pair mode.
-  static constexpr int kTmemReleaseCount = (kEpiWarps / kSplitN) * (PAIR ? 2 : 1);
 };
 
 // Control block at the end of the tile ring.
@@ -161,16 +168,16 @@ template <int kStages>
 struct Ctrl {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tfull[4];     // [buffer * kSplitN + half]
-  uint64_t tempty[4];
-  uint64_t flush;
+  uint64_t tfull[4];     // TMEM partial buffer and its scale slot ready for the epilogue
+  uint64_t tempty[4];    // TMEM partial buffer drained and its scale slot read
+  uint64_t flush[2];     // per MMA issuer: all of its MMAs complete
   uint32_t tmem_base;
   int abort_flag;
   int num_units;
 };
 
 struct Unit {
-  int64_t row0;      // first A/y row of the unit (of the pair in pair mode)
+  int64_t row0;      // first A/y row of the unit
   int64_t row_end;   // rows >= row_end are not stored
   int64_t w_row0;    // first W row (grouped: expert * N + n0)
   int group;
@@ -229,12 +236,12 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   return t;
 }
 
-template <int BN, bool GROUPED, bool PAIR>
-__global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
+template <int BN, bool GROUPED>
+__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w,
                     const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-  using C = Cfg<BN, PAIR>;
+  using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -246,28 +253,34 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
   uint64_t* empty = ctrl->empty;
   uint64_t* tfull = ctrl->tfull;
   uint64_t* tempty = ctrl->tempty;
-  uint64_t* flush = &ctrl->flush;
+  uint64_t* flush = ctrl->flush;
   volatile int* abort_flag = &ctrl->abort_flag;
-  int* tile_prefix = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
+  float* scale_slots =
+      reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
+  int* tile_prefix = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes +
+                                            C::kScaleBytes);
   uint8_t* out_boxes = smem + C::out_offset(GROUPED);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   pdl_trigger();
-  const uint32_t rank = PAIR ? cluster_rank() : 0u;   // 0 = leader
-  const int unit_start = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int unit_start = static_cast<int>(blockIdx.x);
+  const int unit_step = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < C::kSubBuffers; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::kTmemReleaseCount);
+    // tfull[b] completes when the MMA's commit and the scale producer have
+    // both arrived: the partial in TMEM buffer b and the scales of the same
+    // K block in slot b are then ready, so the epilogue waits once per K block.
+    for (int b = 0; b < C::kAccBufs; ++b) {
+      mbar_init(&tfull[b], 2);
+      mbar_init(&tempty[b], C::kEpiWarps);
     }
-    mbar_init(flush, 1);
+    mbar_init(&flush[0], 1);
+    mbar_init(&flush[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -277,13 +290,8 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
     if (p.y_tma) tma_prefetch_descriptor(&tmap_y);
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(&ctrl->tmem_base, C::kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
+    tmem_relinquish();
   }
   // Inputs may come from the previous kernel of the stream (launched with
   // programmatic serialization): wait for it before any global access.
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
         if (g < p.groups) {
           int64_t lo, hi;
           group_rows(p, g, lo, hi);
-          tiles = static_cast<int>((hi - lo + C::kUnitRows - 1) / C::kUnitRows);
+          tiles = static_cast<int>((hi - lo + BM - 1) / BM);
         }
         int incl = tiles;
 #pragma unroll
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
     ctrl->num_units = p.num_units;
   }
   tc_fence_before();
-  if (PAIR) cluster_sync(); else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctrl->tmem_base;
   const int num_units = ctrl->num_units;
@@ -327,10 +335,10 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
   auto unit_of = [&](int u) -> Unit {
     Unit t;
     if (GROUPED) {
-      t = grouped_unit<C::kUnitRows>(p, tile_prefix, u);
+      t = grouped_unit<BM>(p, tile_prefix, u);
       t.w_row0 = static_cast<int64_t>(t.group) * p.N + static_cast<int64_t>(t.n_tile) * BN;
     } else {
-      t = dense_unit<C::kUnitRows>(p, u);
+      t = dense_unit<BM>(p, u);
       t.w_row0 = static_cast<int64_t>(t.n_tile) * BN;
     }
     return t;
@@ -347,30 +355,13 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
       uint32_t armed_phase = 0; // parity each armed stage completes
       for (int u = unit_start; u < num_units; u += unit_step) {
         const Unit t = unit_of(u);
-        const int32_t a_row = static_cast<int32_t>(t.row0 + rank * BM);
-        // W rows of chunk h: sub-tile h (kSubN rows) and, in pair mode, this
-        // CTA's half of it.
-        const int32_t b_row = static_cast<int32_t>(t.w_row0 + rank * C::kBChunkRows);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
-          if (PAIR) {
-            // Both CTAs' bytes complete on the leader's full barrier, which the
-            // leader alone arms.
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-            const uint32_t bar = map_to_rank(&full[stage], 0);
-            tma_load_2d_pair(a_tiles + stage * C::kABytes, &tmap_a, bar, kb * BK, a_row);
-#pragma unroll
-            for (int h = 0; h < C::kSplitN; ++h)
-              tma_load_2d_pair(b_tiles + stage * C::kBBytes + h * C::kBChunkBytes, &tmap_w, bar,
-                               kb * BK, b_row + h * C::kSubN);
-          } else {
-            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-            tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK, a_row);
-#pragma unroll
-            for (int h = 0; h < C::kSplitN; ++h)
-              tma_load_2d(b_tiles + stage * C::kBBytes + h * C::kBChunkBytes, &tmap_w,
-                          &full[stage], kb * BK, b_row + h * C::kSubN);
-          }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
+                      static_cast<int32_t>(t.row0));
+          tma_load_2d(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
+                      static_cast<int32_t>(t.w_row0));
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) {
@@ -380,60 +371,131 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
         }
       }
     producer_done:
-      if (*abort_flag && (!PAIR || rank == 0)) {
-        // Let every load in flight land before the CTA exits (in pair mode the
-        // leader's full barriers count the peer's loads too).
+      if (*abort_flag) {
+        // Let every load in flight land before the CTA exits.
         for (int s = 0; s < C::kStages; ++s)
-          if (armed & (1u << s)) mbar_wait<PAIR>(&full[s], (armed_phase >> s) & 1u, nullptr);
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && (!PAIR || rank == 0)) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(PAIR ? 2 * BM : BM, C::kSubN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int tb = 0;
-      uint32_t tphase = 0;
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two issuing threads: warp 1 takes the even and warp 3 the odd K blocks
+    // of this CTA's sequence (i counts K blocks over all its units).  Each K
+    // block writes a fresh partial into its own TMEM buffer and reads its own
+    // stage, so the two streams need no ordering between them.  One thread
+    // alone would spend about as long per K block on its barrier waits,
+    // commits and four instruction issues as the tensor core spends on the
+    // MMAs, and the tensor core would idle behind it.
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      const uint32_t parity = warp == 1 ? 0u : 1u;
+      uint32_t i = 0;
       for (int u = unit_start; u < num_units; u += unit_step) {
         const Unit t = unit_of(u);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) goto mma_done;
+        for (int kb = t.kb0; kb < t.kb1; ++kb, ++i) {
+          if ((i & 1u) != parity) continue;
+          const int stage = static_cast<int>(i % C::kStages);
+          const uint32_t phase = (i / C::kStages) & 1u;
+          const int tb = static_cast<int>(i % C::kAccBufs);
+          const uint32_t tphase = (i / C::kAccBufs) & 1u;
+          if (!mbar_wait(&full[stage], phase, abort_flag)) goto mma_done;
+          if (!mbar_wait<kSpinWaits>(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
           tc_fence_after();
           const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
           const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
 #pragma unroll
-          for (int h = 0; h < C::kSplitN; ++h) {
-            const int sb = tb * C::kSplitN + h;
-            if (!mbar_wait<PAIR>(&tempty[sb], tphase ^ 1u, abort_flag)) goto mma_done;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN + h * C::kSubN);
-#pragma unroll
-            for (int k = 0; k < BK / 32; ++k) {
-              const uint64_t ad = smem_desc_k_sw128(a_addr + 32 * k);
-              const uint64_t bd = smem_desc_k_sw128(b_addr + h * C::kBChunkBytes + 32 * k);
-              if (PAIR) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
-              else mma_f8f6f4(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
-            }
-            if (PAIR) mma_commit_pair_mask(&tfull[sb], 0x3);
-            else mma_commit(&tfull[sb]);
-          }
-          if (PAIR) mma_commit_pair_mask(&empty[stage], 0x3);
-          else mma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          tb ^= 1;
-          if (tb == 0) tphase ^= 1u;
+          for (int k = 0; k < BK / 32; ++k)
+            mma_f8f6f4(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
+                       smem_desc_k_sw128(b_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
+          mma_commit(&tfull[tb]);
+          mma_commit(&empty[stage]);
         }
       }
     mma_done:
-      // Every MMA issued must finish before the TMEM columns are released.
-      if (PAIR) mma_commit_pair(flush); else mma_commit(flush);
-      mbar_wait(flush, 0, nullptr);
+      // Every MMA this thread issued must finish before the TMEM columns are
+      // released.
+      mma_commit(&flush[parity]);
+      mbar_wait(&flush[parity], 0, nullptr);
     }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale producer
+    // Walks the same (unit, K block) sequence as the epilogue.  A second
+    // cursor runs kAhead steps ahead and loads the scales into a ring of
+    // registers, so the global loads of step i + kAhead overlap the shared-
+    // memory writes of step i.  Step i uses the slot of its TMEM buffer,
+    // i % kAccBufs, once the epilogue has released that buffer (tempty), and
+    // then arrives on its tfull: a_s of the tile's 128 rows (0 past the last
+    // row) and w_s of the weight blocks the tile touches (0 past the last).
+    constexpr int kAhead = 4;
+    constexpr int kNbPerTile = C::kNbSpan;
+    struct Cursor {
+      int u, kb, kb1, group, nb0;
+      int64_t row0, row_end;
+      bool valid;
+    };
+    auto begin = [&](Cursor& c, int u) {
+      c.u = u;
+      c.valid = u < num_units;
+      if (c.valid) {
+        const Unit t = unit_of(u);
+        c.kb = t.kb0;
+        c.kb1 = t.kb1;
+        c.group = t.group;
+        c.nb0 = (t.n_tile * BN) / 128;
+        c.row0 = t.row0;
+        c.row_end = t.row_end;
+      }
+    };
+    auto next = [&](Cursor& c) {
+      if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
+    };
+    auto load = [&](const Cursor& c, float (&va)[4], float& vw) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t row = c.row0 + lane + 32 * j;
+        va[j] = (c.valid && row < c.row_end) ? __ldg(p.sa + row * p.kbn + c.kb) : 0.0f;
+      }
+      const int nb = c.nb0 + lane;
+      vw = (c.valid && lane < kNbPerTile && nb < p.nbn)
+               ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
+               : 0.0f;
+    };
+    float ra[kAhead][4], rw[kAhead];
+    Cursor ahead, cur;
+    begin(ahead, unit_start);
+    begin(cur, unit_start);
+#pragma unroll
+    for (int d = 0; d < kAhead; ++d) {
+      load(ahead, ra[d], rw[d]);
+      next(ahead);
+    }
+    int slot = 0;
+    uint32_t sphase = 0;
+    while (cur.valid) {
+#pragma unroll
+      for (int ph = 0; ph < kAhead; ++ph) {
+        if (!cur.valid) break;
+        const bool ok = mbar_wait(&tempty[slot], sphase ^ 1u, abort_flag);
+        if (!__all_sync(0xFFFFFFFFu, ok)) goto scales_done;
+        float* dst = scale_slots + slot * (C::kScaleSlotBytes / 4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = ra[ph][j];
+        if (lane < kNbPerTile) dst[BM + lane] = rw[ph];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[slot]);
+        load(ahead, ra[ph], rw[ph]);
+        next(ahead);
+        next(cur);
+        if (++slot == C::kAccBufs) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+      }
+    }
+  scales_done:
     __syncwarp();
   }
   } else {
@@ -444,72 +506,91 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
     const int g = e >> 2;                       // column half
     constexpr int CPW = C::kColsPerWarp;
     constexpr int NCH = C::kChunks;
-    const int row_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
+    const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const bool vec_store = (p.N % 8) == 0;
-    // This warp's sub-buffer within each TMEM buffer (both halves are the same
-    // sub-buffer when the MMA is not split).
-    const int half = (g * C::kSplitN) >> 1;
-    const uint32_t tempty_leader0 = PAIR ? map_to_rank(&tempty[half], 0) : 0u;
-    const uint32_t tempty_leader1 = PAIR ? map_to_rank(&tempty[C::kSplitN + half], 0) : 0u;
     int tb = 0;
     uint32_t tphase = 0;
     for (int u = unit_start; u < num_units; u += unit_step) {
       const Unit t = unit_of(u);
       const int64_t row = t.row0 + row_in_tile;
       const bool row_ok = row < t.row_end;
-      const int nb = (t.n_tile * BN + g * CPW) / 128;
-      const bool nb_ok = nb < p.nbn;
-      const float* sa_row = p.sa + (row_ok ? row : 0) * static_cast<int64_t>(p.kbn);
-      const float* sw_row =
-          p.sw + (static_cast<int64_t>(t.group) * p.nbn + (nb_ok ? nb : 0)) * p.kbn;
+      // Weight block of each 32-column chunk of this warp, relative to the
+      // tile's first block (chunks never straddle a block boundary).
+      const int nb0 = (t.n_tile * BN) / 128;
+      int nb_of[NCH];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) nb_of[c] = ((t.n_tile * BN + g * CPW + 32 * c) >> 7) - nb0;
       float2 acc[CPW / 2];
 #pragma unroll
       for (int j = 0; j < CPW / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
-      float sa_next = row_ok ? __ldg(sa_row + t.kb0) : 0.0f;
-      float sw_next = nb_ok ? __ldg(sw_row + t.kb0) : 0.0f;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
-        const float scale = sa_next * sw_next;
-        const float2 scale2 = make_float2(scale, scale);
-        if (kb + 1 < t.kb1) {
-          sa_next = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
-          sw_next = nb_ok ? __ldg(sw_row + kb + 1) : 0.0f;
-        }
-        const bool ok = mbar_wait<PAIR>(&tfull[tb * C::kSplitN + half], tphase, abort_flag);
+        const bool ok = mbar_wait<kSpinWaits>(&tfull[tb], tphase, abort_flag);
         if (!__all_sync(0xFFFFFFFFu, ok)) goto epilogue_done;
         tc_fence_after();
+        // This K block's scale products a_s[row, kb] * w_s[nb, kb], read before
+        // the buffer (and with it the scale slot) is released below.
+        const float* src = scale_slots + tb * (C::kScaleSlotBytes / 4);
+        const float sa_row = src[row_in_tile];
+        float scale_nb[C::kNbSpan];
+#pragma unroll
+        for (int i = 0; i < C::kNbSpan; ++i) scale_nb[i] = sa_row * src[BM + i];
         const uint32_t col_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
-        // Two register buffers: the load of chunk c+1 is in flight while the
-        // FMAs of chunk c run.
-        uint32_t va[32], vb[32];
-        tmem_ld_32x32b_x32(col_addr, va);
-        tmem_ld_wait(va);
+        if (C::kOneBatch) {
+          // All of this warp's columns in one batch, then hand the buffer back
+          // to the MMA before the FMAs.
+          uint32_t v[NCH][32];
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t(&cur)[32] = (c & 1) ? vb : va;
-          uint32_t(&nxt)[32] = (c & 1) ? va : vb;
-          if (c + 1 < NCH) tmem_ld_32x32b_x32(col_addr + 32 * (c + 1), nxt);
-          if (c + 1 == NCH) {
-            // Every load of this buffer has completed: hand it back to the MMA.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              if (PAIR) mbar_arrive_cluster(tb ? tempty_leader1 : tempty_leader0);
-              else mbar_arrive(&tempty[tb * C::kSplitN + half]);
-            }
+          for (int c = 0; c < NCH; ++c) tmem_ld_32x32b_x32(col_addr + 32 * c, v[c]);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tmem_ld_wait(v[c]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            const float sc = C::kNbSpan == 1 ? scale_nb[0] : (nb_of[c] ? scale_nb[C::kNbSpan - 1] : scale_nb[0]);
+            const float2 scale2 = make_float2(sc, sc);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[c * 16 + j] = __ffma2_rn(
+                  make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1])),
+                  scale2, acc[c * 16 + j]);
           }
+        } else {
+          // Two register buffers: the load of chunk c+1 is in flight while the
+          // FMAs of chunk c run.
+          uint32_t va[32], vb[32];
+          tmem_ld_32x32b_x32(col_addr, va);
+          tmem_ld_wait(va);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            acc[c * 16 + j] = __ffma2_rn(
-                make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), scale2,
-                acc[c * 16 + j]);
-          if (c + 1 < NCH) tmem_ld_wait(nxt);
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? vb : va;
+            uint32_t(&nxt)[32] = (c & 1) ? va : vb;
+            if (c + 1 < NCH) tmem_ld_32x32b_x32(col_addr + 32 * (c + 1), nxt);
+            if (c + 1 == NCH) {
+              // Every load of this buffer has completed: hand it back to the MMA.
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[tb]);
+            }
+            const float sc = C::kNbSpan == 1 ? scale_nb[0] : (nb_of[c] ? scale_nb[C::kNbSpan - 1] : scale_nb[0]);
+            const float2 scale2 = make_float2(sc, sc);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[c * 16 + j] = __ffma2_rn(
+                  make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])),
+                  scale2, acc[c * 16 + j]);
+            if (c + 1 < NCH) tmem_ld_wait(nxt);
+          }
         }
-        tb ^= 1;
-        if (tb == 0) tphase ^= 1u;
+        if (++tb == C::kAccBufs) {
+          tb = 0;
+          tphase ^= 1u;
+        }
       }
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
-      const int64_t slab0 = t.row0 + static_cast<int64_t>(rank) * BM + quad * 32;
+      const int64_t slab0 = t.row0 + quad * 32;
       const bool slab_tma = slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end);
       if (p.y_tma == 2 && slab_tma) {
         // FP32 split-K partials of split t.split, 16 columns per box.
@@ -584,13 +665,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  // In pair mode neither CTA may release TMEM or exit while the other can
-  // still touch its shared memory, barriers or TMEM.
-  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
-    else tmem_dealloc(tmem_base, C::kTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

@@ -17,9 +17,6 @@
  * scratch space take it from a caller-provided workspace whose size the
  * matching *_workspace_size() function returns.
  *
- * Environment: FP8BS_GEMM_PAIR=1 lets the GEMM planner use CTA-pair tiles
- * (tcgen05.mma.cta_group::2); they are off by default.
- *
  * Sources of the operations (page title, then section):
  *  [ACT] "Understanding Dynamic and Static Activation Quantization Schemes in
  *        DeepSeek-V3", "How Dynamic Activation Quantization Works";
@@ -183,7 +180,7 @@ FP8BS_API fp8bs_status fp8bs_selftest_block_scale(const float *amax, float *s, i
                                                   int scale_fmt, void *stream);
 
 /* Launch plan fp8_gemm would use for an M x N x K problem on the current
- * device (tile width, CTA pairing, K split, work units, grid), as a
+ * device (tile width, K split, work units, grid), as a
  * NUL-terminated string in thread-local storage; for logs and benchmarks. */
 FP8BS_API const char *fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K);
 

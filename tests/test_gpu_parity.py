@@ -237,6 +237,9 @@ def test_gemm_tiny_linear():
 @pytest.mark.parametrize("M,N,K", [
     (1, 256, 128), (127, 576, 512), (129, 130, 256), (300, 384, 1024), (256, 512, 7168),
     (513, 1280, 384), (64, 2048, 2048), (2, 18432, 256), (200, 136, 128),
+    # 192-wide tiles whose columns straddle a 128-column weight block, a K
+    # split of 192-wide tiles, and a last tile 64 columns wide
+    (384, 200, 1024), (256, 576, 7168), (1000, 7168, 256),
 ])
 def test_gemm_shapes(M, N, K):
     x, qa, sa, qw, sw = _gemm_case(M, N, K, seed=M + N + K)
