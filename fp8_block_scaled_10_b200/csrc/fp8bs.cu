@@ -58,10 +58,10 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G>
+template <int BN, bool G, int AR = 128>
 fp8bs_status setup_gemm_kernel() {
-  using C = gemm::Cfg<BN>;
-  auto kernel = gemm::fp8_gemm_kernel<BN, G>;
+  using C = gemm::Cfg<BN, AR>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -114,6 +114,10 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_kernel<128, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<192, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 64>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 64>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 16>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 16>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, true>()) != FP8BS_OK ||
@@ -154,6 +158,10 @@ fp8bs_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
 constexpr int kMaxSmemOptin = 227 * 1024;
 static_assert(gemm::Cfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::Cfg<192>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<256, 64>::smem_bytes(false) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<128, 64>::smem_bytes(false) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<256, 16>::smem_bytes(false) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<128, 16>::smem_bytes(false) <= kMaxSmemOptin, "smem");
 static_assert(gemm::Cfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 static_assert(gemm::BsCfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
@@ -323,18 +331,28 @@ size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
-template <int BN, bool G>
+template <int BN, bool G, int AR = 128>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                         const gemm::Params& p, int grid, cudaStream_t st) {
-  using C = gemm::Cfg<BN>;
-  return launch(gemm::fp8_gemm_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, ta, tw,
-                ty, p);
+  using C = gemm::Cfg<BN, AR>;
+  return launch(gemm::fp8_gemm_kernel<BN, G, AR>, grid, C::kThreads, C::smem_bytes(G), st, ta,
+                tw, ty, p);
 }
 
+// Rows of A one pipeline stage loads: all 128 rows of a tile, or for
+// decode-sized M (dense calls only) 16 or 64.
+int a_rows_for(int64_t M) { return M <= 16 ? 16 : (M <= 64 ? 64 : 128); }
+
 template <bool G>
-cudaError_t launch_gemm_any(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
+cudaError_t launch_gemm_any(int bn, int a_rows, const CUtensorMap& ta, const CUtensorMap& tw,
                             const CUtensorMap& ty, const gemm::Params& p, int grid,
                             cudaStream_t st) {
+  if (!G && a_rows == 16)
+    return bn == 256 ? launch_gemm<256, G, 16>(ta, tw, ty, p, grid, st)
+                     : launch_gemm<128, G, 16>(ta, tw, ty, p, grid, st);
+  if (!G && a_rows == 64)
+    return bn == 256 ? launch_gemm<256, G, 64>(ta, tw, ty, p, grid, st)
+                     : launch_gemm<128, G, 64>(ta, tw, ty, p, grid, st);
   return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
          : bn == 192 ? launch_gemm<192, G>(ta, tw, ty, p, grid, st)
                      : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
@@ -369,7 +387,10 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
 
   CUtensorMap ta, tw, ty;
   gemm::Params p{};
-  if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
+  // Decode-sized M loads only the rows it has; 192-wide tiles are planned for
+  // M > 128 only.
+  const int a_rows = pl.bn == 192 ? 128 : a_rows_for(M);
+  if ((r = make_tmap(&ta, a, M, K, a_rows)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
   if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
   p.sa = a_s;
@@ -387,7 +408,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
   p.groups = 1;
-  cudaError_t e = launch_gemm_any<false>(pl.bn, ta, tw, ty, p, pl.grid, st);
+  cudaError_t e = launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.splits > 1) {
     const int64_t MN = M * N;
@@ -843,7 +864,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   // Units are only known on the device; an upper bound sizes the grid.
   const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
   const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
-  cudaError_t e = launch_gemm_any<true>(bn, ta, tw, ty, p, grid, as_stream(stream));
+  cudaError_t e = launch_gemm_any<true>(bn, 128, ta, tw, ty, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
   return FP8BS_OK;
 }

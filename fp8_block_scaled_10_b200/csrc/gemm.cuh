@@ -111,13 +111,23 @@ __device__ __forceinline__ void store_out_box(const CUtensorMap* tmap, uint8_t* 
   }
 }
 
-template <int BN>
+// ARows: rows of A that one stage loads.  128 for M > 64; for decode-sized M
+// (at most 16 or 64 rows) only those rows are loaded, so that the shared
+// memory holds more stages of the weight stream, which bounds decode.  The MMA
+// still reads a 128-row A operand: the rows past ARows come from the shared
+// memory that follows the stage's A slot (the next A slots, then the W
+// slots, all inside the CTA's allocation), and they only produce
+// accumulator rows past M, which are never stored.
+template <int BN, int ARows = 128>
 struct Cfg {
   static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
-  static constexpr int kABytes = BM * BK;
+  static_assert(ARows == 128 || ARows == 64 || ARows == 16, "A rows per stage");
+  static constexpr int kABytes = ARows * BK;
   static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+  static constexpr int kStages =
+      ARows == 128 ? (BN == 256 ? 4 : (BN == 192 ? 5 : 6))
+                   : ((200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes);
   // Two epilogue warpgroups: each covers all 128 TMEM lanes (one warp per
   // 32-lane quadrant) and half of the tile's columns.
   static constexpr int kEpiWarps = 8;
@@ -236,12 +246,12 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   return t;
 }
 
-template <int BN, bool GROUPED>
-__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
+template <int BN, bool GROUPED, int ARows = 128>
+__global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w,
                     const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, ARows>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
