@@ -251,7 +251,13 @@ struct Plan {
   int splits, kb_per_split;
   int units;
   int grid;   // persistent CTAs
+  // Split tail (see gemm::Params): 0 = none.
+  int full_units = 0, tail_tiles = 0, tail_splits = 0, tail_kbps = 0;
 };
+
+// The split tail's FP32 partials are kept within this many bytes, so that
+// every prefill plan also fits the library's static scratch array.
+constexpr size_t kTailWorkspaceCap = FP8BS_STATIC_SCRATCH_BYTES;
 
 double wave_efficiency(int64_t units, int slots) {
   const int64_t waves = (units + slots - 1) / slots;
@@ -276,7 +282,11 @@ double kb_time_us(GemmKind kind, int bn) {
 //
 // M > 128 (several 128-row tiles share each W tile): the estimated time is
 // waves of work units x K blocks per unit x kb_time_us, plus, for a K split,
-// the FP32 partials' round trip through HBM and the reduction launch.
+// the FP32 partials' round trip through HBM and the reduction launch.  When
+// the tiles fill the GPU but their last wave would keep at most half of the
+// SMs busy, the promotion kernel can split only the tiles of that wave along
+// K ("split tail"): the whole waves run unchanged and the tail's partials,
+// a few MB, are summed by a small reduction.
 //
 // M <= 128 (decode): the weight stream from HBM bounds every tile width
 // alike; the score is the fraction of persistent slots kept busy, with a
@@ -302,12 +312,35 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
       if (splits != s) continue;
       const int64_t units = tiles * splits;
       bool better;
+      Plan cand{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units),
+                static_cast<int>(std::min<int64_t>(units, slots))};
       if (compute_bound) {
         const double kb_us = kb_time_us(kind, bn);
         const double waves = static_cast<double>((units + slots - 1) / slots);
         double t = waves * per * kb_us;
         if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
           t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
+        const int64_t tail = tiles % slots;
+        if (kind == GemmKind::kPromotion && splits == 1 && tiles > slots && tail > 0 &&
+            2 * tail <= slots) {
+          const size_t tile_bytes = static_cast<size_t>(128) * bn * sizeof(float);
+          const int64_t by_ws = static_cast<int64_t>(kTailWorkspaceCap / (tail * tile_bytes));
+          const int ts = static_cast<int>(std::min<int64_t>({slots / tail, kbn / 4, by_ws}));
+          if (ts >= 2) {
+            const int tkb = (kbn + ts - 1) / ts;
+            const double t_tail = static_cast<double>(tiles / slots) * per * kb_us +
+                                  tkb * kb_us + 3.0;   // + the reduction launch
+            if (t_tail < t) {
+              t = t_tail;
+              cand.full_units = static_cast<int>(tiles - tail);
+              cand.tail_tiles = static_cast<int>(tail);
+              cand.tail_splits = (kbn + tkb - 1) / tkb;
+              cand.tail_kbps = tkb;
+              cand.units = cand.full_units + cand.tail_tiles * cand.tail_splits;
+              cand.grid = slots;
+            }
+          }
+        }
         better = t < best_time - 1e-9;
         if (better) best_time = t;
       } else {
@@ -319,15 +352,15 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
         better = score > best_score + 1e-9;
         if (better) best_score = score;
       }
-      if (better)
-        best = Plan{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units),
-                    static_cast<int>(std::min<int64_t>(units, slots))};
+      if (better) best = cand;
     }
   }
   return best;
 }
 
 size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
+  if (pl.tail_splits > 0)
+    return static_cast<size_t>(pl.tail_tiles) * pl.tail_splits * 128 * pl.bn * sizeof(float);
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
@@ -407,9 +440,22 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.splits = pl.splits;
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
+  p.full_units = pl.full_units;
+  p.tail_tiles = pl.tail_tiles;
+  p.tail_splits = pl.tail_splits;
+  p.tail_kbps = pl.tail_kbps;
+  p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   p.groups = 1;
   cudaError_t e = launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
+  if (pl.tail_splits > 0) {
+    const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
+    e = launch(gemm::tail_reduce_kernel, grid_for(items, 256, info->sms * 8), 256, 0, st,
+               static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), M,
+               static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles, pl.tail_splits,
+               pl.bn);
+    if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
+  }
   if (pl.splits > 1) {
     const int64_t MN = M * N;
     e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,
@@ -676,9 +722,10 @@ const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
   }
   const Plan pl = plan_gemm(M, N, K, *info);
   snprintf(buf, sizeof(buf),
-           "bn=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d sms=%d",
+           "bn=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d sms=%d "
+           "tail_tiles=%d tail_splits=%d",
            pl.bn, pl.m_tiles, pl.n_tiles, pl.splits, pl.kb_per_split, pl.units, pl.grid,
-           info->sms);
+           info->sms, pl.tail_tiles, pl.tail_splits);
   return buf;
 }
 

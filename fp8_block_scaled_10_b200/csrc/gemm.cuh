@@ -74,6 +74,16 @@ struct Params {
   int groups;               // grouped mode
   int y_tma;                // 1: bf16 y written by TMA stores through staging boxes;
                             // 2: FP32 split-K partials written by TMA stores (3-D map)
+  // Split tail (dense mode, one split otherwise): units [0, full_units) are
+  // whole tiles numbered as in the unsplit plan; the tail_tiles tiles after
+  // them each become tail_splits units of tail_kbps K blocks whose FP32
+  // partials go to tail_ws[(tail tile * tail_splits + split)][128][BN], summed
+  // afterwards by tail_reduce_kernel.  tail_splits == 0: no split tail.
+  int full_units;
+  int tail_tiles;
+  int tail_splits;
+  int tail_kbps;
+  float* tail_ws;
 };
 
 // Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
@@ -194,6 +204,7 @@ struct Unit {
   int n_tile;
   int kb0, kb1;
   int split;
+  int tail_slot;     // >= 0: FP32 partial slot of a split tail unit
 };
 
 // Dense units: m tile fastest, so the CTAs running at the same time share W
@@ -201,6 +212,23 @@ struct Unit {
 template <int kUnitRows>
 __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   Unit t;
+  t.tail_slot = -1;
+  if (p.tail_splits > 0 && u >= p.full_units) {
+    // Split tail: consecutive units take different tiles, so the CTAs of the
+    // last wave stream different operands.
+    const int r = u - p.full_units;
+    const int tt = r % p.tail_tiles;
+    const int tile = p.full_units + tt;
+    t.split = r / p.tail_tiles;
+    t.n_tile = tile / p.m_tiles;
+    t.group = 0;
+    t.row0 = static_cast<int64_t>(tile % p.m_tiles) * kUnitRows;
+    t.row_end = p.M;
+    t.kb0 = t.split * p.tail_kbps;
+    t.kb1 = min(p.kbn, t.kb0 + p.tail_kbps);
+    t.tail_slot = tt * p.tail_splits + t.split;
+    return t;
+  }
   const int m_tile = u % p.m_tiles;
   const int rest = u / p.m_tiles;
   t.split = rest % p.splits;
@@ -241,6 +269,7 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   t.row0 = lo + static_cast<int64_t>(gm - tile_prefix[a]) * kUnitRows;
   t.row_end = hi;
   t.split = 0;
+  t.tail_slot = -1;
   t.kb0 = 0;
   t.kb1 = p.kbn;
   return t;
@@ -599,6 +628,16 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
           tphase ^= 1u;
         }
       }
+      if (!GROUPED && t.tail_slot >= 0) {
+        // FP32 partial of a split tail unit: the whole 128 x BN tile, rows and
+        // columns past the matrix included (the reduction masks them).
+        float* dst = p.tail_ws + (static_cast<int64_t>(t.tail_slot) * BM + row_in_tile) * BN + g * CPW;
+#pragma unroll
+        for (int c = 0; c < CPW / 4; ++c)
+          *reinterpret_cast<float4*>(dst + 4 * c) =
+              make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y);
+        continue;
+      }
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
       const int64_t slab0 = t.row0 + quad * 32;
       const bool slab_tma = slab0 < t.row_end && (!GROUPED || slab0 + 32 <= t.row_end);
@@ -678,6 +717,46 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Sum of the FP32 partials of the split tail tiles, in split order, as bf16
+// into y.  One thread per 4 consecutive columns of one tile row.
+__global__ void __launch_bounds__(256)
+    tail_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ y, int64_t M,
+                       int N, int m_tiles, int full_units, int tail_tiles, int splits, int bn) {
+  pdl_trigger();
+  pdl_wait();
+  const int groups = bn / 4;
+  const int64_t items = static_cast<int64_t>(tail_tiles) * BM * groups;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < items;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int tt = static_cast<int>(i / (BM * groups));
+    const int rem = static_cast<int>(i - static_cast<int64_t>(tt) * BM * groups);
+    const int r = rem / groups, c = (rem - r * groups) * 4;
+    const int tile = full_units + tt;
+    const int64_t row = static_cast<int64_t>(tile % m_tiles) * BM + r;
+    const int64_t col = static_cast<int64_t>(tile / m_tiles) * bn + c;
+    if (row >= M || col >= N) continue;
+    float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sp = 0; sp < splits; ++sp) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(
+          ws + ((static_cast<int64_t>(tt) * splits + sp) * BM + r) * bn + c));
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    __nv_bfloat16* dst = y + row * N + col;
+    const float v4[4] = {s.x, s.y, s.z, s.w};
+    if ((N % 4) == 0 && col + 4 <= N) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&lo);
+      u.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(dst) = u;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (col + j < N) dst[j] = __float2bfloat16_rn(v4[j]);
+    }
   }
 }
 

@@ -248,6 +248,20 @@ def test_gemm_shapes(M, N, K):
     assert_gemm_close(y, y_ref, bnd, "gemm %dx%dx%d" % (M, N, K))
 
 
+def test_gemm_split_tail_every_output():
+    """160 tiles on 148 SMs: the 12 tiles of the last wave are split along K
+    and summed by the tail reduction; ragged last row and column tiles."""
+    M, N, K = 1200, 4000, 4096
+    plan = fp8bs.gemm_plan(M, N, K)
+    if fp8bs.lib().fp8bs_gemm_plan_string(M, N, K).decode().find("sms=148") < 0:
+        pytest.skip("plan depends on the SM count: " + plan)
+    assert "tail_splits=0" not in plan, plan
+    x, qa, sa, qw, sw = _gemm_case(M, N, K, seed=77)
+    y = fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw))
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y, y_ref, bnd, "split tail " + plan)
+
+
 def test_gemm_writes_only_its_output():
     """Canary rows and columns around y stay untouched (raw C-ABI call)."""
     M, N, K = 130, 200, 256
