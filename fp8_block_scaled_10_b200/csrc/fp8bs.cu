@@ -112,7 +112,6 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_kernel<192, false>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, false>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<128, true>()) != FP8BS_OK ||
-        (r = setup_gemm_kernel<192, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<128, false, 64>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, false, 64>()) != FP8BS_OK ||
@@ -157,7 +156,7 @@ fp8bs_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
 // Every GEMM configuration fits the 227 KB of shared memory a CTA can opt into.
 constexpr int kMaxSmemOptin = 227 * 1024;
 static_assert(gemm::Cfg<256>::smem_bytes(true) <= kMaxSmemOptin, "smem");
-static_assert(gemm::Cfg<192>::smem_bytes(true) <= kMaxSmemOptin, "smem");
+static_assert(gemm::Cfg<192>::smem_bytes(false) <= kMaxSmemOptin, "smem");
 static_assert(gemm::Cfg<256, 64>::smem_bytes(false) <= kMaxSmemOptin, "smem");
 static_assert(gemm::Cfg<128, 64>::smem_bytes(false) <= kMaxSmemOptin, "smem");
 static_assert(gemm::Cfg<256, 16>::smem_bytes(false) <= kMaxSmemOptin, "smem");
@@ -386,6 +385,8 @@ cudaError_t launch_gemm_any(int bn, int a_rows, const CUtensorMap& ta, const CUt
   if (!G && a_rows == 64)
     return bn == 256 ? launch_gemm<256, G, 64>(ta, tw, ty, p, grid, st)
                      : launch_gemm<128, G, 64>(ta, tw, ty, p, grid, st);
+  if (G) return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
+                          : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
   return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
          : bn == 192 ? launch_gemm<192, G>(ta, tw, ty, p, grid, st)
                      : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
@@ -818,7 +819,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
     return fail(FP8BS_ERR_INVALID_ARG, "m_offsets must be an 8-byte aligned device pointer");
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
-  if (M_total < 0 || M_total > (int64_t(1) << 31))
+  if (M_total < 0 || M_total >= (int64_t(1) << 31))
     return fail(FP8BS_ERR_INVALID_ARG, "M_total out of range");
   if (M_total == 0) return FP8BS_OK;
   if (G * N > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "G*N too large");
@@ -875,15 +876,16 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
     return fail(FP8BS_ERR_INVALID_ARG, "m_offsets must be an 8-byte aligned device pointer");
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
-  if (M_total < 0 || M_total > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M_total out of range");
+  if (M_total < 0 || M_total >= (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M_total out of range");
   if (M_total == 0) return FP8BS_OK;
   if (G * N > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "G*N too large");
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  // The tile width with the least estimated time per 128-row tile of a group.
+  // The tile width with the least estimated time per 128-row tile of a group
+  // (192-wide tiles and the group table do not fit shared memory together).
   int bn = 128;
-  for (int cand : {256, 192}) {
+  for (int cand : {256}) {
     if (N < cand) continue;
     const auto cost = [&](int b) { return ((N + b - 1) / b) * kb_time_us(GemmKind::kPromotion, b); };
     if (cost(cand) < cost(bn) - 1e-9) bn = cand;

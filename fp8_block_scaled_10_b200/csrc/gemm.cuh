@@ -51,6 +51,8 @@ namespace gemm {
 constexpr int BM = 128;      // rows of A per CTA
 constexpr int BK = 128;      // one K block per pipeline stage
 constexpr int kMaxGroups = 1024;
+// Ints of the grouped mode's table in shared memory (see group_table).
+constexpr int kGroupTableInts = 2 * (kMaxGroups + 1);
 #ifndef FP8BS_SPIN_WAITS
 #define FP8BS_SPIN_WAITS 0
 #endif
@@ -172,7 +174,7 @@ struct Cfg {
   static constexpr int kScaleSlotBytes = 4 * (BM + 4);
   static constexpr int kScaleBytes = kScaleSlots * kScaleSlotBytes;
   // grouped mode: per-group m-tile prefix (int)
-  static constexpr int kGroupBytes = 4 * (kMaxGroups + 1);
+  static constexpr int kGroupBytes = 4 * kGroupTableInts;
   // output staging boxes (one per epilogue warp), 1024-byte aligned
   __host__ __device__ static constexpr int out_offset(bool grouped) {
     return (kStages * kStageBytes + kCtrlBytes + kScaleBytes + (grouped ? kGroupBytes : 0) +
@@ -241,18 +243,46 @@ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   return t;
 }
 
-// Row range [lo, hi) of group g: the device offsets clamped to [0, M] and
-// made non-decreasing.
-__device__ __forceinline__ void group_rows(const Params& p, int g, int64_t& lo, int64_t& hi) {
-  lo = __ldg(p.m_offsets + g);
-  hi = __ldg(p.m_offsets + g + 1);
-  lo = lo < 0 ? 0 : (lo > p.M ? p.M : lo);
-  hi = hi < lo ? lo : (hi > p.M ? p.M : hi);
-}
-
 // Grouped units: n tile fastest inside one global m tile, so the CTAs running
 // at the same time work on one or two experts and read each W_e once.
-// tile_prefix[g] is the number of m tiles of groups < g.
+// The group table in shared memory: tile_prefix[g] (g <= G) is the number of
+// m tiles of groups < g, and row_off[g] = tile_prefix[kMaxGroups + 1 + g]
+// (g <= G) is the device offset g clamped to [0, M]; group g's rows are
+// [row_off[g], max(row_off[g + 1], row_off[g])), the device offsets clamped to [0, M] and made non-decreasing.
+// Built once per CTA by group_table, so that a unit's rows cost no global
+// load on the producer's and the MMA issuers' paths.
+__device__ __forceinline__ void group_table(const Params& p, int* table, int lane,
+                                            int* num_units) {
+  int* row_off = table + kMaxGroups + 1;
+  for (int g = lane; g <= p.groups; g += 32) {
+    int64_t o = __ldg(p.m_offsets + g);
+    o = o < 0 ? 0 : (o > p.M ? p.M : o);
+    row_off[g] = static_cast<int>(o);
+  }
+  __syncwarp();
+  int carry = 0;
+  for (int g0 = 0; g0 < p.groups; g0 += 32) {
+    const int g = g0 + lane;
+    int tiles = 0;
+    if (g < p.groups) {
+      const int lo = row_off[g], hi = max(row_off[g + 1], lo);
+      tiles = (hi - lo + BM - 1) / BM;
+    }
+    int incl = tiles;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (g < p.groups) table[g] = carry + incl - tiles;
+    carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+  }
+  if (lane == 0) {
+    table[p.groups] = carry;
+    *num_units = carry * p.n_tiles;
+  }
+}
+
 template <int kUnitRows>
 __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix, int u) {
   Unit t;
@@ -264,8 +294,8 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
     if (tile_prefix[mid] <= gm) a = mid; else b = mid;
   }
   t.group = a;
-  int64_t lo, hi;
-  group_rows(p, a, lo, hi);
+  const int* row_off = tile_prefix + kMaxGroups + 1;
+  const int64_t lo = row_off[a], hi = max(row_off[a + 1], row_off[a]);
   t.row0 = lo + static_cast<int64_t>(gm - tile_prefix[a]) * kUnitRows;
   t.row_end = hi;
   t.split = 0;
@@ -338,30 +368,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
   if (GROUPED) {
     // Clamp the device offsets to [0, M], count each group's m tiles and form
     // their exclusive prefix sum (warp 2, 32 groups per step).
-    if (warp == 2) {
-      int carry = 0;
-      for (int g0 = 0; g0 < p.groups; g0 += 32) {
-        const int g = g0 + lane;
-        int tiles = 0;
-        if (g < p.groups) {
-          int64_t lo, hi;
-          group_rows(p, g, lo, hi);
-          tiles = static_cast<int>((hi - lo + BM - 1) / BM);
-        }
-        int incl = tiles;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += v;
-        }
-        if (g < p.groups) tile_prefix[g] = carry + incl - tiles;
-        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-      if (lane == 0) {
-        tile_prefix[p.groups] = carry;
-        ctrl->num_units = carry * p.n_tiles;
-      }
-    }
+    if (warp == 2) group_table(p, tile_prefix, lane, &ctrl->num_units);
   } else if (threadIdx.x == 0) {
     ctrl->num_units = p.num_units;
   }

@@ -54,7 +54,7 @@ struct BsCfg {
   static constexpr int kFirstEpiWarp = 4;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
   static constexpr int kCtrlBytes = 256;
-  static constexpr int kGroupBytes = 4 * (kMaxGroups + 1);
+  static constexpr int kGroupBytes = 4 * kGroupTableInts;
   __host__ __device__ static constexpr int out_offset(bool grouped) {
     return (kStages * (kStageBytes + kSFBytes) + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1023) &
            ~1023;
@@ -141,30 +141,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
   // programmatic serialization): wait for it before any global access.
   pdl_wait();
   if (GROUPED) {
-    if (warp == 2) {
-      int carry = 0;
-      for (int g0 = 0; g0 < p.groups; g0 += 32) {
-        const int g = g0 + lane;
-        int tiles = 0;
-        if (g < p.groups) {
-          int64_t lo, hi;
-          group_rows(p, g, lo, hi);
-          tiles = static_cast<int>((hi - lo + BM - 1) / BM);
-        }
-        int incl = tiles;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += v;
-        }
-        if (g < p.groups) tile_prefix[g] = carry + incl - tiles;
-        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-      if (lane == 0) {
-        tile_prefix[p.groups] = carry;
-        ctrl->num_units = carry * p.n_tiles;
-      }
-    }
+    if (warp == 2) group_table(p, tile_prefix, lane, &ctrl->num_units);
   } else if (threadIdx.x == 0) {
     ctrl->num_units = p.num_units;
   }
