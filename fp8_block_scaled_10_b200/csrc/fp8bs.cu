@@ -283,9 +283,9 @@ double kb_time_us(GemmKind kind, int bn) {
 // waves of work units x K blocks per unit x kb_time_us, plus, for a K split,
 // the FP32 partials' round trip through HBM and the reduction launch.  When
 // the tiles fill the GPU but their last wave would keep at most half of the
-// SMs busy, the promotion kernel can split only the tiles of that wave along
-// K ("split tail"): the whole waves run unchanged and the tail's partials,
-// a few MB, are summed by a small reduction.
+// SMs busy, the plan can split only the tiles of that wave along
+// K ("split tail", both kernels): the whole waves run unchanged and the
+// tail's partials, a few MB, are summed by a small reduction.
 //
 // M <= 128 (decode): the weight stream from HBM bounds every tile width
 // alike; the score is the fraction of persistent slots kept busy, with a
@@ -320,8 +320,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
         if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
           t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
         const int64_t tail = tiles % slots;
-        if (kind == GemmKind::kPromotion && splits == 1 && tiles > slots && tail > 0 &&
-            2 * tail <= slots) {
+        if (splits == 1 && tiles > slots && tail > 0 && 2 * tail <= slots) {
           const size_t tile_bytes = static_cast<size_t>(128) * bn * sizeof(float);
           const int64_t by_ws = static_cast<int64_t>(kTailWorkspaceCap / (tail * tile_bytes));
           const int ts = static_cast<int>(std::min<int64_t>({slots / tail, kbn / 4, by_ws}));
@@ -508,10 +507,23 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   p.splits = pl.splits;
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
+  p.full_units = pl.full_units;
+  p.tail_tiles = pl.tail_tiles;
+  p.tail_splits = pl.tail_splits;
+  p.tail_kbps = pl.tail_kbps;
+  p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   p.groups = 1;
   cudaError_t e = pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, ty, p, pl.grid, st)
                                : launch_gemm_bs<128, false>(ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
+  if (pl.tail_splits > 0) {
+    const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
+    e = launch(gemm::tail_reduce_kernel, grid_for(items, 256, info->sms * 8), 256, 0, st,
+               static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), M,
+               static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles, pl.tail_splits,
+               pl.bn);
+    if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
+  }
   if (pl.splits > 1) {
     const int64_t MN = M * N;
     e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,

@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
       const bool row_ok = row < t.row_end;
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
       const uint32_t acc_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
-      if (p.splits == 1) {
+      if (p.splits == 1 && t.tail_slot < 0) {
         // Read all of this warp's columns as packed bf16 first and hand the
         // accumulator back, so the next tile's MMAs start before the stores.
         uint32_t h[NCH][16];
@@ -414,6 +414,18 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
             if (lane == 0) mbar_arrive(&tempty[tb]);
           }
           const int64_t col = col0 + 32 * c;
+          if (!GROUPED && t.tail_slot >= 0) {
+            // FP32 partial of a split tail unit: the whole 128 x BN tile
+            // (rows and columns past the matrix are masked by the reduction).
+            float* dst = p.tail_ws + (static_cast<int64_t>(t.tail_slot) * BM + row_in_tile) * BN +
+                         g * CPW + 32 * c;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(dst + 4 * q) =
+                  make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                              __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+            continue;
+          }
           if (slab_tma) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {

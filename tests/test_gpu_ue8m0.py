@@ -40,6 +40,8 @@ def _case(M, N, K, seed, heavy=False):
 @pytest.mark.parametrize("M,N,K", [
     (128, 256, 512), (1, 256, 128), (127, 576, 512), (129, 130, 256), (300, 384, 1024),
     (256, 512, 7168), (513, 1280, 384), (64, 2048, 2048), (2, 18432, 256), (200, 136, 128),
+    # 160 tiles on 148 SMs: the last wave's tiles split along K, ragged edges
+    (1200, 4000, 4096),
 ])
 def test_gemm_ue8m0_shapes(M, N, K):
     x, qa, sa, qw, sw = _case(M, N, K, seed=M + 2 * N + K)
