@@ -78,16 +78,21 @@ def peaks():
 # distributed plumbing (timing only: barrier and max over ranks)
 # ---------------------------------------------------------------------------
 class Dist:
-    def __init__(self):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE from torchrun).  The
+    benchmark's only collectives are the timing barrier and the max over ranks;
+    "nccl" on GPUs, "gloo" where the tests run it on CPU."""
+
+    def __init__(self, backend="nccl", timeout_s=120):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
             self.pg = dist
 
     def barrier(self):
@@ -95,9 +100,11 @@ class Dist:
             self.pg.barrier()
 
     def max(self, v):
+        """The largest v over all ranks (every rank calls it, in the same order)."""
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
@@ -206,6 +213,11 @@ class Linear:
         st = self.L.fp8bs_fp8_gemm_ue8m0(vp(self.q), vp(self.s), vp(self.qw), vp(self.sw), self.m,
                                          self.n, self.k, vp(self.y), vp(self.ws), self.nws, stream)
         assert st == 0, self.L.fp8bs_last_error_message()
+
+
+def whole_job_tflops(flops_per_step, steps, world, max_ms):
+    """Whole-job throughput: the FLOPs every rank ran over the slowest rank's time."""
+    return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
 
 
 def time_events(fn, iters, flush=None):
@@ -428,7 +440,7 @@ def ours(args, dist):
     aq_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     total_ms = dist.max(total_ms)
     ms_per_step = total_ms / args.steps
-    value = flops * dist.world * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, dist.world, total_ms)
     assert fp8bs.device_error() == 0
 
     # ---- end to end through the C ABI: pinned host x in, host y out, every step
@@ -450,7 +462,7 @@ def ours(args, dist):
     b.record()
     torch.cuda.synchronize()
     e2e_ms = dist.max(a.elapsed_time(b))
-    e2e_value = flops * dist.world * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(flops, e2e_steps, dist.world, e2e_ms)
 
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     aq_bytes = M * K * 3 + M * (K // 128) * 4
