@@ -50,7 +50,7 @@ FP8_OVER_BF16 = 2.0     # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLO
 # DRAM bytes (read + write) of one prefill GEMM launch from the ncu capture
 # summarised in profiles/fp8_gemm_prefill_M4096_N18432_K7168.md.  It belongs
 # to the kernel as captured; reset it to None whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES = 165.717504e6 + 131.728384e6
+GEMM_TRAFFIC_BYTES = 165.936128e6 + 134.464768e6
 
 
 def parse_args():
@@ -220,19 +220,24 @@ def whole_job_tflops(flops_per_step, steps, world, max_ms):
     return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
 
 
-def time_events(fn, iters, flush=None):
-    """Mean device time (ms) of fn() over iters launches, each bracketed by events
-    on the current stream; flush() (untimed) runs before each one."""
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(iters)]
-    for a, b in evs:
-        if flush:
-            flush()
-        a.record()
-        fn()
-        b.record()
-    torch.cuda.synchronize()
-    return sum(a.elapsed_time(b) for a, b in evs) / iters
+def time_events(fn, iters, flush=None, rounds=3):
+    """Device time (ms) of fn(): the median over `rounds` rounds of the mean over
+    iters launches, each launch bracketed by events on the current stream;
+    flush() (untimed) runs before each one.  The median of rounds keeps one
+    disturbed round (the GPUs are shared) from setting the number."""
+    means = []
+    for _ in range(rounds):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(iters)]
+        for a, b in evs:
+            if flush:
+                flush()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        means.append(sum(a.elapsed_time(b) for a, b in evs) / iters)
+    return statistics.median(means)
 
 
 def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
@@ -493,7 +498,7 @@ def ours(args, dist):
     torch.cuda.empty_cache()
     if not args.quick:
         result["parts"] = run_parts(fp8bs, wl, hbm, fp8_peak, stream)
-        result["parts_note"] = "each part: mean of 10 event-timed launches after 3 warm-ups; memory-bound parts and decode GEMMs flush L2 before each launch (memset of 4x L2 size, then a read of 2x L2 size so no dirty lines are written back inside the timed launch); GB/s of algorithmic bytes vs %s HBM %.1f GB/s" % (peak_kind, hbm)
+        result["parts_note"] = "each part: median over 3 rounds of the mean of 10 event-timed launches, after 3 warm-ups; memory-bound parts and decode GEMMs flush L2 before each launch (memset of 4x L2 size, then a read of 2x L2 size so no dirty lines are written back inside the timed launch); GB/s of algorithmic bytes vs %s HBM %.1f GB/s" % (peak_kind, hbm)
     if dist.rank == 0:
         rows, run, _ = cpu_baseline(args.cpu_seconds)
         t = run(rows)
