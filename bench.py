@@ -325,6 +325,28 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
                     "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
                     "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
             del lin
+    # FP8-output GEMM (the epilogue quantizes y for the next layer) against the
+    # bf16-output GEMM followed by act_quant of y, prefill K=7168, N=18432
+    lin = Linear(fp8bs, wl, wl.PREFILL_M, 7168, 18432, fmt=0, seed=300)
+    mm, nn, kk = lin.m, lin.n, lin.k
+    lin.act_quant(stream)
+    q_out = torch.empty(mm, nn, dtype=torch.uint8, device="cuda")
+    s_out = torch.empty(mm, nn // 128, dtype=torch.float32, device="cuda")
+    fl = 2 * mm * nn * kk
+    for ofmt, oname in ((0, "none"), (1, "ue8m0")):
+        fq = lambda: L.fp8bs_fp8_gemm_quant(vp(lin.q), vp(lin.s), vp(lin.qw), vp(lin.sw), mm, nn, kk,
+                                            ofmt, vp(q_out), vp(s_out), None, stream)
+        fs = lambda: (lin.gemm(stream),
+                      L.fp8bs_act_quant(vp(lin.y), 0, mm, nn, 128, ofmt, vp(q_out), vp(s_out), stream))
+        for _ in range(3):
+            fq(); fs()
+        ms_q = time_events(fq, 10)
+        ms_s = time_events(fs, 10)
+        parts["prefill_K7168_N18432_fp8_output_" + oname] = {
+            "fused_us": ms_q * 1e3, "fused_TFLOP/s": fl / ms_q / 1e9,
+            "gemm_then_act_quant_us": ms_s * 1e3,
+            "note": "fp8bs_fp8_gemm_quant vs fp8bs_fp8_gemm + fp8bs_act_quant of the bf16 y"}
+    del lin, q_out, s_out
     # expert-batched grouped GEMM: 32 x W [2048, 7168], 65536 routed rows
     counts = wl.expert_counts(wl.EXPERT_TOKENS * wl.EXPERT_TOPK, wl.EXPERTS, seed=70)
     offs = torch.cat([torch.zeros(1, dtype=torch.int64), counts.cumsum(0)]).cuda()

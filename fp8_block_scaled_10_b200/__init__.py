@@ -14,6 +14,7 @@ the pages describe:
 * ``fp8_gemm(a, a_s, b, b_s) -> y``
 * ``fp8_linear(x, weight, weight_scale, scale_fmt=None) -> y``
 * ``fp8_gemm_grouped(a, a_s, w, w_s, m_offsets) -> y``
+* ``fp8_gemm_quant(a, a_s, b, b_s, out_scale_fmt=None) -> (q, s)`` (FP8 output)
 * ``weight_quant(w, block_size=128, scale_fmt=None) -> (q, s)``
 """
 import ctypes
@@ -24,7 +25,7 @@ import torch
 
 __all__ = [
     "act_quant", "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
-    "fp8_gemm_grouped", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
+    "fp8_gemm_grouped", "fp8_gemm_quant", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
     "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -79,6 +80,7 @@ def lib():
         "fp8bs_fp8_linear_ue8m0": (i32, [p, i64, i64, p, p, i64, p, p, p, p, sz, p]),
         "fp8bs_fp8_gemm_grouped_ue8m0": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
         "fp8bs_fp8_gemm_grouped": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
+        "fp8bs_fp8_gemm_quant": (i32, [p, p, p, p, i64, i64, i64, i32, p, p, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -222,6 +224,28 @@ def fp8_gemm(a, a_s, b, b_s, scale_fmt=None):
     _check(fn(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, _ptr(y), _ptr(ws), nws,
               _stream(a.device)))
     return y
+
+
+def fp8_gemm_quant(a, a_s, b, b_s, out_scale_fmt=None, return_y=False):
+    """fp8_gemm with an FP8 output: y = a @ b^T rounded to bf16, then quantized
+    per 1x128 block of each row as act_quant(y, 128, out_scale_fmt) would.
+
+    Returns (q e4m3fn [..., N], s float32 [..., N/128]), plus the bf16 y when
+    return_y.  N must be a multiple of 128."""
+    a, b = _codes(a), _codes(b)
+    _need_cuda(a, a_s, b, b_s)
+    K = a.shape[-1]
+    M = a.numel() // K if K else 0
+    N = b.shape[0]
+    q = torch.empty(*a.shape[:-1], N, dtype=torch.uint8, device=a.device)
+    s = torch.empty(*a.shape[:-1], N // 128 if N % 128 == 0 else 1, dtype=torch.float32,
+                    device=a.device)
+    y = torch.empty(*a.shape[:-1], N, dtype=torch.bfloat16, device=a.device) if return_y else None
+    _check(lib().fp8bs_fp8_gemm_quant(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K,
+                                      _scale_fmt(out_scale_fmt), _ptr(q), _ptr(s), _ptr(y),
+                                      _stream(a.device)))
+    q = q.view(torch.float8_e4m3fn)
+    return (q, s, y) if return_y else (q, s)
 
 
 def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,

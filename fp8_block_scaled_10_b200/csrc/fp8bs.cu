@@ -931,3 +931,72 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
 }
 
 }  // extern "C"
+
+extern "C" {
+
+fp8bs_status fp8bs_fp8_gemm_quant(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                  const float* w_s, int64_t M, int64_t N, int64_t K,
+                                  fp8bs_scale_fmt out_fmt, uint8_t* q_out, float* s_out,
+                                  uint16_t* y, void* stream) {
+  fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, reinterpret_cast<uint16_t*>(q_out), N, K);
+  if (r != FP8BS_OK) return r;
+  if (N % 128 != 0)
+    return fail(FP8BS_ERR_INVALID_ARG, "N=%lld must be a multiple of 128 (1x128 output blocks)",
+                (long long)N);
+  if (out_fmt != FP8BS_SCALE_FMT_NONE && out_fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "out_fmt");
+  if (s_out == nullptr || (reinterpret_cast<uintptr_t>(s_out) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "s_out must be a 4-byte aligned device pointer");
+  if (y != nullptr && !aligned16(y)) return fail(FP8BS_ERR_INVALID_ARG, "y must be 16-byte aligned");
+  if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (M == 0) return FP8BS_OK;
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  // One 128 x 256 tile per unit, no K split: each epilogue thread then owns
+  // exactly one 1x128 block of its output row.
+  const int bn = 256;
+  const int a_rows = a_rows_for(M);
+  CUtensorMap ta, tw, tq;
+  gemm::Params p{};
+  if ((r = make_tmap(&ta, a, M, K, a_rows)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, bn)) != FP8BS_OK) return r;
+  {
+    // q_out [M, N] uint8 in boxes of 32 rows x 64 codes, 64-byte swizzle.
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N)};
+    const cuuint32_t box[2] = {64u, 32u};
+    const cuuint32_t elem[2] = {1u, 1u};
+    const CUresult cr = g_encode(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_out, dims, strides, box,
+                                 elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)cr);
+  }
+  const int m_tiles = static_cast<int>((M + 127) / 128);
+  const int n_tiles = static_cast<int>((N + bn - 1) / bn);
+  const int64_t units = static_cast<int64_t>(m_tiles) * n_tiles;
+  if (units > (int64_t(1) << 31) - 1) return fail(FP8BS_ERR_INVALID_ARG, "problem too large");
+  p.sa = a_s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.M = M;
+  p.N = static_cast<int>(N);
+  p.kbn = static_cast<int>(K / 128);
+  p.nbn = static_cast<int>((N + 127) / 128);
+  p.m_tiles = m_tiles;
+  p.n_tiles = n_tiles;
+  p.splits = 1;
+  p.kb_per_split = p.kbn;
+  p.num_units = static_cast<int>(units);
+  p.groups = 1;
+  p.y_tma = 3;
+  p.q_out = q_out;
+  p.s_out = s_out;
+  p.q_ue8m0 = out_fmt == FP8BS_SCALE_FMT_UE8M0 ? 1 : 0;
+  const int grid = static_cast<int>(std::min<int64_t>(units, info->sms));
+  const cudaError_t e = launch_gemm_any<false>(bn, a_rows, ta, tw, tq, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_quant launch");
+  return FP8BS_OK;
+}
+
+}  // extern "C"

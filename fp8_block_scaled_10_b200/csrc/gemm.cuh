@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "quant.cuh"
 #include "sm100.cuh"
 
 namespace fp8bs {
@@ -86,6 +87,13 @@ struct Params {
   int tail_splits;
   int tail_kbps;
   float* tail_ws;
+  // FP8 output (dense, BN = 256, one split): instead of storing y, the
+  // epilogue rounds each row's 128-column block to bf16 and quantizes it as
+  // act_quant would (q_out [M, N] e4m3 codes, s_out [M, N/128]); y (nullable)
+  // then receives the bf16 values too.  With y_tma == 3, tmap_y maps q_out.
+  uint8_t* q_out;
+  float* s_out;
+  int q_ue8m0;
 };
 
 // Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
@@ -634,6 +642,59 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
           tb = 0;
           tphase ^= 1u;
         }
+      }
+      if (!GROUPED && BN == 256 && p.q_out != nullptr) {
+        // FP8 output: this thread's 128 columns of its row are one 1x128
+        // block of y.  Same steps as act_quant on the bf16 y: round to bf16,
+        // amax over the bf16 values, s = block_scale(amax), q = e4m3(y / s).
+        const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
+        if (col0 < p.N) {
+          uint32_t hb[CPW / 2];
+          float amax = 0.0f;
+#pragma unroll
+          for (int j = 0; j < CPW / 2; ++j) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[j].x, acc[j].y);
+            hb[j] = *reinterpret_cast<const uint32_t*>(&b2);
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(hb[j] << 16)),
+                                     fabsf(__uint_as_float(hb[j] & 0xFFFF0000u))));
+          }
+          const float sc = block_scale(amax, p.q_ue8m0 != 0);
+          const float r = __frcp_rn(sc);
+          uint32_t codes[CPW / 4];
+#pragma unroll
+          for (int h = 0; h < CPW / 8; ++h) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              v[2 * j] = __uint_as_float(hb[4 * h + j] << 16);
+              v[2 * j + 1] = __uint_as_float(hb[4 * h + j] & 0xFFFF0000u);
+            }
+            const uint2 c = p.q_ue8m0 ? quantize8<true>(v, sc, r) : quantize8<false>(v, sc, r);
+            codes[2 * h] = c.x;
+            codes[2 * h + 1] = c.y;
+          }
+          if (row_ok) p.s_out[row * (p.N / 128) + col0 / 128] = sc;
+          const int64_t slab0 = t.row0 + quad * 32;
+          if (p.y_tma == 3 && slab0 < t.row_end) {
+            uint8_t* box = out_boxes + e * kOutBoxBytes;
+#pragma unroll
+            for (int c = 0; c < CPW / 64; ++c)
+              store_out_box(&tmap_y, box, lane, *reinterpret_cast<const uint32_t(*)[16]>(&codes[16 * c]),
+                            static_cast<int32_t>(col0 + 64 * c), static_cast<int32_t>(slab0));
+          } else if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(p.q_out + row * p.N + col0);
+#pragma unroll
+            for (int c = 0; c < CPW / 16; ++c)
+              dst[c] = make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
+          }
+          if (p.y != nullptr && row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(p.y + row * p.N + col0);
+#pragma unroll
+            for (int c = 0; c < CPW / 8; ++c)
+              dst[c] = make_uint4(hb[4 * c], hb[4 * c + 1], hb[4 * c + 2], hb[4 * c + 3]);
+          }
+        }
+        continue;
       }
       if (!GROUPED && t.tail_slot >= 0) {
         // FP32 partial of a split tail unit: the whole 128 x BN tile, rows and

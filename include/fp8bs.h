@@ -298,6 +298,30 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t *m_
                                                     const float *w_s, int64_t N, int64_t K,
                                                     uint16_t *y, void *stream);
 
+/*
+ * fp8_gemm_quant: fp8_gemm with an FP8 output, for a following FP8 linear.
+ * The product y = a * w^T (same operands, layouts, constraints and
+ * tolerance as fp8_gemm, any fp32 scales) is rounded to bf16 and quantized
+ * exactly as fp8bs_act_quant(y_bf16, block = 128, out_fmt) would quantize it:
+ * per 1x128 block of each output row, s = max(amax, 1e-4) / 448 (ue8m0:
+ * the next power of two up), q = e4m3(y / s).  This is the "fuse the
+ * activation quantization into the producing GEMM's epilogue" step that the
+ * pages' linear layer leaves to a separate act_quant call ("Understanding
+ * Dynamic and Static Activation Quantization Schemes in DeepSeek-V3", "How
+ * Dynamic Activation Quantization Works"; the fused form has no counterpart on
+ * the pages and is checked bit for bit against fp8bs_act_quant of the bf16 y).
+ *   q_out  device, [M, N] uint8 (e4m3fn codes), 16-byte aligned
+ *   s_out  device, [M, N / 128] float32
+ *   y      device, [M, N] bf16, or NULL; when given it receives the bf16 y
+ *          that q_out and s_out quantize.
+ * N % 128 == 0 (else FP8BS_ERR_INVALID_ARG).  Needs no workspace.  Runs the
+ * promotion kernel with 128 x 256 tiles and no K split.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_quant(const uint8_t *a, const float *a_s, const uint8_t *w,
+                                            const float *w_s, int64_t M, int64_t N, int64_t K,
+                                            fp8bs_scale_fmt out_fmt, uint8_t *q_out, float *s_out,
+                                            uint16_t *y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -69,10 +69,19 @@ def test_host_side_argument_errors_without_gpu(L):
     # grouped: G out of range
     st = L.fp8bs_fp8_gemm_grouped(0, dummy, 8, dummy, dummy, dummy, dummy, 256, 128, dummy, None)
     assert st == fp8bs.ERR_INVALID_ARG
+    # FP8-output GEMM: N must be a multiple of 128, the output format known
+    st = L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 8, 200, 128, 0, dummy, dummy, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG and b"N=200" in L.fp8bs_last_error_message()
+    st = L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 8, 256, 128, 5, dummy, dummy, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    st = L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 8, 256, 128, 0, dummy, None, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG
     # empty problems are successful no-ops
     assert L.fp8bs_act_quant(None, 0, 0, 256, 128, 0, None, None, None) == fp8bs.OK
     assert L.fp8bs_weight_dequant(None, None, 0, 16, 128, None, 0, None) == fp8bs.OK
     assert L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 0, 256, 128, dummy, None, 0, None) == fp8bs.OK
+    assert L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 0, 256, 128, 0, dummy, dummy, None,
+                                  None) == fp8bs.OK
 
 
 def test_binding_refuses_cpu_tensors():
