@@ -222,16 +222,30 @@ def whole_job_tflops(flops_per_step, steps, world, max_ms):
 
 def time_events(fn, iters, flush=None, rounds=3):
     """Device time (ms) of fn(): the median over `rounds` rounds of the mean over
-    iters launches, each launch bracketed by events on the current stream;
-    flush() (untimed) runs before each one.  The median of rounds keeps one
-    disturbed round (the GPUs are shared) from setting the number."""
+    iters launches, timed with events on the current stream.  With flush(),
+    each launch is bracketed by its own events and flush() (untimed) runs
+    before it; without, one event pair spans the iters back-to-back launches.
+    The median of rounds keeps one disturbed round (the GPUs are shared) from
+    setting the number."""
     means = []
     for _ in range(rounds):
+        if flush is None:
+            # Back-to-back launches between one pair of events: the GPU time per
+            # launch, with the host's per-call work (argument checks, tensor
+            # maps, launch) overlapped by the launches already queued.
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            for _ in range(iters):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            means.append(a.elapsed_time(b) / iters)
+            continue
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(iters)]
         for a, b in evs:
-            if flush:
-                flush()
+            flush()          # long enough on the GPU that the host's launch work stays ahead
             a.record()
             fn()
             b.record()
@@ -268,6 +282,15 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
         ms = time_events(f, 10, flush)
         parts[name] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nbytes / ms / 1e6,
                        "frac_hbm": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    # the configurable block size (the pages' default is 128)
+    for blk in (32, 64, 256):
+        f = lambda: L.fp8bs_act_quant(vp(x), 0, R, C, blk, 0, vp(q), vp(s), stream)
+        for _ in range(3):
+            f()
+        ms = time_events(f, 10, flush)
+        nb = R * C * 3 + R * (C // blk) * 4
+        parts["act_quant_none_block%d" % blk] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                                                 "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
     del x, q, s
     # weight_dequant, e4m3 [18432, 7168] -> bf16, s [144, 56]
     R, C = 18432, 7168
@@ -281,7 +304,28 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
     ms = time_events(f, 10, flush)
     parts["weight_dequant"] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nbytes / ms / 1e6,
                                "frac_hbm": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    for blk in (64, 256):
+        sb = wl.uniform((-(-R // blk), -(-C // blk)), 1e-5, 1e-3, seed=32, device="cuda")
+        f = lambda: L.fp8bs_weight_dequant(vp(qw), vp(sb), R, C, blk, vp(y), 0, stream)
+        for _ in range(3):
+            f()
+        ms = time_events(f, 10, flush)
+        nb = R * C * 3 + sb.numel() * 4
+        parts["weight_dequant_block%d" % blk] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                                                 "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
     del qw, sw, y
+    # weight_quant (the offline quantizer as a library call), fp32 [18432, 7168]
+    wf = wl.weight_f32(R, C, seed=33, device="cuda")
+    qo = torch.empty(R, C, dtype=torch.uint8, device="cuda")
+    so = torch.empty(R // 128, C // 128, dtype=torch.float32, device="cuda")
+    f = lambda: L.fp8bs_weight_quant(vp(wf), 1, R, C, 128, 0, vp(qo), vp(so), stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10, flush)
+    nb = R * C * (4 + 1) + so.numel() * 4
+    parts["weight_quant_f32"] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                                 "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
+    del wf, qo, so
     # decode GEMMs (ue8m0 scales), bytes = W + w_s + A + a_s + y
     for kk, nn in wl.DECODE_KN:
         lin = None

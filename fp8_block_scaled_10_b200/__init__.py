@@ -176,7 +176,7 @@ def weight_dequant(x, s, block_size=128, out_dtype=torch.bfloat16):
 
 
 def weight_quant(w, block_size=128, scale_fmt=None):
-    """128 x 128 block quantization of a dense 2-D weight -> (q e4m3fn, s float32)."""
+    """block_size x block_size quantization of a dense 2-D weight -> (q e4m3fn, s float32)."""
     _need_cuda(w)
     if w.dim() != 2:
         raise ValueError("weight_quant expects a 2-D weight")

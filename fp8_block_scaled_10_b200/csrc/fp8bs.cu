@@ -236,6 +236,28 @@ InvariantDiv invariant_div(uint32_t d) {
   return InvariantDiv{static_cast<uint32_t>(m), l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
 }
 
+// log2 of a supported quantization block size (32, 64, 128 or 256), else -1.
+int block_log2(int64_t block) {
+  switch (block) {
+    case 32: return 5;
+    case 64: return 6;
+    case 128: return 7;
+    case 256: return 8;
+  }
+  return -1;
+}
+
+template <typename T, bool UE>
+cudaError_t launch_act_quant(int64_t block, int grid, cudaStream_t st, const T* x, uint8_t* q,
+                             float* s, int64_t nblocks) {
+  switch (block) {
+    case 32: return launch(act_quant_kernel<T, UE, 32>, grid, kActThreads, 0, st, x, q, s, nblocks);
+    case 64: return launch(act_quant_kernel<T, UE, 64>, grid, kActThreads, 0, st, x, q, s, nblocks);
+    case 256: return launch(act_quant_kernel<T, UE, 256>, grid, kActThreads, 0, st, x, q, s, nblocks);
+    default: return launch(act_quant_kernel<T, UE, 128>, grid, kActThreads, 0, st, x, q, s, nblocks);
+  }
+}
+
 int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
   const int64_t need = (work_items + per_cta - 1) / per_cta;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, max_ctas)));
@@ -536,7 +558,8 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
 fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
                            int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
                            cudaStream_t st) {
-  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  if (block_log2(block) < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
   if (rows < 0 || cols <= 0 || cols % block != 0)
     return fail(FP8BS_ERR_INVALID_ARG, "cols=%lld must be a positive multiple of block", (long long)cols);
   if (x_dtype != FP8BS_DTYPE_BF16 && x_dtype != FP8BS_DTYPE_F32)
@@ -551,19 +574,20 @@ fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int
   DeviceInfo* info;
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
-  const int64_t nblocks = rows * (cols / 128);
-  // (kActThreads / kActLanes) blocks per CTA per unroll step; up to 8 CTAs per SM.
-  const int grid = grid_for(nblocks, (kActThreads / kActLanes) * kActUnroll, info->sms * 8);
+  const int64_t nblocks = rows * (cols / block);
+  // Each thread holds 32 elements: kActThreads * 32 / block blocks per CTA per
+  // step; up to 8 CTAs per SM.
+  const int grid = grid_for(nblocks, (kActThreads * kActElems / block) * kActUnroll, info->sms * 8);
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   cudaError_t e;
   if (x_dtype == FP8BS_DTYPE_BF16) {
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
-    e = ue ? launch(act_quant_kernel<__nv_bfloat16, true>, grid, kActThreads, 0, st, xb, q, s, nblocks)
-           : launch(act_quant_kernel<__nv_bfloat16, false>, grid, kActThreads, 0, st, xb, q, s, nblocks);
+    e = ue ? launch_act_quant<__nv_bfloat16, true>(block, grid, st, xb, q, s, nblocks)
+           : launch_act_quant<__nv_bfloat16, false>(block, grid, st, xb, q, s, nblocks);
   } else {
     const auto* xf = static_cast<const float*>(x);
-    e = ue ? launch(act_quant_kernel<float, true>, grid, kActThreads, 0, st, xf, q, s, nblocks)
-           : launch(act_quant_kernel<float, false>, grid, kActThreads, 0, st, xf, q, s, nblocks);
+    e = ue ? launch_act_quant<float, true>(block, grid, st, xf, q, s, nblocks)
+           : launch_act_quant<float, false>(block, grid, st, xf, q, s, nblocks);
   }
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return FP8BS_OK;
@@ -617,7 +641,9 @@ fp8bs_status fp8bs_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, i
 
 fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, int64_t N,
                                   int64_t block, void* y, fp8bs_dtype y_dtype, void* stream) {
-  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  const int lb = block_log2(block);
+  if (lb < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
   if (M < 0 || N < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
   if (y_dtype != FP8BS_DTYPE_BF16 && y_dtype != FP8BS_DTYPE_F32)
     return fail(FP8BS_ERR_INVALID_ARG, "y_dtype");
@@ -630,7 +656,7 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
   cudaStream_t st = as_stream(stream);
-  const int64_t nbn = (N + 127) / 128;
+  const int64_t nbn = (N + block - 1) / block;
   const bool bf = y_dtype == FP8BS_DTYPE_BF16;
   cudaError_t e;
   if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
@@ -639,13 +665,13 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
     const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
     const InvariantDiv row_div = invariant_div(cpr);
     e = bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
-                    row_div, nbn)
+                    row_div, nbn, lb)
            : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
-                    row_div, nbn);
+                    row_div, nbn, lb);
   } else {
     const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
-    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn)
-           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn);
+    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn, lb)
+           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn, lb);
   }
   if (e != cudaSuccess) return cuda_fail(e, "weight_dequant launch");
   return FP8BS_OK;
@@ -654,7 +680,9 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
 fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, int64_t N,
                                 int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
                                 void* stream) {
-  if (block != 128) return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (only 128 is implemented)", (long long)block);
+  const int lb = block_log2(block);
+  if (lb < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
   if (M < 0 || N < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
   if (w_dtype != FP8BS_DTYPE_BF16 && w_dtype != FP8BS_DTYPE_F32)
     return fail(FP8BS_ERR_INVALID_ARG, "w_dtype");
@@ -662,7 +690,7 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
     return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
   if (M == 0 || N == 0) return FP8BS_OK;
   if (!w || !q || !s) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
-  const int64_t rb = (M + 127) / 128, cb = (N + 127) / 128;
+  const int64_t rb = (M + block - 1) / block, cb = (N + block - 1) / block;
   if (rb > 65535 || cb > 0x7FFFFFFF) return fail(FP8BS_ERR_INVALID_ARG, "matrix too large");
   int dev;
   DeviceInfo* info;
@@ -674,10 +702,10 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
   cudaError_t e;
   if (w_dtype == FP8BS_DTYPE_F32)
     e = launch(weight_quant_kernel<float>, grid, 256, 0, st, static_cast<const float*>(w), q, s,
-               M, N, cb, ue);
+               M, N, cb, ue, lb);
   else
     e = launch(weight_quant_kernel<__nv_bfloat16>, grid, 256, 0, st,
-               static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue);
+               static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue, lb);
   if (e != cudaSuccess) return cuda_fail(e, "weight_quant launch");
   return FP8BS_OK;
 }

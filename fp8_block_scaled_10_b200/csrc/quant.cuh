@@ -146,23 +146,25 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 // ---------------------------------------------------------------------------
 // act_quant
 // ---------------------------------------------------------------------------
-// The input is a flat run of nblocks blocks of 128 elements (the last
-// dimension is a multiple of 128, so blocks never straddle rows) and block b's
-// scale is s[b].  kActLanes lanes own one block, each holding 128 / kActLanes
-// consecutive elements; the amax is a log2(kActLanes)-step xor shuffle among
-// them, each thread computes one scale per block and writes its code bytes.
-// A warp covers (32 / kActLanes) * kActUnroll consecutive blocks per
-// iteration with all loads issued first.
+// The input is a flat run of nblocks blocks of BLOCK elements (the last
+// dimension is a multiple of BLOCK, so blocks never straddle rows) and block
+// b's scale is s[b].  BLOCK / 32 lanes own one block, each holding 32
+// consecutive elements; the amax is a log2(BLOCK / 32)-step xor shuffle among
+// them, each thread computes the block's scale and writes its code bytes.  A
+// warp covers 32 * 32 / BLOCK consecutive blocks per iteration with all loads
+// issued first.  The pages' block size is 128 (the default of the
+// block_size parameter); 32, 64 and 256 are the other sizes built.
 constexpr int kActThreads = 256;
-constexpr int kActLanes = 4;
 constexpr int kActUnroll = 1;
-constexpr int kActElems = 128 / kActLanes;
-constexpr int kActBlocksPerWarp = 32 / kActLanes;
+constexpr int kActElems = 32;
 
-template <typename T, bool UE8M0>
+template <typename T, bool UE8M0, int BLOCK = 128>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const T* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
                      int64_t nblocks) {
+  constexpr int kActLanes = BLOCK / kActElems;
+  constexpr int kActBlocksPerWarp = 32 / kActLanes;
+  static_assert(BLOCK == 32 || BLOCK == 64 || BLOCK == 128 || BLOCK == 256, "block size");
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kActThreads)
     for (int u = 0; u < kActUnroll; ++u) {
       const int64_t b = base + kActBlocksPerWarp * u + group;
       if (b < nblocks) {
-        const T* p = x + b * 128 + li * kActElems;
+        const T* p = x + b * BLOCK + li * kActElems;
 #pragma unroll
         for (int h = 0; h < kActElems / 8; ++h)
           load8(p + 8 * h, *reinterpret_cast<float(*)[8]>(&v[u][8 * h]));
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kActThreads)
       const float sc = block_scale(amax, UE8M0);
       const float r = __frcp_rn(sc);
       if (b < nblocks) {
-        uint8_t* qp = q + b * 128 + li * kActElems;
+        uint8_t* qp = q + b * BLOCK + li * kActElems;
 #pragma unroll
         for (int h = 0; h < kActElems / 16; ++h) {
           const uint2 lo = quantize8<UE8M0>(*reinterpret_cast<const float(*)[8]>(&v[u][16 * h]), sc, r);
@@ -273,7 +275,7 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
                           void* __restrict__ y, uint32_t total_chunks, uint32_t chunks_per_row,
-                          InvariantDiv row_div, int64_t nbn) {
+                          InvariantDiv row_div, int64_t nbn, int lb) {
   pdl_trigger();
   pdl_wait();
   const uint32_t stride = gridDim.x * kDeqThreads * kDeqUnroll;
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kDeqThreads)
         const uint32_t col = (c - row * chunks_per_row) * 16;
         off[u] = static_cast<int64_t>(c) * 16;
         raw[u] = __ldcs(reinterpret_cast<const uint4*>(q + off[u]));
-        sc[u] = __ldg(s + (row >> 7) * nbn + (col >> 7));
+        sc[u] = __ldg(s + (row >> lb) * nbn + (col >> lb));
       } else {
         off[u] = -1;
       }
@@ -340,14 +342,14 @@ __global__ void __launch_bounds__(kDeqThreads)
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_any_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
-                              void* __restrict__ y, int64_t M, int64_t N, int64_t nbn) {
+                              void* __restrict__ y, int64_t M, int64_t N, int64_t nbn, int lb) {
   pdl_trigger();
   pdl_wait();
   const int64_t total = M * N;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDeqThreads + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * kDeqThreads) {
     const int64_t row = i / N, col = i - row * N;
-    const float v = e4m3_value(q[i]) * __ldg(s + (row >> 7) * nbn + (col >> 7));
+    const float v = e4m3_value(q[i]) * __ldg(s + (row >> lb) * nbn + (col >> lb));
     if (OUT_BF16)
       static_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
     else
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kDeqThreads)
 }
 
 // ---------------------------------------------------------------------------
-// weight_quant: one CTA per 128 x 128 tile (partial at the edges)
+// weight_quant: one CTA per block x block tile (partial at the edges)
 // ---------------------------------------------------------------------------
 template <typename T>
 __device__ __forceinline__ float load_elem(const T* p);
@@ -372,17 +374,18 @@ __device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p
 template <typename T>
 __global__ void __launch_bounds__(256)
     weight_quant_kernel(const T* __restrict__ w, uint8_t* __restrict__ q, float* __restrict__ s,
-                        int64_t M, int64_t N, int64_t nbn, bool ue8m0) {
+                        int64_t M, int64_t N, int64_t nbn, bool ue8m0, int lb) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[8];
   const int64_t bi = blockIdx.y, bj = blockIdx.x;
-  const int64_t r0 = bi * 128, c0 = bj * 128;
-  const int rows = static_cast<int>(M - r0 < 128 ? M - r0 : 128);
-  const int cols = static_cast<int>(N - c0 < 128 ? N - c0 : 128);
+  const int blk = 1 << lb;
+  const int64_t r0 = bi * blk, c0 = bj * blk;
+  const int rows = static_cast<int>(M - r0 < blk ? M - r0 : blk);
+  const int cols = static_cast<int>(N - c0 < blk ? N - c0 : blk);
   float amax = 0.0f;
-  for (int e = threadIdx.x; e < rows * 128; e += 256) {
-    const int r = e >> 7, c = e & 127;
+  for (int e = threadIdx.x; e < (rows << lb); e += 256) {
+    const int r = e >> lb, c = e & (blk - 1);
     if (c < cols) amax = fmaxf(amax, fabsf(load_elem(w + (r0 + r) * N + c0 + c)));
   }
   for (int off = 16; off >= 1; off >>= 1)
@@ -393,8 +396,8 @@ __global__ void __launch_bounds__(256)
   for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
   const float sc = block_scale(amax, ue8m0);
   if (threadIdx.x == 0) s[bi * nbn + bj] = sc;
-  for (int e = threadIdx.x; e < rows * 128; e += 256) {
-    const int r = e >> 7, c = e & 127;
+  for (int e = threadIdx.x; e < (rows << lb); e += 256) {
+    const int r = e >> lb, c = e & (blk - 1);
     if (c < cols) {
       const int64_t i = (r0 + r) * N + c0 + c;
       q[i] = static_cast<uint8_t>(e4m3x2(__fdiv_rn(load_elem(w + i), sc), 0.0f) & 0xFFu);

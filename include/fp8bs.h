@@ -50,7 +50,7 @@ extern "C" {
 typedef enum fp8bs_status {
     FP8BS_OK = 0,
     FP8BS_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or shape; nothing launched */
-    FP8BS_ERR_UNSUPPORTED = 2, /* well-formed but not implemented (e.g. block != 128)    */
+    FP8BS_ERR_UNSUPPORTED = 2, /* well-formed but not implemented (e.g. block = 48)      */
     FP8BS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size()   */
     FP8BS_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                      */
     FP8BS_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up (device error word) */
@@ -96,8 +96,10 @@ FP8BS_API fp8bs_status fp8bs_get_device_error(void *stream, int *code);
  *   x      device, [rows, cols], bf16 (x_dtype = BF16) or fp32 (F32)
  *   q      device, [rows, cols], e4m3fn codes (uint8), written
  *   s      device, [rows, cols / block], fp32, written
- * cols must be a multiple of block; block must be 128 (others return
- * FP8BS_ERR_UNSUPPORTED).  rows == 0 is a no-op.  Results are bit-exact with
+ * cols must be a multiple of block.  block is 128 in the pages' layers and
+ * is configurable ([DEQ] "Per-Block Scaling Architecture": block_size is a
+ * parameter); 32, 64, 128 and 256 are implemented, other sizes return
+ * FP8BS_ERR_UNSUPPORTED.  rows == 0 is a no-op.  Results are bit-exact with
  * the definition above.
  */
 FP8BS_API fp8bs_status fp8bs_act_quant(const void *x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
@@ -113,19 +115,21 @@ FP8BS_API fp8bs_status fp8bs_act_quant(const void *x, fp8bs_dtype x_dtype, int64
  *   s      device, [cdiv(M, block), cdiv(N, block)] fp32, row-major, so the
  *          scale of block (bi, bj) sits at bi * cdiv(N, block) + bj
  *   y      device, [M, N], bf16 (y_dtype = BF16) or fp32 (F32), written
- * Ragged M and N are allowed (edge blocks are partial).  block must be 128.
+ * Ragged M and N are allowed (edge blocks are partial).  block is 32, 64,
+ * 128 or 256 (else FP8BS_ERR_UNSUPPORTED).
  * M == 0 or N == 0 is a no-op.  Bit-exact with the definition above.
  */
 FP8BS_API fp8bs_status fp8bs_weight_dequant(const uint8_t *q, const float *s, int64_t M, int64_t N,
                                   int64_t block, void *y, fp8bs_dtype y_dtype, void *stream);
 
 /*
- * weight_quant: the inverse of weight_dequant, 128 x 128 block quantization of
+ * weight_quant: the inverse of weight_dequant, block x block quantization of
  * a dense weight with the act_quant scale rule applied per tile:
  *   s[bi, bj] = max(amax_tile, 1e-4f) / 448.0f (optionally rounded up to 2^k)
- *   q[i, j]   = e4m3fn_rne_satfinite(w[i, j] / s[i / 128, j / 128])
+ *   q[i, j]   = e4m3fn_rne_satfinite(w[i, j] / s[i / block, j / block])
  *   w      device, [M, N], bf16 or fp32
- *   q      device, [M, N] uint8, written;  s  device, [cdiv(M,128), cdiv(N,128)] fp32, written
+ *   q      device, [M, N] uint8, written;  s  device, [cdiv(M,block), cdiv(N,block)] fp32, written
+ * block is 32, 64, 128 (the pages' weight_block_size) or 256.
  * Ragged M and N are allowed.  The pages state the per-tile scale layout that
  * weight_dequant consumes ([DEQ] "Per-Block Scaling Architecture"); they do
  * not print the offline quantizer, whose rule is read here as the activation

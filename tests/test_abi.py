@@ -57,9 +57,11 @@ def test_host_side_argument_errors_without_gpu(L):
     # misaligned operand
     st = L.fp8bs_fp8_gemm(_p(4097), dummy, dummy, dummy, 8, 256, 128, dummy, None, 0, None)
     assert st == fp8bs.ERR_INVALID_ARG
-    # block sizes other than 128 are not implemented
-    st = L.fp8bs_act_quant(dummy, 0, 4, 256, 64, 0, dummy, dummy, None)
+    # block sizes other than 32, 64, 128 and 256 are not implemented
+    st = L.fp8bs_act_quant(dummy, 0, 4, 192, 48, 0, dummy, dummy, None)
     assert st == fp8bs.ERR_UNSUPPORTED
+    assert L.fp8bs_weight_dequant(dummy, dummy, 4, 4, 512, dummy, 0, None) == fp8bs.ERR_UNSUPPORTED
+    assert L.fp8bs_weight_quant(dummy, 0, 4, 4, 16, 0, dummy, dummy, None) == fp8bs.ERR_UNSUPPORTED
     # last dimension not a multiple of the block
     st = L.fp8bs_act_quant(dummy, 0, 4, 200, 128, 0, dummy, dummy, None)
     assert st == fp8bs.ERR_INVALID_ARG

@@ -117,6 +117,21 @@ def test_act_quant_many_midpoints_fp32():
     assert np.array_equal(u8(q), q_ref)
 
 
+@pytest.mark.parametrize("block", [32, 64, 256])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+def test_act_quant_other_block_sizes(block, fmt, dtype):
+    """The configurable block_size: 1 x block scales, bit-exact with the oracle."""
+    rows, cols = 257, 7 * 256
+    x = wl.normal_with_outliers(rows, cols, seed=block + 3, frac=0.01, factor=50.0, dtype=dtype)
+    q, s = fp8bs.act_quant(x.cuda(), block, fmt)
+    arr = wl.bf16_bits(x) if dtype == torch.bfloat16 else x.numpy()
+    q_ref, s_ref = oracle.act_quant(arr, block=block, scale_fmt=fmt)
+    assert tuple(s.shape) == (rows, cols // block)
+    assert np.array_equal(u8(q), q_ref)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
+
+
 @pytest.mark.parametrize("fmt", [None, "ue8m0"])
 def test_act_quant_full_size(fmt):
     """act_quant on x bf16 [16384, 7168] ~N(0,1) with 0.1% entries x100, every byte."""
@@ -179,6 +194,29 @@ def test_weight_dequant_every_code_and_scale_range(out):
     fin = ~np.isnan(r)
     assert fin.mean() > 0.99
     assert np.array_equal(f32bits(g[fin]), f32bits(r[fin]))
+
+
+@pytest.mark.parametrize("block", [32, 64, 256])
+@pytest.mark.parametrize("shape", [(300, 1024), (129, 130), (256, 7 * 64)])
+def test_weight_dequant_other_block_sizes(block, shape):
+    M, N = shape
+    rng = np.random.default_rng(M + N + block)
+    q = rng.integers(0, 254, (M, N)).astype(np.uint8)
+    q = np.where(q >= 0x7F, q + 1, q).astype(np.uint8)
+    s = rng.uniform(1e-5, 1e-3, (-(-M // block), -(-N // block))).astype(np.float32)
+    y = fp8bs.weight_dequant(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(), block)
+    ref = oracle.weight_dequant(q, s, block=block)
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("block", [32, 64, 256])
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+def test_weight_quant_other_block_sizes(block, fmt):
+    w = wl.weight_f32(300, 576, seed=block)
+    q, s = fp8bs.weight_quant(w.cuda(), block, fmt)
+    q_ref, s_ref = oracle.weight_quant(w.numpy(), block=block, scale_fmt=fmt)
+    assert np.array_equal(u8(q), q_ref)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
 
 
 def test_weight_dequant_pages_example_shape():

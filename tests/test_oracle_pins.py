@@ -278,6 +278,44 @@ def test_act_quant_matches_library_division_and_cast():
             assert np.array_equal(q, ref)
 
 
+@pytest.mark.parametrize("block", [32, 64, 256])
+def test_act_quant_other_block_sizes_match_library_ops(block):
+    """block_size is configurable: per 1 x block run, amax (torch max), the
+    clamp and /448 in fp32, the ue8m0 round-up as an exact power-of-two
+    ceiling (frexp), then torch's division and torch's e4m3 cast."""
+    g = torch.Generator().manual_seed(block)
+    x = torch.randn(24, 8 * block, generator=g) * 2
+    x[torch.rand(x.shape, generator=g) < 0.02] *= 40
+    x[3, :block] = 0.0                                   # an all-zero block
+    for fmt in (None, "ue8m0"):
+        q, s = oracle.act_quant(x.numpy(), block=block, scale_fmt=fmt)
+        assert s.shape == (24, 8)
+        amax = x.abs().reshape(24, 8, block).amax(dim=-1)
+        a = torch.clamp(amax, min=float(f32(CLAMP)))
+        sref = (a / torch.tensor(448.0)).numpy().astype(np.float32)
+        if fmt == "ue8m0":
+            m, e = np.frexp(sref.astype(np.float64))
+            sref = np.where(m == 0.5, sref, np.ldexp(1.0, e)).astype(np.float32)
+        assert np.array_equal(s.view(np.uint32), sref.view(np.uint32))
+        st = torch.from_numpy(s).repeat_interleave(block, dim=1)
+        ref = (x / st).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(q, ref)
+
+
+@pytest.mark.parametrize("block", [32, 64, 256])
+def test_weight_dequant_other_block_sizes_match_library_ops(block):
+    M, N = 2 * block + 5, 3 * block - 7
+    g = torch.Generator().manual_seed(block + 1)
+    codes = torch.randint(0, 254, (M, N), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8)
+    rb, cb = -(-M // block), -(-N // block)
+    s = torch.rand(rb, cb, generator=g) * (1e-3 - 1e-5) + 1e-5
+    y = oracle.weight_dequant(codes.numpy(), s.numpy(), block=block)
+    st = s.repeat_interleave(block, 0)[:M].repeat_interleave(block, 1)[:, :N]
+    deq = codes.view(torch.float8_e4m3fn).float() * st
+    assert np.array_equal(y, deq.bfloat16().view(torch.int16).numpy().view(np.uint16))
+
+
 # --------------------------------------------------------------------------
 # Test-data weight quantizer
 # --------------------------------------------------------------------------
