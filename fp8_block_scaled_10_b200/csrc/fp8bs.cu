@@ -700,6 +700,20 @@ fp8bs_status fp8bs_weight_quant(const void* w, fp8bs_dtype w_dtype, int64_t M, i
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   cudaStream_t st = as_stream(stream);
   cudaError_t e;
+  if (block == 128) {
+    // One pass with the tile in registers; rows of 16 (bf16) or 8 (fp32)
+    // bytes per 4 elements must be aligned for the vector loads.
+    const size_t esz = w_dtype == FP8BS_DTYPE_F32 ? 4 : 2;
+    const bool vec_ok = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(w) % (4 * esz)) == 0 &&
+                        (reinterpret_cast<uintptr_t>(q) % 4) == 0;
+    e = w_dtype == FP8BS_DTYPE_F32
+            ? launch(weight_quant128_kernel<float>, grid, 256, 0, st, static_cast<const float*>(w),
+                     q, s, M, N, cb, ue, vec_ok)
+            : launch(weight_quant128_kernel<__nv_bfloat16>, grid, 256, 0, st,
+                     static_cast<const __nv_bfloat16*>(w), q, s, M, N, cb, ue, vec_ok);
+    if (e != cudaSuccess) return cuda_fail(e, "weight_quant launch");
+    return FP8BS_OK;
+  }
   if (w_dtype == FP8BS_DTYPE_F32)
     e = launch(weight_quant_kernel<float>, grid, 256, 0, st, static_cast<const float*>(w), q, s,
                M, N, cb, ue, lb);

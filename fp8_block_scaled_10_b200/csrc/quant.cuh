@@ -405,6 +405,83 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// weight_quant for 128 x 128 tiles, one pass: the tile stays in registers.
+// Thread t owns columns 4 * (t % 32) .. +3 of rows t / 32 + 8 k (k < 16), so
+// every warp-wide load reads 128 consecutive elements of one row and every
+// warp-wide store writes 128 consecutive codes.  The tile amax is a warp
+// shuffle then a reduction over the 8 warps in shared memory; the scale is the
+// act_quant rule and each quotient is the correctly rounded w / s (Markstein's
+// correction, as in act_quant), so the codes are those of the two-pass
+// kernel.  Elements past the matrix's ragged edges read as 0 and are not
+// stored.
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(p));
+  v[0] = __uint_as_float(raw.x << 16);
+  v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(raw.y << 16);
+  v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    weight_quant128_kernel(const T* __restrict__ w, uint8_t* __restrict__ q, float* __restrict__ s,
+                           int64_t M, int64_t N, int64_t nbn, bool ue8m0, bool vec_ok) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 128, c0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int64_t col = c0 + 4 * lane;
+  float v[16][4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int64_t row = r0 + wid + 8 * k;
+    if (row < M && vec_ok && col + 4 <= N) {
+      load4(w + row * N + col, v[k]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        v[k][j] = (row < M && col + j < N) ? load_elem(w + row * N + col + j) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(v[k][j]));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  if (lane == 0) red[wid] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = block_scale(amax, ue8m0);
+  if (threadIdx.x == 0) s[static_cast<int64_t>(blockIdx.y) * nbn + blockIdx.x] = sc;
+  const float r = __frcp_rn(sc);
+#pragma unroll
+  for (int k = 0; k < 16; k += 2) {
+    const float v8[8] = {v[k][0], v[k][1], v[k][2], v[k][3], v[k + 1][0], v[k + 1][1], v[k + 1][2], v[k + 1][3]};
+    const uint2 c = ue8m0 ? quantize8<true>(v8, sc, r) : quantize8<false>(v8, sc, r);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t row = r0 + wid + 8 * (k + h);
+      const uint32_t codes = h ? c.y : c.x;
+      if (row >= M) continue;
+      if (vec_ok && col + 4 <= N) {
+        *reinterpret_cast<uint32_t*>(q + row * N + col) = codes;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (col + j < N) q[row * N + col + j] = static_cast<uint8_t>(codes >> (8 * j));
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Split-K reduction: y[m, n] = bf16(sum_s ws[s][m][n]), summed in split order.
 // ---------------------------------------------------------------------------
