@@ -77,6 +77,7 @@ def lib():
         "fp8bs_fp8_gemm_static_scratch": (i32, [p, p, p, p, i64, i64, i64, p, p]),
         "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
         "fp8bs_fp8_gemm_ue8m0": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
+        "fp8bs_fp8_gemm_f32": (i32, [p, p, p, p, i64, i64, i64, i32, p, p, sz, p]),
         "fp8bs_fp8_linear_ue8m0": (i32, [p, i64, i64, p, p, i64, p, p, p, p, sz, p]),
         "fp8bs_fp8_gemm_grouped_ue8m0": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
         "fp8bs_fp8_gemm_grouped": (i32, [i64, p, i64, p, p, p, p, i64, i64, p, p]),
@@ -206,21 +207,29 @@ def _workspace(M, N, K, device):
     return torch.empty(n, dtype=torch.uint8, device=device), n
 
 
-def fp8_gemm(a, a_s, b, b_s, scale_fmt=None):
-    """y = a @ b^T on block-scaled FP8 operands, bf16 output.
+def fp8_gemm(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.bfloat16):
+    """y = a @ b^T on block-scaled FP8 operands.
 
     a: [..., K] e4m3fn, a_s: [..., K/128] float32, b: [N, K] e4m3fn,
-    b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] bfloat16.
+    b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] of out_dtype
+    (torch.bfloat16, or torch.float32 for the unrounded FP32 accumulator).
     scale_fmt="ue8m0" promises that every scale is a power of two and uses
     the tensor core's block-scaled MMA."""
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
     a, b = _codes(a), _codes(b)
     _need_cuda(a, a_s, b, b_s)
     K = a.shape[-1]
     M = a.numel() // K if K else 0
     N = b.shape[0]
-    y = torch.empty(*a.shape[:-1], N, dtype=torch.bfloat16, device=a.device)
+    y = torch.empty(*a.shape[:-1], N, dtype=out_dtype, device=a.device)
     ws, nws = _workspace(M, N, K, a.device)
-    fn = lib().fp8bs_fp8_gemm_ue8m0 if _scale_fmt(scale_fmt) else lib().fp8bs_fp8_gemm
+    fmt = _scale_fmt(scale_fmt)
+    if out_dtype == torch.float32:
+        _check(lib().fp8bs_fp8_gemm_f32(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, fmt,
+                                        _ptr(y), _ptr(ws), nws, _stream(a.device)))
+        return y
+    fn = lib().fp8bs_fp8_gemm_ue8m0 if fmt else lib().fp8bs_fp8_gemm
     _check(fn(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, _ptr(y), _ptr(ws), nws,
               _stream(a.device)))
     return y

@@ -169,15 +169,17 @@ static_assert(gemm::BsCfg<128>::smem_bytes(true) <= kMaxSmemOptin, "smem");
 // cols] in boxes of 32 rows x 32 columns (needs cols % 8 == 0, a 16-byte row
 // pitch).  Several: the FP32 workspace [splits][rows][cols] in boxes of 32
 // rows x 16 columns of one split (needs cols % 4 == 0), so rows past M are
-// clipped inside each split.  Both in the 64-byte swizzle the epilogue stages
-// them in.  Otherwise *map is zeroed and the kernel stores directly
-// (y_tma = 0).
+// clipped inside each split; an FP32 y with one split is mapped the same way
+// as a workspace of one split (ws = y).  Both in the 64-byte swizzle the
+// epilogue stages them in.  Otherwise *map is zeroed and the kernel stores
+// directly (y_tma = 0).
 fp8bs_status make_tmap_out(CUtensorMap* map, const void* y, const void* ws, int64_t rows,
-                           int64_t cols, int splits, int* y_tma) {
+                           int64_t cols, int splits, int* y_tma, bool out_f32 = false) {
   memset(map, 0, sizeof(*map));
   *y_tma = 0;
   CUresult r;
-  if (splits == 1) {
+  if (splits == 1 && out_f32) ws = y;
+  if (splits == 1 && !out_f32) {
     if (cols % 8 != 0) return FP8BS_OK;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
@@ -414,7 +416,7 @@ cudaError_t launch_gemm_any(int bn, int a_rows, const CUtensorMap& ta, const CUt
 }
 
 fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
-                                 const float* w_s, uint16_t* y, int64_t N, int64_t K) {
+                                 const float* w_s, const void* y, int64_t N, int64_t K) {
   if (!a || !a_s || !w || !w_s || !y) return fail(FP8BS_ERR_INVALID_ARG, "null operand pointer");
   if (K <= 0 || K % 128 != 0) return fail(FP8BS_ERR_INVALID_ARG, "K=%lld must be a positive multiple of 128", (long long)K);
   if (N <= 0 || N > (1 << 30)) return fail(FP8BS_ERR_INVALID_ARG, "N=%lld out of range", (long long)N);
@@ -426,8 +428,8 @@ fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8
 }
 
 fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
-                      int64_t M, int64_t N, int64_t K, uint16_t* y, void* ws, size_t ws_bytes,
-                      cudaStream_t st) {
+                      int64_t M, int64_t N, int64_t K, void* y, void* ws, size_t ws_bytes,
+                      cudaStream_t st, bool out_f32 = false) {
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
@@ -447,11 +449,12 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   const int a_rows = pl.bn == 192 ? 128 : a_rows_for(M);
   if ((r = make_tmap(&ta, a, M, K, a_rows)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
-  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma, out_f32)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
-  p.ws = static_cast<float*>(ws);
+  p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
+  p.out_f32 = out_f32 ? 1 : 0;
   p.m_offsets = nullptr;
   p.M = M;
   p.N = static_cast<int>(N);
@@ -472,16 +475,25 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.tail_splits > 0) {
     const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
-    e = launch(gemm::tail_reduce_kernel, grid_for(items, 256, info->sms * 8), 256, 0, st,
-               static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), M,
-               static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles, pl.tail_splits,
-               pl.bn);
+    e = out_f32
+            ? launch(gemm::tail_reduce_kernel<float>, grid_for(items, 256, info->sms * 8), 256, 0,
+                     st, static_cast<const float*>(ws), static_cast<float*>(y), M,
+                     static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles,
+                     pl.tail_splits, pl.bn)
+            : launch(gemm::tail_reduce_kernel<__nv_bfloat16>, grid_for(items, 256, info->sms * 8),
+                     256, 0, st, static_cast<const float*>(ws),
+                     reinterpret_cast<__nv_bfloat16*>(y), M, static_cast<int>(N), pl.m_tiles,
+                     pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
     if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
   }
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,
-        static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
+    e = out_f32 ? launch(splitk_reduce_kernel<float>, grid_for(MN, 256 * 4, info->sms * 8), 256,
+                         0, st, static_cast<const float*>(ws), static_cast<float*>(y), MN,
+                         pl.splits)
+                : launch(splitk_reduce_kernel<__nv_bfloat16>, grid_for(MN, 256 * 4, info->sms * 8),
+                         256, 0, st, static_cast<const float*>(ws),
+                         reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
     if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
   return FP8BS_OK;
@@ -497,8 +509,8 @@ cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const C
 
 // Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel.
 fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
-                         int64_t M, int64_t N, int64_t K, uint16_t* y, void* ws, size_t ws_bytes,
-                         cudaStream_t st) {
+                         int64_t M, int64_t N, int64_t K, void* y, void* ws, size_t ws_bytes,
+                         cudaStream_t st, bool out_f32 = false) {
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
@@ -514,11 +526,12 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   gemm::Params p{};
   if ((r = make_tmap(&ta, a, M, K, 128)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
-  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma, out_f32)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
-  p.ws = static_cast<float*>(ws);
+  p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
+  p.out_f32 = out_f32 ? 1 : 0;
   p.m_offsets = nullptr;
   p.M = M;
   p.N = static_cast<int>(N);
@@ -540,16 +553,25 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
   if (pl.tail_splits > 0) {
     const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
-    e = launch(gemm::tail_reduce_kernel, grid_for(items, 256, info->sms * 8), 256, 0, st,
-               static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), M,
-               static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles, pl.tail_splits,
-               pl.bn);
+    e = out_f32
+            ? launch(gemm::tail_reduce_kernel<float>, grid_for(items, 256, info->sms * 8), 256, 0,
+                     st, static_cast<const float*>(ws), static_cast<float*>(y), M,
+                     static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles,
+                     pl.tail_splits, pl.bn)
+            : launch(gemm::tail_reduce_kernel<__nv_bfloat16>, grid_for(items, 256, info->sms * 8),
+                     256, 0, st, static_cast<const float*>(ws),
+                     reinterpret_cast<__nv_bfloat16*>(y), M, static_cast<int>(N), pl.m_tiles,
+                     pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
     if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
   }
   if (pl.splits > 1) {
     const int64_t MN = M * N;
-    e = launch(splitk_reduce_kernel, grid_for(MN, 256 * 4, info->sms * 8), 256, 0, st,
-        static_cast<const float*>(ws), reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
+    e = out_f32 ? launch(splitk_reduce_kernel<float>, grid_for(MN, 256 * 4, info->sms * 8), 256,
+                         0, st, static_cast<const float*>(ws), static_cast<float*>(y), MN,
+                         pl.splits)
+                : launch(splitk_reduce_kernel<__nv_bfloat16>, grid_for(MN, 256 * 4, info->sms * 8),
+                         256, 0, st, static_cast<const float*>(ws),
+                         reinterpret_cast<__nv_bfloat16*>(y), MN, pl.splits);
     if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
   return FP8BS_OK;
@@ -847,6 +869,18 @@ fp8bs_status fp8bs_fp8_gemm_ue8m0(const uint8_t* a, const float* a_s, const uint
                                   const float* w_s, int64_t M, int64_t N, int64_t K, uint16_t* y,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   return run_gemm_bs(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream));
+}
+
+fp8bs_status fp8bs_fp8_gemm_f32(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                const float* w_s, int64_t M, int64_t N, int64_t K,
+                                fp8bs_scale_fmt fmt, float* y, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fp8bs::fail(FP8BS_ERR_INVALID_ARG, "scale format %d", (int)fmt);
+  if (fmt == FP8BS_SCALE_FMT_UE8M0)
+    return run_gemm_bs(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream),
+                       true);
+  return run_gemm(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream), true);
 }
 
 fp8bs_status fp8bs_fp8_linear_ue8m0(const uint16_t* x, int64_t M, int64_t K, const uint8_t* w,

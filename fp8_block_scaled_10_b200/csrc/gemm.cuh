@@ -63,7 +63,8 @@ struct Params {
   const float* sa;          // [M_total, kbn]
   const float* sw;          // [G][nbn][kbn]
   __nv_bfloat16* y;         // [M_total, N]
-  float* ws;                // [splits][M][N] FP32 partials when splits > 1
+  float* ws;                // [splits][M][N] FP32 partials when splits > 1; with
+                            // out_f32 and one split, the FP32 output y itself
   const int64_t* m_offsets; // grouped mode: [G + 1] prefix row offsets (device)
   int64_t M;                // rows of A (M_total in grouped mode)
   int N;
@@ -94,6 +95,10 @@ struct Params {
   uint8_t* q_out;
   float* s_out;
   int q_ue8m0;
+  // FP32 output: y is stored unrounded, through the FP32 partial path (one
+  // split: ws = y, y_tma 2 maps y as a single split; several: the reduction
+  // writes FP32).  p.y is unused then.
+  int out_f32;
 };
 
 // Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
@@ -737,7 +742,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
                         static_cast<int32_t>(slab0));
         }
       } else if (row_ok) {
-        if (p.splits == 1) {
+        if (p.splits == 1 && !p.out_f32) {
           __nv_bfloat16* yrow = p.y + row * p.N;
 #pragma unroll
           for (int c = 0; c < CPW / 8; ++c) {
@@ -788,10 +793,12 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
   }
 }
 
-// Sum of the FP32 partials of the split tail tiles, in split order, as bf16
-// into y.  One thread per 4 consecutive columns of one tile row.
+// Sum of the FP32 partials of the split tail tiles, in split order, into y
+// (bf16, rounded to nearest even, or FP32).  One thread per 4 consecutive
+// columns of one tile row.
+template <typename OutT>
 __global__ void __launch_bounds__(256)
-    tail_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ y, int64_t M,
+    tail_reduce_kernel(const float* __restrict__ ws, OutT* __restrict__ y, int64_t M,
                        int N, int m_tiles, int full_units, int tail_tiles, int splits, int bn) {
   pdl_trigger();
   pdl_wait();
@@ -812,9 +819,17 @@ __global__ void __launch_bounds__(256)
           ws + ((static_cast<int64_t>(tt) * splits + sp) * BM + r) * bn + c));
       s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
     }
-    __nv_bfloat16* dst = y + row * N + col;
+    OutT* dst = y + row * N + col;
     const float v4[4] = {s.x, s.y, s.z, s.w};
-    if ((N % 4) == 0 && col + 4 <= N) {
+    if constexpr (std::is_same_v<OutT, float>) {
+      if ((N % 4) == 0 && col + 4 <= N) {
+        *reinterpret_cast<float4*>(dst) = s;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (col + j < N) dst[j] = v4[j];
+      }
+    } else if ((N % 4) == 0 && col + 4 <= N) {
       const __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
       uint2 u;
       u.x = *reinterpret_cast<const uint32_t*>(&lo);

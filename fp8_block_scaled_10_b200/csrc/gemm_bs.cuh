@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
       const bool row_ok = row < t.row_end;
       const int64_t col0 = static_cast<int64_t>(t.n_tile) * BN + g * CPW;
       const uint32_t acc_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
-      if (p.splits == 1 && t.tail_slot < 0) {
+      if (p.splits == 1 && t.tail_slot < 0 && !p.out_f32) {
         // Read all of this warp's columns as packed bf16 first and hand the
         // accumulator back, so the next tile's MMAs start before the stores.
         uint32_t h[NCH][16];

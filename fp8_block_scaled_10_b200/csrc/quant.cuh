@@ -15,6 +15,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -483,10 +484,12 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// Split-K reduction: y[m, n] = bf16(sum_s ws[s][m][n]), summed in split order.
+// Split-K reduction: y[m, n] = sum_s ws[s][m][n], summed in split order, as
+// bf16 (rounded to nearest even) or FP32.
 // ---------------------------------------------------------------------------
+template <typename OutT>
 __global__ void __launch_bounds__(256)
-    splitk_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ y,
+    splitk_reduce_kernel(const float* __restrict__ ws, OutT* __restrict__ y,
                          int64_t MN, int splits) {
   pdl_trigger();
   pdl_wait();
@@ -494,7 +497,10 @@ __global__ void __launch_bounds__(256)
        i += static_cast<int64_t>(gridDim.x) * 256) {
     float acc = 0.0f;
     for (int sp = 0; sp < splits; ++sp) acc += ws[sp * MN + i];
-    y[i] = __float2bfloat16_rn(acc);
+    if constexpr (std::is_same_v<OutT, float>)
+      y[i] = acc;
+    else
+      y[i] = __float2bfloat16_rn(acc);
   }
 }
 

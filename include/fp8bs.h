@@ -243,6 +243,26 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_ue8m0(const uint8_t *a, const float *a_s, 
                                             void *stream);
 
 /*
+ * fp8_gemm_f32: fp8_gemm with an FP32 output ("DeepSeek-V3: How Selective FP8
+ * Stays Stable", "Lower precision is a constrained budget": the FP8 GEMMs'
+ * outputs may be BF16 or FP32).  The same product as fp8bs_fp8_gemm, stored
+ * as the FP32 accumulator without the final rounding to bf16.
+ *
+ *   a, a_s, w, w_s, M, N, K, workspace: as for fp8bs_fp8_gemm (the same
+ *     fp8bs_gemm_workspace_size(M, N, K) bytes suffice);
+ *   fmt   FP8BS_SCALE_FMT_NONE: any positive fp32 scales (per-K-block
+ *         promotion, as fp8bs_fp8_gemm); FP8BS_SCALE_FMT_UE8M0: every scale a
+ *         positive normal power of two (block-scaled MMA, as
+ *         fp8bs_fp8_gemm_ue8m0, with the same FP8BS_ERR_SCALE report);
+ *         anything else is FP8BS_ERR_INVALID_ARG;
+ *   y     device, [M, N] fp32, written (16-byte aligned).
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_f32(const uint8_t *a, const float *a_s, const uint8_t *w,
+                                          const float *w_s, int64_t M, int64_t N, int64_t K,
+                                          fp8bs_scale_fmt fmt, float *y, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+
+/*
  * fp8_linear_ue8m0: act_quant(x, 128, UE8M0) followed by fp8_gemm_ue8m0 on
  * one stream.  Arguments as for fp8bs_fp8_linear; w_s must hold powers of
  * two (weights quantized with the ue8m0 scale format).

@@ -78,10 +78,17 @@ def test_host_side_argument_errors_without_gpu(L):
     assert st == fp8bs.ERR_INVALID_ARG
     st = L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 8, 256, 128, 0, dummy, None, None, None)
     assert st == fp8bs.ERR_INVALID_ARG
+    # FP32-output GEMM: the scale format must be known, K a multiple of 128
+    st = L.fp8bs_fp8_gemm_f32(dummy, dummy, dummy, dummy, 8, 256, 128, 3, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    st = L.fp8bs_fp8_gemm_f32(dummy, dummy, dummy, dummy, 8, 256, 96, 0, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG and b"K=96" in L.fp8bs_last_error_message()
     # empty problems are successful no-ops
     assert L.fp8bs_act_quant(None, 0, 0, 256, 128, 0, None, None, None) == fp8bs.OK
     assert L.fp8bs_weight_dequant(None, None, 0, 16, 128, None, 0, None) == fp8bs.OK
     assert L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 0, 256, 128, dummy, None, 0, None) == fp8bs.OK
+    assert L.fp8bs_fp8_gemm_f32(dummy, dummy, dummy, dummy, 0, 256, 128, 1, dummy, None, 0,
+                                None) == fp8bs.OK
     assert L.fp8bs_fp8_gemm_quant(dummy, dummy, dummy, dummy, 0, 256, 128, 0, dummy, dummy, None,
                                   None) == fp8bs.OK
 
