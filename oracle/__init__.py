@@ -50,6 +50,10 @@ def _load():
         lib.oracle_weight_dequant.argtypes = [c_p, c_p, c_i64, c_i64, c_i64, c_int, c_p]
         lib.oracle_gemm.restype = None
         lib.oracle_gemm.argtypes = [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i64, c_p, c_p]
+        lib.oracle_act_quant_static.restype = None
+        lib.oracle_act_quant_static.argtypes = [c_p, c_int, c_i64, c_i64, c_i64, c_p, c_i64, c_p]
+        lib.oracle_act_dequant.restype = None
+        lib.oracle_act_dequant.argtypes = [c_p, c_p, c_i64, c_i64, c_i64, c_i64, c_int, c_p]
         lib.oracle_num_threads.restype = c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -127,6 +131,57 @@ def act_quant(x, block=128, scale_fmt=None):
     _load().oracle_act_quant(_ptr(x), is_bf16, rows, cols, block,
                              int(scale_fmt == "ue8m0"), _ptr(q), _ptr(s))
     return q, s
+
+
+def _act_input(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return x, 1
+    if x.dtype == np.float32:
+        return x, 0
+    raise TypeError("x must be bf16 bits (uint16) or float32")
+
+
+def _scale_table(s, rows, nblk):
+    """A static scale vector [nblk] (row stride 0) or a per-row table [rows, nblk]."""
+    s = _c(s, np.float32)
+    if s.shape == (nblk,):
+        return s, 0
+    if s.shape == (rows, nblk):
+        return s, nblk
+    raise ValueError("scales must be [cols/block] or [rows, cols/block]")
+
+
+def act_quant_static(x, s, block=128):
+    """Static activation scheme: q = e4m3(x / s) with precomputed scales.
+
+    x: [rows, cols] bf16 bits (uint16) or float32; s: float32 [cols/block]
+    (one scale per block of channels, shared by all rows) or [rows, cols/block].
+    Returns q uint8 [rows, cols]."""
+    x, is_bf16 = _act_input(x)
+    rows, cols = x.shape
+    if cols % block != 0:
+        raise ValueError("last dimension must be a multiple of block")
+    s, stride = _scale_table(s, rows, cols // block)
+    q = np.empty((rows, cols), dtype=np.uint8)
+    _load().oracle_act_quant_static(_ptr(x), is_bf16, rows, cols, block, _ptr(s), stride, _ptr(q))
+    return q
+
+
+def act_dequant(q, s, block=128, out="bf16"):
+    """static_dequant: y = fp8 value * its block's scale (fp32 product).
+
+    q: [rows, cols] uint8; s as for act_quant_static.  out="bf16" returns
+    uint16 bit patterns, out="f32" float32."""
+    q = _c(q, np.uint8)
+    rows, cols = q.shape
+    if cols % block != 0:
+        raise ValueError("last dimension must be a multiple of block")
+    s, stride = _scale_table(s, rows, cols // block)
+    y = np.empty((rows, cols), dtype=np.uint16 if out == "bf16" else np.float32)
+    _load().oracle_act_dequant(_ptr(q), _ptr(s), stride, rows, cols, block, int(out == "bf16"),
+                               _ptr(y))
+    return y
 
 
 def weight_quant(w, block=128, scale_fmt=None):

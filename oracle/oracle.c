@@ -216,6 +216,48 @@ void oracle_act_quant(const void *x, int x_is_bf16, int64_t rows, int64_t cols,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Static activation scheme [P1 "How Static Activation Quantization          */
+/* Differs"]: the scales are fixed ahead of time (from calibration) and      */
+/* stored with the checkpoint, so no amax is taken.  The scale of element    */
+/* (r, c) is s[r * s_row_stride + c / block]: s_row_stride = 0 is one scale   */
+/* per block of channels shared by every row (the static scheme); a stride of */
+/* cols / block is a per-row scale table such as act_quant writes.  Each code */
+/* is the same rule as in act_quant without the scale step:                   */
+/* q = encode(fl32(x / s)), IEEE fp32 division, then the round-to-nearest-    */
+/* even, saturating cast, which now can saturate (|x| may exceed 448 s).      */
+/* ------------------------------------------------------------------------ */
+
+void oracle_act_quant_static(const void *x, int x_is_bf16, int64_t rows, int64_t cols,
+                             int64_t block, const float *s, int64_t s_row_stride, uint8_t *q)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            float sc = s[r * s_row_stride + c / block];
+            q[r * cols + c] = oracle_e4m3_encode(load_x(x, x_is_bf16, r * cols + c) / sc);
+        }
+}
+
+/* Activation dequantization [P1 "How Static Activation Quantization         */
+/* Differs", static_dequant]: value = fp8 value times its block's scale, the */
+/* product in fp32 (the page multiplies q_x.float() by the scales broadcast   */
+/* over each block), stored as fp32 or rounded to bf16 (RNE).  Scale lookup   */
+/* as in oracle_act_quant_static.                                             */
+void oracle_act_dequant(const uint8_t *q, const float *s, int64_t s_row_stride, int64_t rows,
+                        int64_t cols, int64_t block, int y_is_bf16, void *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            float p = (float)oracle_e4m3_decode(q[r * cols + c]) * s[r * s_row_stride + c / block];
+            if (y_is_bf16)
+                ((uint16_t *)y)[r * cols + c] = oracle_bf16_from_f32(p);
+            else
+                ((float *)y)[r * cols + c] = p;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Test-data weight quantizer: the same scale rule over block x block tiles   */
 /* of an fp32 matrix [rows, cols]; edge tiles are partial.  s has            */
 /* cdiv(rows,block) x cdiv(cols,block) entries.  Not a library call: it makes */

@@ -466,3 +466,88 @@ def test_gemm_special_cases():
     # sign: negating A negates y exactly
     yn, _ = oracle.gemm(qa ^ np.uint8(0x80), sa, qw, sw)
     assert np.array_equal(yn, -y)
+
+
+# --------------------------------------------------------------------------
+# static activation scheme: precomputed scales, static_dequant
+# --------------------------------------------------------------------------
+
+def _static_case(rows, nblk, block, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, nblk * block, generator=g) * 2
+    x[torch.rand(x.shape, generator=g) < 0.02] *= 300       # saturating entries
+    s = torch.exp2(torch.rand(nblk, generator=g) * 8 - 6) * (1 + torch.rand(nblk, generator=g))
+    return x, s.to(torch.float32)
+
+
+def _torch_static_codes(x, st):
+    """torch's fp32 division and e4m3 cast; where the rounded quotient lies at
+    or beyond 464 (halfway from 448 to the next binade step, 480) torch gives
+    NaN, and the saturating cast gives the signed maximum 448 (code 0x7E)."""
+    y = x / st
+    ref = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+    big = (y.abs() >= 464).numpy()
+    ref[big] = np.where(y.numpy()[big] < 0, 0xFE, 0x7E)
+    return ref
+
+
+@pytest.mark.parametrize("block", [128, 32, 256])
+def test_act_quant_static_matches_library_division_and_cast(block):
+    x, s = _static_case(20, 6, block, seed=block + 11)
+    for as_bf16 in (False, True):
+        arr = _bf16(x) if as_bf16 else x.numpy()
+        xf = torch.from_numpy(oracle.bf16_bits_to_f32(arr) if as_bf16 else arr.copy())
+        q = oracle.act_quant_static(arr, s.numpy(), block=block)
+        st = s.repeat_interleave(block).unsqueeze(0).expand_as(xf)
+        ref = _torch_static_codes(xf, st)
+        assert np.array_equal(q, ref)
+        assert ((q & 0x7F) == 0x7E).sum() > 0                # saturation was exercised
+
+
+def test_act_quant_static_scale_index_is_the_channel_block():
+    """x = 1 everywhere and s[b] = 2^-b: every row's block b holds 2^b, so a
+    scale looked up by row, or by column modulo the block count, fails."""
+    rows, nblk = 5, 7
+    x = np.ones((rows, nblk * BLOCK), np.float32)
+    s = np.exp2(-np.arange(nblk, dtype=np.float32)).astype(np.float32)
+    q = oracle.act_quant_static(x, s)
+    want = torch_e4m3_bytes(np.exp2(np.arange(nblk, dtype=np.float32)))
+    assert np.array_equal(q, np.broadcast_to(np.repeat(want, BLOCK), q.shape))
+    # and the per-row table form: row r uses s_tab[r, b]
+    s_tab = np.stack([s * np.float32(2.0 ** r) for r in range(rows)]).astype(np.float32)
+    q2 = oracle.act_quant_static(x, s_tab)
+    for r in range(rows):
+        want = torch_e4m3_bytes(np.exp2(np.arange(nblk, dtype=np.float32) - r))
+        assert np.array_equal(q2[r], np.repeat(want, BLOCK))
+
+
+def test_act_quant_static_with_dynamic_scales_is_act_quant():
+    """Given the scales the dynamic scheme computes, as a per-row table, the
+    static quantizer reproduces its codes (same division, same cast)."""
+    x = torch.randn(33, 5 * BLOCK, generator=torch.Generator().manual_seed(21)) * 4
+    arr = _bf16(x)
+    for fmt in (None, "ue8m0"):
+        q, s = oracle.act_quant(arr, scale_fmt=fmt)
+        assert np.array_equal(oracle.act_quant_static(arr, s), q)
+
+
+@pytest.mark.parametrize("block", [128, 64])
+def test_act_dequant_matches_pages_static_dequant(block):
+    """static_dequant as the page writes it: q_x.float() times the scales
+    unsqueezed over the last axis (q viewed as [rows, blocks, block]), in
+    torch fp32, then torch's bf16 cast; and with a per-row table."""
+    rows, nblk = 9, 5
+    g = torch.Generator().manual_seed(block + 5)
+    codes = torch.randint(0, 254, (rows, nblk * block), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8)   # skip the NaN code 0x7F
+    s = (torch.rand(nblk, generator=g) * 1e-2 + 1e-5).to(torch.float32)
+    qf = codes.view(torch.float8_e4m3fn).float().reshape(rows, nblk, block)
+    ref = (qf * s.unsqueeze(-1)).reshape(rows, -1)
+    y32 = oracle.act_dequant(codes.numpy(), s.numpy(), block=block, out="f32")
+    assert np.array_equal(y32.view(np.uint32), ref.numpy().view(np.uint32))
+    y16 = oracle.act_dequant(codes.numpy(), s.numpy(), block=block)
+    assert np.array_equal(y16, ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    s_tab = (torch.rand(rows, nblk, generator=g) * 3 + 0.1).to(torch.float32)
+    ref = (qf * s_tab.unsqueeze(-1)).reshape(rows, -1)
+    y32 = oracle.act_dequant(codes.numpy(), s_tab.numpy(), block=block, out="f32")
+    assert np.array_equal(y32.view(np.uint32), ref.numpy().view(np.uint32))
