@@ -291,7 +291,25 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
         nb = R * C * 3 + R * (C // blk) * 4
         parts["act_quant_none_block%d" % blk] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
                                                  "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
-    del x, q, s
+    # the static activation scheme on the same x: precomputed scales, one per
+    # block of 128 channels shared by all rows (no amax), then static_dequant
+    s_static = wl.uniform((C // 128,), 0.01, 0.5, seed=22, device="cuda")
+    f = lambda: L.fp8bs_act_quant_static(vp(x), 0, R, C, 128, vp(s_static), 0, vp(q), None, stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10, flush)
+    nb = R * C * (2 + 1) + s_static.numel() * 4
+    parts["act_quant_static"] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                                 "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
+    y_act = torch.empty(R, C, dtype=torch.bfloat16, device="cuda")
+    f = lambda: L.fp8bs_act_dequant(vp(q), vp(s_static), 0, R, C, 128, vp(y_act), 0, stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10, flush)
+    nb = R * C * (1 + 2) + s_static.numel() * 4
+    parts["static_dequant"] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                               "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
+    del x, q, s, y_act
     # weight_dequant, e4m3 [18432, 7168] -> bf16, s [144, 56]
     R, C = 18432, 7168
     qw = wl.e4m3_codes(R, C, seed=30, device="cuda")

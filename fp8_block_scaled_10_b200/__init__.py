@@ -24,7 +24,8 @@ import re
 import torch
 
 __all__ = [
-    "act_quant", "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
+    "act_quant", "act_quant_static", "act_dequant", "static_dequant",
+    "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
     "fp8_gemm_grouped", "fp8_gemm_quant", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
     "LIB_PATH", "HEADER_PATH",
 ]
@@ -69,6 +70,8 @@ def lib():
         "fp8bs_act_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
         "fp8bs_weight_dequant": (i32, [p, p, i64, i64, i64, p, i32, p]),
         "fp8bs_weight_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
+        "fp8bs_act_quant_static": (i32, [p, i32, i64, i64, i64, p, i64, p, p, p]),
+        "fp8bs_act_dequant": (i32, [p, p, i64, i64, i64, i64, p, i32, p]),
         "fp8bs_gemm_workspace_size": (sz, [i64, i64, i64]),
         "fp8bs_gemm_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
         "fp8bs_selftest_quotient": (i32, [p, p, p, i64, p]),
@@ -157,6 +160,68 @@ def act_quant(x, block_size=128, scale_fmt=None):
     _check(lib().fp8bs_act_quant(_ptr(x), dt, rows, cols, block_size, _scale_fmt(scale_fmt),
                                  _ptr(q), _ptr(s), _stream(x.device)))
     return q, s
+
+
+def _act_scales(s, lead, cols, block_size):
+    """Row stride of a static scale vector [cols/block] (0) or a per-row table
+    [..., cols/block] (cols/block)."""
+    nblk = cols // block_size
+    if s.dtype != torch.float32 or not s.is_contiguous():
+        raise ValueError("scales must be contiguous float32")
+    if tuple(s.shape) == (nblk,):
+        return 0
+    if tuple(s.shape) == tuple(lead) + (nblk,):
+        return nblk
+    raise ValueError("scales must be [cols/block] (static) or x.shape[:-1] + [cols/block]")
+
+
+def act_quant_static(x, s, block_size=128, return_scales=False):
+    """Static activation scheme: q = e4m3(x / s) with precomputed scales, no amax.
+
+    s: float32 [cols/block_size] (one scale per block of channels, shared by
+    every row) or a per-row table shaped like act_quant's.  Values beyond
+    448 * s saturate.  With return_scales, also returns the per-row table
+    ``x.shape[:-1] + (cols/block_size,)`` that fp8_gemm takes as a_s."""
+    _need_cuda(x, s)
+    if x.dtype == torch.bfloat16:
+        dt = DTYPE_BF16
+    elif x.dtype == torch.float32:
+        dt = DTYPE_F32
+    else:
+        raise TypeError("x must be bfloat16 or float32")
+    cols = x.shape[-1]
+    if cols % block_size != 0:
+        raise ValueError("last dimension must be a multiple of block_size")
+    stride = _act_scales(s, x.shape[:-1], cols, block_size)
+    rows = x.numel() // cols if cols else 0
+    q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s_out = torch.empty(*x.shape[:-1], cols // block_size, dtype=torch.float32,
+                        device=x.device) if return_scales else None
+    _check(lib().fp8bs_act_quant_static(_ptr(x), dt, rows, cols, block_size, _ptr(s), stride,
+                                        _ptr(q), _ptr(s_out), _stream(x.device)))
+    return (q, s_out) if return_scales else q
+
+
+def act_dequant(q, s, block_size=128, out_dtype=torch.float32):
+    """y = q.float() * s per 1 x block_size block (the pages' static_dequant).
+
+    s as for act_quant_static (a static vector or act_quant's per-row
+    table); the fp32 product is returned as float32 or rounded to bfloat16."""
+    q = _codes(q)
+    _need_cuda(q, s)
+    cols = q.shape[-1]
+    if cols % block_size != 0:
+        raise ValueError("last dimension must be a multiple of block_size")
+    stride = _act_scales(s, q.shape[:-1], cols, block_size)
+    rows = q.numel() // cols if cols else 0
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[out_dtype]
+    y = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    _check(lib().fp8bs_act_dequant(_ptr(q), _ptr(s), stride, rows, cols, block_size, _ptr(y), dt,
+                                   _stream(q.device)))
+    return y
+
+
+static_dequant = act_dequant
 
 
 def weight_dequant(x, s, block_size=128, out_dtype=torch.bfloat16):

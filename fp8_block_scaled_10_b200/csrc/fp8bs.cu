@@ -577,6 +577,28 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   return FP8BS_OK;
 }
 
+// y = decode(q) * scale over an M x N code matrix, the scale of (row, col)
+// being s[(row >> row_shift) * s_row_stride + (col >> lb)].
+cudaError_t launch_dequant(const uint8_t* q, const float* s, int64_t M, int64_t N,
+                           int64_t s_row_stride, int row_shift, int lb, void* y, bool bf,
+                           int sms, cudaStream_t st) {
+  if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
+    const uint32_t cpr = static_cast<uint32_t>(N / 16);
+    const uint32_t total = static_cast<uint32_t>(M * (N / 16));
+    const int grid = grid_for(total, kDeqThreads * kDeqUnroll, sms * 16);
+    const InvariantDiv row_div = invariant_div(cpr);
+    return bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
+                       row_div, s_row_stride, row_shift, lb)
+              : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, total,
+                       cpr, row_div, s_row_stride, row_shift, lb);
+  }
+  const int grid = grid_for(M * N, kDeqThreads, sms * 8);
+  return bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, M, N,
+                     s_row_stride, row_shift, lb)
+            : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, M, N,
+                     s_row_stride, row_shift, lb);
+}
+
 fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int64_t cols,
                            int64_t block, fp8bs_scale_fmt fmt, uint8_t* q, float* s,
                            cudaStream_t st) {
@@ -677,25 +699,81 @@ fp8bs_status fp8bs_weight_dequant(const uint8_t* q, const float* s, int64_t M, i
   DeviceInfo* info;
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
-  cudaStream_t st = as_stream(stream);
   const int64_t nbn = (N + block - 1) / block;
-  const bool bf = y_dtype == FP8BS_DTYPE_BF16;
-  cudaError_t e;
-  if (N % 16 == 0 && M * (N / 16) < (int64_t(1) << 32) - kDeqThreads * kDeqUnroll * 8 * 1024) {
-    const uint32_t cpr = static_cast<uint32_t>(N / 16);
-    const uint32_t total = static_cast<uint32_t>(M * (N / 16));
-    const int grid = grid_for(total, kDeqThreads * kDeqUnroll, info->sms * 16);
-    const InvariantDiv row_div = invariant_div(cpr);
-    e = bf ? launch(weight_dequant_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
-                    row_div, nbn, lb)
-           : launch(weight_dequant_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, total, cpr,
-                    row_div, nbn, lb);
-  } else {
-    const int grid = grid_for(M * N, kDeqThreads, info->sms * 8);
-    e = bf ? launch(weight_dequant_any_kernel<true>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn, lb)
-           : launch(weight_dequant_any_kernel<false>, grid, kDeqThreads, 0, st, q, s, y, M, N, nbn, lb);
-  }
+  const cudaError_t e = launch_dequant(q, s, M, N, nbn, lb, lb, y, y_dtype == FP8BS_DTYPE_BF16,
+                                       info->sms, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "weight_dequant launch");
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_act_dequant(const uint8_t* q, const float* s, int64_t s_row_stride,
+                               int64_t rows, int64_t cols, int64_t block, void* y,
+                               fp8bs_dtype y_dtype, void* stream) {
+  const int lb = block_log2(block);
+  if (lb < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
+  if (rows < 0 || cols <= 0 || cols % block != 0)
+    return fail(FP8BS_ERR_INVALID_ARG, "cols=%lld must be a positive multiple of block", (long long)cols);
+  if (s_row_stride != 0 && s_row_stride < cols / block)
+    return fail(FP8BS_ERR_INVALID_ARG, "s_row_stride=%lld must be 0 or at least cols / block",
+                (long long)s_row_stride);
+  if (y_dtype != FP8BS_DTYPE_BF16 && y_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "y_dtype");
+  if (rows == 0) return FP8BS_OK;
+  if (!q || !s || !y) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(y) || (reinterpret_cast<uintptr_t>(s) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "q and y must be 16-byte aligned, s 4-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const cudaError_t e = launch_dequant(q, s, rows, cols, s_row_stride, 0, lb, y,
+                                       y_dtype == FP8BS_DTYPE_BF16, info->sms, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "act_dequant launch");
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_act_quant_static(const void* x, fp8bs_dtype x_dtype, int64_t rows,
+                                    int64_t cols, int64_t block, const float* s,
+                                    int64_t s_row_stride, uint8_t* q, float* s_out,
+                                    void* stream) {
+  const int lb = block_log2(block);
+  if (lb < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
+  if (rows < 0 || cols <= 0 || cols % block != 0)
+    return fail(FP8BS_ERR_INVALID_ARG, "cols=%lld must be a positive multiple of block", (long long)cols);
+  if (s_row_stride != 0 && s_row_stride < cols / block)
+    return fail(FP8BS_ERR_INVALID_ARG, "s_row_stride=%lld must be 0 or at least cols / block",
+                (long long)s_row_stride);
+  if (x_dtype != FP8BS_DTYPE_BF16 && x_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "x_dtype");
+  if (rows == 0) return FP8BS_OK;
+  if (!x || !s || !q) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u) ||
+      (reinterpret_cast<uintptr_t>(s_out) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "x and q must be 16-byte aligned, s and s_out 4-byte aligned");
+  const int64_t chunks = rows * (cols / kStaticElems);
+  if (chunks >= (int64_t(1) << 32) - int64_t(kStaticThreads) * kStaticUnroll * 8 * 1024)
+    return fail(FP8BS_ERR_INVALID_ARG, "rows * cols too large");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const uint32_t cpr = static_cast<uint32_t>(cols / kStaticElems);
+  const uint32_t total = static_cast<uint32_t>(chunks);
+  const int grid = grid_for(total, kStaticThreads * kStaticUnroll, info->sms * 8);
+  const InvariantDiv row_div = invariant_div(cpr);
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e;
+  if (x_dtype == FP8BS_DTYPE_BF16)
+    e = launch(act_quant_static_kernel<__nv_bfloat16>, grid, kStaticThreads, 0, st,
+               static_cast<const __nv_bfloat16*>(x), s, q, s_out, total, cpr, row_div,
+               s_row_stride, cols / block, lb);
+  else
+    e = launch(act_quant_static_kernel<float>, grid, kStaticThreads, 0, st,
+               static_cast<const float*>(x), s, q, s_out, total, cpr, row_div, s_row_stride,
+               cols / block, lb);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_static launch");
   return FP8BS_OK;
 }
 

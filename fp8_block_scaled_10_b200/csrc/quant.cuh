@@ -216,6 +216,125 @@ __global__ void __launch_bounds__(kActThreads)
   }
 }
 
+// Quotient n / d for a divisor fixed per launch, by multiplication
+// (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", 1994, the round-up method): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, t = mulhi(m, n) and
+// n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0).
+struct InvariantDiv {
+  uint32_t m, sh1, sh2;
+};
+
+__device__ __forceinline__ uint32_t div_invariant(uint32_t n, const InvariantDiv& d) {
+  const uint32_t t = __umulhi(n, d.m);
+  return (t + ((n - t) >> d.sh1)) >> d.sh2;
+}
+
+// ---------------------------------------------------------------------------
+// act_quant with precomputed scales (the static activation scheme)
+// ---------------------------------------------------------------------------
+// Thread-chunks of kStaticElems consecutive elements of one row (it divides
+// every block size, so a chunk has one scale): s[row * s_row_stride + (col >> lb)], with
+// s_row_stride = 0 for per-channel-block scales shared by all rows.  With
+// s_out, the chunk that starts a block also writes that scale to
+// s_out[row, block] (the per-row table fp8_gemm reads).
+//
+// q = e4m3_satfinite(RN(x / s)).  For s in [2^-89, 2^100], r = RN(1/s) is a
+// normal number and Markstein's correction (quotient2) yields the correctly
+// rounded quotient whenever it is below 2^10 in magnitude and |x| >= 2^-100;
+// below that |x / s| < 2^-11, which encodes to a signed zero whatever the
+// rounding of the quotient.  A first estimate |x * r| >= 2^10 means a true
+// quotient far above 448, which saturates: that estimate is used as it is
+// (it may be infinite, and the correction would turn inf into NaN).  Scales
+// outside that range (or not positive) take the IEEE division itself.
+// 32 elements per thread and one chunk per loop step measured fastest on
+// B200 (0.86 of the measured copy bandwidth on [16384, 7168] bf16; 16
+// elements or two chunks per step held more registers and ran at 0.68-0.73).
+constexpr int kStaticThreads = 256;
+constexpr int kStaticUnroll = 1;
+constexpr int kStaticElems = 32;   // elements per thread-chunk (divides every block size)
+
+template <int E>
+__device__ __forceinline__ void load_n(const __nv_bfloat16* p, float (&v)[E]) {
+#pragma unroll
+  for (int h = 0; h < E / 8; ++h) load8(p + 8 * h, *reinterpret_cast<float(*)[8]>(&v[8 * h]));
+}
+template <int E>
+__device__ __forceinline__ void load_n(const float* p, float (&v)[E]) {
+#pragma unroll
+  for (int h = 0; h < E / 8; ++h) load8(p + 8 * h, *reinterpret_cast<float(*)[8]>(&v[8 * h]));
+}
+
+// Codes of 16 values sharing the scale sc (r = RN(1/sc) when `recip`).
+__device__ __forceinline__ uint4 quantize16_given_scale(const float* v, float sc, float r,
+                                                        bool recip) {
+  float t[16];
+  if (recip) {
+    const float2 r2 = make_float2(r, r), ns2 = make_float2(-sc, -sc);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 x = make_float2(v[2 * j], v[2 * j + 1]);
+      const float2 q0 = __fmul2_rn(x, r2);
+      const float2 q = quotient2(x, r2, ns2);
+      t[2 * j] = fabsf(q0.x) >= 1024.0f ? q0.x : q.x;
+      t[2 * j + 1] = fabsf(q0.y) >= 1024.0f ? q0.y : q.y;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) t[j] = __fdiv_rn(v[j], sc);
+  }
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    w[j] = e4m3x2(t[4 * j], t[4 * j + 1]) | (e4m3x2(t[4 * j + 2], t[4 * j + 3]) << 16);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kStaticThreads)
+    act_quant_static_kernel(const T* __restrict__ x, const float* __restrict__ s,
+                            uint8_t* __restrict__ q, float* __restrict__ s_out,
+                            uint32_t total_chunks, uint32_t chunks_per_row, InvariantDiv row_div,
+                            int64_t s_row_stride, int64_t nblk, int lb) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int E = kStaticElems;
+  const uint32_t stride = gridDim.x * kStaticThreads * kStaticUnroll;
+  for (uint32_t c0 = blockIdx.x * kStaticThreads * kStaticUnroll + threadIdx.x; c0 < total_chunks;
+       c0 += stride) {
+    float v[kStaticUnroll][E];
+    float sc[kStaticUnroll];
+#pragma unroll
+    for (int u = 0; u < kStaticUnroll; ++u) {
+      const uint32_t c = c0 + u * kStaticThreads;
+      if (c < total_chunks) {
+        const uint32_t row = div_invariant(c, row_div);
+        const uint32_t col = (c - row * chunks_per_row) * E;
+        load_n<E>(x + static_cast<int64_t>(c) * E, v[u]);
+        sc[u] = __ldg(s + static_cast<int64_t>(row) * s_row_stride + (col >> lb));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kStaticUnroll; ++u) {
+      const uint32_t c = c0 + u * kStaticThreads;
+      if (c >= total_chunks) continue;
+      const bool recip = sc[u] >= 0x1p-89f && sc[u] <= 0x1p100f;
+      const float r = recip ? __frcp_rn(sc[u]) : 0.0f;
+      uint8_t* qp = q + static_cast<int64_t>(c) * E;
+#pragma unroll
+      for (int h = 0; h < E / 16; ++h)
+        __stcs(reinterpret_cast<uint4*>(qp + 16 * h),
+               quantize16_given_scale(&v[u][16 * h], sc[u], r, recip));
+      if (s_out != nullptr) {
+        const uint32_t row = div_invariant(c, row_div);
+        const uint32_t col = (c - row * chunks_per_row) * E;
+        if ((col & ((1u << lb) - 1u)) == 0)
+          s_out[static_cast<int64_t>(row) * nblk + (col >> lb)] = sc[u];
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // weight_dequant
 // ---------------------------------------------------------------------------
@@ -236,23 +355,6 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
 constexpr int kDeqThreads = 512;
 constexpr int kDeqUnroll = 2;
 
-// Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row;
-// all 16 share one block scale because 16 divides 128.  Chunk indices fit in
-// 32 bits (the host checks M * N / 16 < 2^32).
-// Quotient n / d for a divisor fixed per launch, by multiplication
-// (Granlund and Montgomery, "Division by Invariant Integers using
-// Multiplication", 1994, the round-up method): with l = ceil(log2 d) and
-// m = floor(2^32 (2^l - d) / d) + 1, t = mulhi(m, n) and
-// n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0).
-struct InvariantDiv {
-  uint32_t m, sh1, sh2;
-};
-
-__device__ __forceinline__ uint32_t div_invariant(uint32_t n, const InvariantDiv& d) {
-  const uint32_t t = __umulhi(n, d.m);
-  return (t + ((n - t) >> d.sh1)) >> d.sh2;
-}
-
 // fp32 bits of (e4m3 value of the byte in bits 24..31 of c) * 2^-120: an
 // arithmetic shift by 4 moves the 7 magnitude bits to 26..20 (exponent field
 // e, mantissa m of e4m3 become the low exponent bits and top mantissa bits of
@@ -267,7 +369,13 @@ __device__ __forceinline__ uint32_t has_nan_code(uint32_t w) {
   return ((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
 }
 
-// Contiguous weights: thread-chunks of 16 codes (one 16-byte load).  The fast
+// Vector path (N % 16 == 0): a thread owns 16 consecutive codes of one row
+// (one 16-byte load); all 16 share one scale because 16 divides every block
+// size.  Chunk indices fit in 32 bits (the host checks M * N / 16 < 2^32).  Element
+// (row, col) takes the scale s[(row >> row_shift) * s_row_stride + (col >> lb)]:
+// row_shift = lb and s_row_stride = cdiv(N, block) for a weight's block x block
+// tiles; row_shift = 0 for activations, s_row_stride = cols / block for a
+// per-row table or 0 for static per-channel-block scales.  The fast
 // path multiplies the shifted decode by s * 2^120, which is exact while
 // |s| < 2^7 (the product of the real factors is q * s, rounded once, as in
 // fl32(decode(q) * s)); chunks with a larger or non-finite scale, or with a
@@ -276,7 +384,7 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
                           void* __restrict__ y, uint32_t total_chunks, uint32_t chunks_per_row,
-                          InvariantDiv row_div, int64_t nbn, int lb) {
+                          InvariantDiv row_div, int64_t s_row_stride, int row_shift, int lb) {
   pdl_trigger();
   pdl_wait();
   const uint32_t stride = gridDim.x * kDeqThreads * kDeqUnroll;
@@ -293,7 +401,7 @@ __global__ void __launch_bounds__(kDeqThreads)
         const uint32_t col = (c - row * chunks_per_row) * 16;
         off[u] = static_cast<int64_t>(c) * 16;
         raw[u] = __ldcs(reinterpret_cast<const uint4*>(q + off[u]));
-        sc[u] = __ldg(s + (row >> lb) * nbn + (col >> lb));
+        sc[u] = __ldg(s + static_cast<int64_t>(row >> row_shift) * s_row_stride + (col >> lb));
       } else {
         off[u] = -1;
       }
@@ -343,14 +451,15 @@ __global__ void __launch_bounds__(kDeqThreads)
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDeqThreads)
     weight_dequant_any_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
-                              void* __restrict__ y, int64_t M, int64_t N, int64_t nbn, int lb) {
+                              void* __restrict__ y, int64_t M, int64_t N, int64_t s_row_stride,
+                              int row_shift, int lb) {
   pdl_trigger();
   pdl_wait();
   const int64_t total = M * N;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDeqThreads + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * kDeqThreads) {
     const int64_t row = i / N, col = i - row * N;
-    const float v = e4m3_value(q[i]) * __ldg(s + (row >> lb) * nbn + (col >> lb));
+    const float v = e4m3_value(q[i]) * __ldg(s + (row >> row_shift) * s_row_stride + (col >> lb));
     if (OUT_BF16)
       static_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
     else

@@ -30,6 +30,9 @@
  *        b, b_s), scaling fused into the matrix product); "DeepSeek-V3: How
  *        Selective FP8 Stays Stable", "Learning outcomes" (1x128 activation
  *        tiles, 128x128 weight blocks, FP32 promotion of partial sums).
+ *  [STATIC] "Understanding Dynamic and Static Activation Quantization Schemes
+ *        in DeepSeek-V3", "How Static Activation Quantization Differs"
+ *        (precomputed scales; static_dequant multiplies the codes by them).
  */
 #ifndef FP8BS_H
 #define FP8BS_H
@@ -121,6 +124,50 @@ FP8BS_API fp8bs_status fp8bs_act_quant(const void *x, fp8bs_dtype x_dtype, int64
  */
 FP8BS_API fp8bs_status fp8bs_weight_dequant(const uint8_t *q, const float *s, int64_t M, int64_t N,
                                   int64_t block, void *y, fp8bs_dtype y_dtype, void *stream);
+
+/*
+ * act_quant_static: the static activation scheme ([STATIC]): the scales were
+ * fixed ahead of time (by calibration) and ship with the checkpoint, so no
+ * amax is taken; each element is divided by its block's given scale:
+ *   q[r, c] = e4m3fn_rne_satfinite(x[r, c] / s[r * s_row_stride + c / block])
+ * (IEEE fp32 division).  Values beyond 448 * s saturate to +-448, which the
+ * dynamic scheme never needs.
+ *   x            device, [rows, cols], bf16 or fp32; cols % block == 0
+ *   s            device fp32 scales (4-byte aligned): s_row_stride = 0 is one
+ *                scale per block of channels, [cols / block], shared by
+ *                every row (the static scheme); s_row_stride >= cols / block
+ *                is a per-row table with that row pitch (act_quant's s layout
+ *                when equal to cols / block)
+ *   q            device, [rows, cols] uint8, written
+ *   s_out        device, [rows, cols / block] fp32 or NULL: when given, the
+ *                scale of every (row, block) is written there, the per-row
+ *                table fp8_gemm reads as a_s
+ * block is 32, 64, 128 or 256 (else FP8BS_ERR_UNSUPPORTED).  Errors
+ * (FP8BS_ERR_INVALID_ARG, nothing launched): cols not a positive multiple of
+ * block, a stride between 0 and cols / block, an unknown dtype, null or
+ * misaligned pointers, rows * cols / 16 at or above about 2^32.  rows == 0 is
+ * a no-op.  A scale that is zero, negative, infinite or NaN is not an error:
+ * the division and the saturating cast then give what IEEE arithmetic gives
+ * (zero scale: +-448 or NaN for 0 / 0).
+ */
+FP8BS_API fp8bs_status fp8bs_act_quant_static(const void *x, fp8bs_dtype x_dtype, int64_t rows,
+                                              int64_t cols, int64_t block, const float *s,
+                                              int64_t s_row_stride, uint8_t *q, float *s_out,
+                                              void *stream);
+
+/*
+ * act_dequant: static_dequant of [STATIC], the inverse of act_quant_static
+ * (and, with a per-row table, of act_quant):
+ *   y[r, c] = decode(q[r, c]) * s[r * s_row_stride + c / block]
+ * with the product in fp32, stored as bf16 (round to nearest even) or fp32.
+ *   q            device, [rows, cols] uint8 e4m3fn codes; cols % block == 0
+ *   s, s_row_stride, block: as for fp8bs_act_quant_static
+ *   y            device, [rows, cols], bf16 (y_dtype = BF16) or fp32, written
+ * Errors as for fp8bs_act_quant_static.
+ */
+FP8BS_API fp8bs_status fp8bs_act_dequant(const uint8_t *q, const float *s, int64_t s_row_stride,
+                                         int64_t rows, int64_t cols, int64_t block, void *y,
+                                         fp8bs_dtype y_dtype, void *stream);
 
 /*
  * weight_quant: the inverse of weight_dequant, block x block quantization of

@@ -83,7 +83,23 @@ def test_host_side_argument_errors_without_gpu(L):
     assert st == fp8bs.ERR_INVALID_ARG
     st = L.fp8bs_fp8_gemm_f32(dummy, dummy, dummy, dummy, 8, 256, 96, 0, dummy, None, 0, None)
     assert st == fp8bs.ERR_INVALID_ARG and b"K=96" in L.fp8bs_last_error_message()
+    # static activation scheme: scale row stride 0 or >= cols / block
+    st = L.fp8bs_act_quant_static(dummy, 0, 4, 256, 128, dummy, 1, dummy, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG and b"s_row_stride" in L.fp8bs_last_error_message()
+    st = L.fp8bs_act_quant_static(dummy, 0, 4, 200, 128, dummy, 0, dummy, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    st = L.fp8bs_act_quant_static(dummy, 0, 4, 256, 48, dummy, 0, dummy, None, None)
+    assert st == fp8bs.ERR_UNSUPPORTED
+    st = L.fp8bs_act_quant_static(dummy, 0, 4, 256, 128, None, 0, dummy, None, None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    st = L.fp8bs_act_quant_static(dummy, 0, 4, 256, 128, dummy, 0, dummy, _p(4098), None)
+    assert st == fp8bs.ERR_INVALID_ARG
+    assert L.fp8bs_act_dequant(dummy, dummy, 1, 4, 256, 128, dummy, 0, None) == fp8bs.ERR_INVALID_ARG
+    assert L.fp8bs_act_dequant(dummy, dummy, 0, 4, 256, 128, dummy, 7, None) == fp8bs.ERR_INVALID_ARG
+    assert L.fp8bs_act_dequant(dummy, dummy, 0, 4, 256, 512, dummy, 0, None) == fp8bs.ERR_UNSUPPORTED
     # empty problems are successful no-ops
+    assert L.fp8bs_act_quant_static(None, 0, 0, 256, 128, None, 0, None, None, None) == fp8bs.OK
+    assert L.fp8bs_act_dequant(None, None, 2, 0, 256, 128, None, 0, None) == fp8bs.OK
     assert L.fp8bs_act_quant(None, 0, 0, 256, 128, 0, None, None, None) == fp8bs.OK
     assert L.fp8bs_weight_dequant(None, None, 0, 16, 128, None, 0, None) == fp8bs.OK
     assert L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 0, 256, 128, dummy, None, 0, None) == fp8bs.OK
