@@ -49,7 +49,7 @@ def _load():
         lib.oracle_weight_dequant.restype = None
         lib.oracle_weight_dequant.argtypes = [c_p, c_p, c_i64, c_i64, c_i64, c_int, c_p]
         lib.oracle_gemm.restype = None
-        lib.oracle_gemm.argtypes = [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i64, c_p, c_p]
+        lib.oracle_gemm.argtypes = [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i64, c_i64, c_p, c_p]
         lib.oracle_act_quant_static.restype = None
         lib.oracle_act_quant_static.argtypes = [c_p, c_int, c_i64, c_i64, c_i64, c_p, c_i64, c_p]
         lib.oracle_act_dequant.restype = None
@@ -211,10 +211,13 @@ def weight_dequant(q, s, block=128, out="bf16"):
     return y
 
 
-def gemm(qa, sa, qw, sw, block=128, with_bound=True):
+def gemm(qa, sa, qw, sw, block=128, with_bound=True, w_scales="block"):
     """FP64 reference of y = A W^T on block-scaled FP8 operands.
 
-    qa [M,K] uint8, sa [M,K/block] f32, qw [N,K] uint8, sw [cdiv(N,block),K/block] f32.
+    qa [M,K] uint8, sa [M,K/block] f32, qw [N,K] uint8, and sw
+    [cdiv(N,block),K/block] f32 (w_scales="block": 128x128 weight blocks) or
+    [N,K/block] (w_scales="row": one scale per row and K block, as for a
+    second activation-like operand).
     Returns (y [M,N] float64, bound [M,N] float64 or None)."""
     qa = _c(qa, np.uint8)
     qw = _c(qw, np.uint8)
@@ -224,13 +227,39 @@ def gemm(qa, sa, qw, sw, block=128, with_bound=True):
     N = qw.shape[0]
     if qw.shape[1] != K or K % block:
         raise ValueError("bad K")
-    if sa.shape != (M, K // block) or sw.shape != (-(-N // block), K // block):
+    if w_scales not in ("block", "row"):
+        raise ValueError("w_scales must be 'block' or 'row'")
+    sw_rows = block if w_scales == "block" else 1
+    if sa.shape != (M, K // block) or sw.shape != (-(-N // sw_rows), K // block):
         raise ValueError("bad scale shapes")
     y = np.empty((M, N), dtype=np.float64)
     b = np.empty((M, N), dtype=np.float64) if with_bound else None
-    _load().oracle_gemm(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, N, K, block,
+    _load().oracle_gemm(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), M, N, K, block, sw_rows,
                         _ptr(y), _ptr(b) if b is not None else None)
     return y, b
+
+
+def act_quant_transposed(x, block=128, scale_fmt=None):
+    """Quantization in block x 1 column blocks, written transposed: the
+    operand layout of the weight-gradient GEMM, contracted over the rows of x.
+
+    By definition this is act_quant of x^T: x [rows, cols] (bf16 bits or
+    float32, rows % block == 0) -> q [cols, rows] uint8, s [cols, rows/block]."""
+    x = np.ascontiguousarray(x)
+    if x.ndim != 2:
+        raise ValueError("x must be 2-D")
+    return act_quant(np.ascontiguousarray(x.T), block, scale_fmt)
+
+
+def fp8_transpose(q, s, block=128):
+    """The transposed FP8 matrix with its transposed block scales (exact):
+    q [R, C] uint8, s [cdiv(R,block), cdiv(C,block)] -> (q^T, s^T)."""
+    q = _c(q, np.uint8)
+    s = _c(s, np.float32)
+    R, C = q.shape
+    if s.shape != (-(-R // block), -(-C // block)):
+        raise ValueError("scale shape must be (cdiv(R,block), cdiv(C,block))")
+    return np.ascontiguousarray(q.T), np.ascontiguousarray(s.T)
 
 
 def bf16_bits_to_f32(h):

@@ -318,7 +318,12 @@ void oracle_weight_dequant(const uint8_t *q, const float *s, int64_t M, int64_t 
 /*   y[m,n] = sum_kb sa[m,kb] * sw[n/block,kb] * P_kb[m,n],                   */
 /*   P_kb[m,n] = sum_{k in kb} dec(qa[m,k]) * dec(qw[n,k]),                   */
 /* with A = [M,K], W = [N,K] (y = A W^T), sa = [M, K/block],                  */
-/* sw = [cdiv(N,block), K/block].  P_kb is exact in double: each product is a */
+/* sw = [cdiv(N,block), K/block].  sw_rows = block gives that weight layout;  */
+/* sw_rows = 1 gives one scale per row of W and K block, sw = [N, K/block],   */
+/* the second operand of the weight-gradient GEMM [P5 "Lower precision is a   */
+/* constrained budget": all three GEMMs of a linear layer run in FP8], whose  */
+/* operands are both activations-like (quantized along the contracted dim).   */
+/* P_kb is exact in double: each product is a */
 /* multiple of 2^-18 below 2^18 and 128 of them need under 53 bits.  Also    */
 /* returns bound[m,n] = sum_k |dec(qa)*sa * dec(qw)*sw|, the scale of the    */
 /* rounding error that FP32 accumulation may make.                            */
@@ -327,7 +332,8 @@ void oracle_weight_dequant(const uint8_t *q, const float *s, int64_t M, int64_t 
 /* ------------------------------------------------------------------------ */
 
 void oracle_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const float *sw,
-                 int64_t M, int64_t N, int64_t K, int64_t block, double *y, double *bound)
+                 int64_t M, int64_t N, int64_t K, int64_t block, int64_t sw_rows, double *y,
+                 double *bound)
 {
     int64_t kbn = K / block;
     double table[256];
@@ -337,7 +343,7 @@ void oracle_gemm(const uint8_t *qa, const float *sa, const uint8_t *qw, const fl
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t n = 0; n < N; n++) {
         const uint8_t *wrow = qw + n * K;
-        const float *swrow = sw + (n / block) * kbn;
+        const float *swrow = sw + (n / sw_rows) * kbn;
         for (int64_t m = 0; m < M; m++) {
             const uint8_t *arow = qa + m * K;
             double acc = 0.0, babs = 0.0;

@@ -390,10 +390,11 @@ def _random_problem(M, N, K, seed, ue8m0=False):
     return codes_a, sa, codes_w, sw
 
 
-def _exact_gemm(qa, sa, qw, sw):
+def _exact_gemm(qa, sa, qw, sw, w_rows=128):
     """Exact y and bound with integer arithmetic: every e4m3 value times 2^9 is
     an integer, so each 128-wide partial sum is an integer times 2^-18; the
-    scales are then applied as exact rationals."""
+    scales are then applied as exact rationals.  Row n of W takes scale row
+    n // w_rows (128: weight blocks; 1: per-row scales)."""
     table = oracle.e4m3_table()
     ia = np.rint(table[qa] * 512).astype(np.int64)
     iw = np.rint(table[qw] * 512).astype(np.int64)
@@ -408,7 +409,7 @@ def _exact_gemm(qa, sa, qw, sw):
         for m in range(M):
             fa = Fraction(float(sa[m, kb]))
             for n in range(N):
-                sc = fa * Fraction(float(sw[n // 128, kb])) / (1 << 18)
+                sc = fa * Fraction(float(sw[n // w_rows, kb])) / (1 << 18)
                 y[m][n] += sc * int(P[m, n])
                 b[m][n] += abs(sc) * int(Pabs[m, n])
     return y, b
@@ -551,3 +552,92 @@ def test_act_dequant_matches_pages_static_dequant(block):
     ref = (qf * s_tab.unsqueeze(-1)).reshape(rows, -1)
     y32 = oracle.act_dequant(codes.numpy(), s_tab.numpy(), block=block, out="f32")
     assert np.array_equal(y32.view(np.uint32), ref.numpy().view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# training GEMMs: per-row scales on both operands, transposed operands
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(3, 130, 128), (2, 257, 384)])
+def test_gemm_row_scaled_b_matches_exact_integer_arithmetic(M, N, K):
+    """One scale per row of the second operand and K block (w_scales="row")."""
+    qa, sa, qw, _ = _random_problem(M, N, K, seed=M * 7 + N + K)
+    g = torch.Generator().manual_seed(N)
+    sb = (torch.rand(N, K // 128, generator=g) * 0.5 + 1e-3).numpy().astype(np.float32)
+    y, bnd = oracle.gemm(qa, sa, qw, sb, w_scales="row")
+    ye, be = _exact_gemm(qa, sa, qw, sb, w_rows=1)
+    for m in range(M):
+        for n in range(N):
+            tol = float(be[m][n]) * 2.0 ** -50
+            assert abs(Fraction(float(y[m, n])) - ye[m][n]) <= Fraction(tol), (m, n)
+            assert abs(bnd[m, n] - float(be[m][n])) <= tol
+
+
+def test_gemm_row_scales_equal_to_block_scales_agree():
+    """Row scales that repeat each weight block's scale over its 128 rows
+    give the block-scaled result exactly."""
+    qa, sa, qw, sw = _random_problem(5, 300, 256, seed=31)
+    y_blk, _ = oracle.gemm(qa, sa, qw, sw)
+    y_row, _ = oracle.gemm(qa, sa, qw, np.repeat(sw, 128, axis=0)[:300].copy(), w_scales="row")
+    assert np.array_equal(y_blk, y_row)
+
+
+def test_act_quant_transposed_matches_library_ops():
+    """128 x 1 column blocks of x (amax over 128 consecutive rows of one
+    column, by torch on x itself, no transpose), torch's division and cast,
+    then the result laid out transposed."""
+    g = torch.Generator().manual_seed(41)
+    R, C = 3 * BLOCK, 200
+    x = torch.randn(R, C, generator=g) * 3
+    x[torch.rand(x.shape, generator=g) < 0.01] *= 60
+    x[:BLOCK, 7] = 0.0                                  # an all-zero column block
+    arr = _bf16(x)
+    xf = torch.from_numpy(oracle.bf16_bits_to_f32(arr).copy())
+    for fmt in (None, "ue8m0"):
+        q, s = oracle.act_quant_transposed(arr, scale_fmt=fmt)
+        assert q.shape == (C, R) and s.shape == (C, R // BLOCK)
+        amax = xf.abs().reshape(R // BLOCK, BLOCK, C).amax(dim=1)          # [R/128, C]
+        a = torch.clamp(amax, min=float(f32(CLAMP)))
+        sref = (a / torch.tensor(448.0)).numpy().astype(np.float32)
+        if fmt == "ue8m0":
+            m, e = np.frexp(sref.astype(np.float64))
+            sref = np.where(m == 0.5, sref, np.ldexp(1.0, e)).astype(np.float32)
+        assert np.array_equal(s.view(np.uint32), sref.T.view(np.uint32))
+        st = torch.from_numpy(sref).repeat_interleave(BLOCK, dim=0)        # [R, C]
+        ref = (xf / st).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(q, ref.T)
+
+
+def test_weight_gradient_gemm_matches_library_matmul():
+    """dW = dy^T x with both operands quantized in 128 x 1 blocks along the
+    token dimension: the row-scaled GEMM of the transposed operands equals
+    torch's float64 matmul of the dequantized dy and x."""
+    g = torch.Generator().manual_seed(43)
+    T, N, K = 256, 192, 136                       # tokens, out features, in features
+    dy = torch.randn(T, N, generator=g) * 1e-2
+    x = torch.randn(T, K, generator=g)
+    qd, sd = oracle.act_quant_transposed(_bf16(dy))            # [N, T], [N, T/128]
+    qx, sx = oracle.act_quant_transposed(_bf16(x))             # [K, T], [K, T/128]
+    dw, bnd = oracle.gemm(qd, sd, qx, sx, w_scales="row")       # [N, K]
+    t = torch.from_numpy(oracle.e4m3_table())
+    d_hat = t[torch.from_numpy(qd).long()] * torch.from_numpy(sd).double().repeat_interleave(BLOCK, 1)
+    x_hat = t[torch.from_numpy(qx).long()] * torch.from_numpy(sx).double().repeat_interleave(BLOCK, 1)
+    ref = (d_hat @ x_hat.T).numpy()                             # dy_hat^T x_hat, [N, K]
+    assert np.all(np.abs(dw - ref) <= 1e-12 * bnd)
+
+
+def test_fp8_transpose_and_dequant_commute():
+    """dequant(q^T, s^T) is the transpose of dequant(q, s), on ragged shapes,
+    and transposing twice is the identity."""
+    g = torch.Generator().manual_seed(47)
+    R, C = 300, 200
+    codes = torch.randint(0, 254, (R, C), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8).numpy()
+    s = (torch.rand(3, 2, generator=g) + 0.01).numpy().astype(np.float32)
+    qt, st = oracle.fp8_transpose(codes, s)
+    assert qt.shape == (C, R) and st.shape == (2, 3)
+    y = oracle.weight_dequant(codes, s, out="f32")
+    yt = oracle.weight_dequant(qt, st, out="f32")
+    assert np.array_equal(yt, y.T)
+    q2, s2 = oracle.fp8_transpose(qt, st)
+    assert np.array_equal(q2, codes) and np.array_equal(s2, s)
