@@ -26,7 +26,8 @@ import torch
 __all__ = [
     "act_quant", "act_quant_static", "act_dequant", "static_dequant",
     "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
-    "fp8_gemm_grouped", "fp8_gemm_quant", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
+    "fp8_gemm_grouped", "fp8_gemm_quant", "fp8_gemm_rowwise", "act_quant_transposed",
+    "fp8_transpose", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
     "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -71,6 +72,9 @@ def lib():
         "fp8bs_weight_dequant": (i32, [p, p, i64, i64, i64, p, i32, p]),
         "fp8bs_weight_quant": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
         "fp8bs_act_quant_static": (i32, [p, i32, i64, i64, i64, p, i64, p, p, p]),
+        "fp8bs_act_quant_transposed": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
+        "fp8bs_fp8_transpose": (i32, [p, p, i64, i64, i64, p, p, p]),
+        "fp8bs_fp8_gemm_rowwise": (i32, [p, p, p, p, i64, i64, i64, i32, p, i32, p, sz, p]),
         "fp8bs_act_dequant": (i32, [p, p, i64, i64, i64, i64, p, i32, p]),
         "fp8bs_gemm_workspace_size": (sz, [i64, i64, i64]),
         "fp8bs_gemm_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
@@ -253,6 +257,61 @@ def weight_quant(w, block_size=128, scale_fmt=None):
     _check(lib().fp8bs_weight_quant(_ptr(w), dt, M, N, block_size, _scale_fmt(scale_fmt),
                                     _ptr(q), _ptr(s), _stream(w.device)))
     return q, s
+
+
+def act_quant_transposed(x, block_size=128, scale_fmt=None):
+    """Quantization in block_size x 1 column blocks, written transposed:
+    act_quant(x.T) for a 2-D x [rows, cols] (rows % block_size == 0).
+
+    Returns q [cols, rows] float8_e4m3fn and s [cols, rows // block_size]
+    float32, the K-major operand of the weight-gradient GEMM."""
+    _need_cuda(x)
+    if x.dim() != 2:
+        raise ValueError("act_quant_transposed expects a 2-D x")
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[x.dtype]
+    rows, cols = x.shape
+    q = torch.empty(cols, rows, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty(cols, rows // block_size, dtype=torch.float32, device=x.device)
+    _check(lib().fp8bs_act_quant_transposed(_ptr(x), dt, rows, cols, block_size,
+                                            _scale_fmt(scale_fmt), _ptr(q), _ptr(s),
+                                            _stream(x.device)))
+    return q, s
+
+
+def fp8_transpose(q, s, block_size=128):
+    """(q^T, s^T) of an FP8 matrix with block_size x block_size scales, exact."""
+    q = _codes(q)
+    _need_cuda(q, s)
+    R, C = q.shape
+    if tuple(s.shape) != (-(-R // block_size), -(-C // block_size)) or s.dtype != torch.float32:
+        raise ValueError("s must be float32 of shape (cdiv(R, block), cdiv(C, block))")
+    qt = torch.empty(C, R, dtype=torch.float8_e4m3fn, device=q.device)
+    st = torch.empty(s.shape[1], s.shape[0], dtype=torch.float32, device=q.device)
+    _check(lib().fp8bs_fp8_transpose(_ptr(q), _ptr(s.contiguous()), R, C, block_size,
+                                     _ptr(qt), _ptr(st), _stream(q.device)))
+    return qt, st
+
+
+def fp8_gemm_rowwise(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.float32):
+    """y = a @ b^T where both operands carry one scale per row and 128-wide
+    K block (a_s [M, K/128], b_s [N, K/128]): the weight-gradient GEMM
+    dW = dy^T x on act_quant_transposed(dy) and act_quant_transposed(x).
+    out_dtype float32 (the default: weight gradients stay FP32) or bfloat16."""
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    a, b = _codes(a), _codes(b)
+    _need_cuda(a, a_s, b, b_s)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K or tuple(a_s.shape) != (M, K // 128) or tuple(b_s.shape) != (N, K // 128):
+        raise ValueError("a [M,K], a_s [M,K/128], b [N,K], b_s [N,K/128] expected")
+    y = torch.empty(M, N, dtype=out_dtype, device=a.device)
+    ws, nws = _workspace(M, N, K, a.device)
+    dt = DTYPE_F32 if out_dtype == torch.float32 else DTYPE_BF16
+    _check(lib().fp8bs_fp8_gemm_rowwise(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K,
+                                        _scale_fmt(scale_fmt), _ptr(y), dt, _ptr(ws), nws,
+                                        _stream(a.device)))
+    return y
 
 
 def gemm_workspace_size(M, N, K):

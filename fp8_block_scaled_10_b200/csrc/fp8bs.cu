@@ -17,6 +17,7 @@
 #include "gemm_bs.cuh"
 #include "quant.cuh"
 #include "sm100.cuh"
+#include "transpose.cuh"
 
 namespace fp8bs {
 namespace {
@@ -58,10 +59,10 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G, int AR = 128>
+template <int BN, bool G, int AR = 128, bool BROW = false>
 fp8bs_status setup_gemm_kernel() {
   using C = gemm::Cfg<BN, AR>;
-  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR, BROW>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -79,10 +80,10 @@ fp8bs_status setup_gemm_kernel() {
   return FP8BS_OK;
 }
 
-template <int BN, bool G>
+template <int BN, bool G, bool BROW = false>
 fp8bs_status setup_gemm_bs_kernel() {
   const cudaError_t e =
-      cudaFuncSetAttribute(gemm::fp8_gemm_bs_kernel<BN, G>,
+      cudaFuncSetAttribute(gemm::fp8_gemm_bs_kernel<BN, G, BROW>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            gemm::BsCfg<BN>::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -120,7 +121,11 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_bs_kernel<128, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, false>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, true>()) != FP8BS_OK ||
-        (r = setup_gemm_bs_kernel<256, true>()) != FP8BS_OK)
+        (r = setup_gemm_bs_kernel<256, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<128, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_bs_kernel<256, false, true>()) != FP8BS_OK)
       return r;
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -288,7 +293,9 @@ double wave_efficiency(int64_t units, int slots) {
 }
 
 // The two GEMM kernels the planner serves.
-enum class GemmKind { kPromotion, kBlockScaled };
+// kRowScaled: the promotion kernel with one scale per row of W (per column of
+// y) and K block, whose epilogue multiplies each column's scale in.
+enum class GemmKind { kPromotion, kBlockScaled, kRowScaled };
 
 // Time per K block of one 128-row work unit, in microseconds, measured on
 // B200 at M = 4096 with every SM busy.
@@ -298,6 +305,7 @@ enum class GemmKind { kPromotion, kBlockScaled };
 //   block-scaled kernel: 128 x 256 ~0.5, 128 x 128 ~1/3 (operand feed).
 double kb_time_us(GemmKind kind, int bn) {
   if (kind == GemmKind::kPromotion) return bn == 256 ? 0.55 : (bn == 192 ? 0.48 : 0.36);
+  if (kind == GemmKind::kRowScaled) return bn == 256 ? 0.62 : 0.40;
   return bn == 256 ? 0.5 : 1.0 / 3.0;
 }
 
@@ -386,12 +394,12 @@ size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
-template <int BN, bool G, int AR = 128>
+template <int BN, bool G, int AR = 128, bool BROW = false>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                         const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::Cfg<BN, AR>;
-  return launch(gemm::fp8_gemm_kernel<BN, G, AR>, grid, C::kThreads, C::smem_bytes(G), st, ta,
-                tw, ty, p);
+  return launch(gemm::fp8_gemm_kernel<BN, G, AR, BROW>, grid, C::kThreads, C::smem_bytes(G), st,
+                ta, tw, ty, p);
 }
 
 // Rows of A one pipeline stage loads: all 128 rows of a tile, or for
@@ -429,7 +437,8 @@ fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8
 
 fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
                       int64_t M, int64_t N, int64_t K, void* y, void* ws, size_t ws_bytes,
-                      cudaStream_t st, bool out_f32 = false) {
+                      cudaStream_t st, bool out_f32 = false,
+                      bool w_rowwise = false) {
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
@@ -437,7 +446,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const Plan pl = plan_gemm(M, N, K, *info);
+  const Plan pl = plan_gemm(M, N, K, *info, w_rowwise ? GemmKind::kRowScaled : GemmKind::kPromotion);
   const size_t need = plan_workspace(pl, M, N);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
@@ -446,7 +455,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   gemm::Params p{};
   // Decode-sized M loads only the rows it has; 192-wide tiles are planned for
   // M > 128 only.
-  const int a_rows = pl.bn == 192 ? 128 : a_rows_for(M);
+  const int a_rows = (pl.bn == 192 || w_rowwise) ? 128 : a_rows_for(M);
   if ((r = make_tmap(&ta, a, M, K, a_rows)) != FP8BS_OK) return r;
   if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
   if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma, out_f32)) != FP8BS_OK) return r;
@@ -471,7 +480,10 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.tail_kbps = pl.tail_kbps;
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   p.groups = 1;
-  cudaError_t e = launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st);
+  cudaError_t e =
+      !w_rowwise ? launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st)
+      : pl.bn == 256 ? launch_gemm<256, false, 128, true>(ta, tw, ty, p, pl.grid, st)
+                     : launch_gemm<128, false, 128, true>(ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.tail_splits > 0) {
     const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
@@ -499,18 +511,19 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   return FP8BS_OK;
 }
 
-template <int BN, bool G>
+template <int BN, bool G, bool BROW = false>
 cudaError_t launch_gemm_bs(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                            const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::BsCfg<BN>;
-  return launch(gemm::fp8_gemm_bs_kernel<BN, G>, grid, C::kThreads, C::smem_bytes(G), st, ta,
-                tw, ty, p);
+  return launch(gemm::fp8_gemm_bs_kernel<BN, G, BROW>, grid, C::kThreads, C::smem_bytes(G), st,
+                ta, tw, ty, p);
 }
 
 // Block-scaled (ue8m0) GEMM: the same plan as the promotion kernel.
 fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
                          int64_t M, int64_t N, int64_t K, void* y, void* ws, size_t ws_bytes,
-                         cudaStream_t st, bool out_f32 = false) {
+                         cudaStream_t st, bool out_f32 = false,
+                         bool w_rowwise = false) {
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
@@ -548,8 +561,11 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   p.tail_kbps = pl.tail_kbps;
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   p.groups = 1;
-  cudaError_t e = pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, ty, p, pl.grid, st)
-                               : launch_gemm_bs<128, false>(ta, tw, ty, p, pl.grid, st);
+  cudaError_t e = w_rowwise
+                      ? (pl.bn == 256 ? launch_gemm_bs<256, false, true>(ta, tw, ty, p, pl.grid, st)
+                                      : launch_gemm_bs<128, false, true>(ta, tw, ty, p, pl.grid, st))
+                      : (pl.bn == 256 ? launch_gemm_bs<256, false>(ta, tw, ty, p, pl.grid, st)
+                                      : launch_gemm_bs<128, false>(ta, tw, ty, p, pl.grid, st));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_ue8m0 launch");
   if (pl.tail_splits > 0) {
     const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);
@@ -733,6 +749,81 @@ fp8bs_status fp8bs_act_dequant(const uint8_t* q, const float* s, int64_t s_row_s
   return FP8BS_OK;
 }
 
+fp8bs_status fp8bs_fp8_transpose(const uint8_t* q, const float* s, int64_t R, int64_t C,
+                                 int64_t block, uint8_t* qt, float* st, void* stream) {
+  if (block_log2(block) < 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (32, 64, 128 and 256 are implemented)", (long long)block);
+  if (R < 0 || C < 0) return fail(FP8BS_ERR_INVALID_ARG, "negative size");
+  if (R == 0 || C == 0) return FP8BS_OK;
+  if (!q || !s || !qt || !st) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(qt) || (reinterpret_cast<uintptr_t>(s) & 3u) ||
+      (reinterpret_cast<uintptr_t>(st) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "q and qt must be 16-byte aligned, s and st 4-byte aligned");
+  if (q == qt) return fail(FP8BS_ERR_INVALID_ARG, "the transpose is not in place");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const int64_t sr = (R + block - 1) / block, sc = (C + block - 1) / block;
+  cudaStream_t stm = as_stream(stream);
+  cudaError_t e;
+  if (R % 16 == 0 && C % 16 == 0) {
+    const int64_t tiles = ((R + 127) / 128) * ((C + 127) / 128);
+    e = launch(fp8_transpose_kernel, grid_for(tiles, 1, info->sms * 6), kTrThreads, 0, stm, q, s,
+               qt, st, R, C, sr, sc);
+  } else {
+    e = launch(fp8_transpose_any_kernel, grid_for(R * C, 256, info->sms * 8), 256, 0, stm, q, s,
+               qt, st, R, C, sr, sc);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_transpose launch");
+  return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_act_quant_transposed(const void* x, fp8bs_dtype x_dtype, int64_t rows,
+                                        int64_t cols, int64_t block, fp8bs_scale_fmt fmt,
+                                        uint8_t* qt, float* st, void* stream) {
+  if (block != 128)
+    return fail(FP8BS_ERR_UNSUPPORTED, "block=%lld (the transposed quantizer implements 128)",
+                (long long)block);
+  if (rows < 0 || rows % 128 != 0)
+    return fail(FP8BS_ERR_INVALID_ARG, "rows=%lld must be a multiple of 128", (long long)rows);
+  if (cols <= 0) return fail(FP8BS_ERR_INVALID_ARG, "cols=%lld", (long long)cols);
+  if (cols % 8 != 0)
+    return fail(FP8BS_ERR_UNSUPPORTED, "cols=%lld (multiples of 8 are implemented)", (long long)cols);
+  if (x_dtype != FP8BS_DTYPE_BF16 && x_dtype != FP8BS_DTYPE_F32)
+    return fail(FP8BS_ERR_INVALID_ARG, "x_dtype");
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
+  if (rows == 0) return FP8BS_OK;
+  if (!x || !qt || !st) return fail(FP8BS_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(qt) || (reinterpret_cast<uintptr_t>(st) & 3u))
+    return fail(FP8BS_ERR_INVALID_ARG, "x and qt must be 16-byte aligned, st 4-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  fp8bs_status r = device_setup(&dev, &info);
+  if (r != FP8BS_OK) return r;
+  const int64_t tiles = (rows / 128) * ((cols + 127) / 128);
+  const int grid = grid_for(tiles, 1, info->sms * 4);
+  cudaStream_t stm = as_stream(stream);
+  const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
+  cudaError_t e;
+  if (x_dtype == FP8BS_DTYPE_BF16) {
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    e = ue ? launch(act_quant_transposed_kernel<__nv_bfloat16, true>, grid, kAqtThreads, 0, stm, xb,
+                    qt, st, rows, cols)
+           : launch(act_quant_transposed_kernel<__nv_bfloat16, false>, grid, kAqtThreads, 0, stm,
+                    xb, qt, st, rows, cols);
+  } else {
+    const auto* xf = static_cast<const float*>(x);
+    e = ue ? launch(act_quant_transposed_kernel<float, true>, grid, kAqtThreads, 0, stm, xf, qt,
+                    st, rows, cols)
+           : launch(act_quant_transposed_kernel<float, false>, grid, kAqtThreads, 0, stm, xf, qt,
+                    st, rows, cols);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_transposed launch");
+  return FP8BS_OK;
+}
+
 fp8bs_status fp8bs_act_quant_static(const void* x, fp8bs_dtype x_dtype, int64_t rows,
                                     int64_t cols, int64_t block, const float* s,
                                     int64_t s_row_stride, uint8_t* q, float* s_out,
@@ -863,8 +954,9 @@ size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   DeviceInfo* info;
   if (device_setup(&dev, &info) != FP8BS_OK) return 0;
   // One size serves both GEMM entry points (their plans may differ).
-  return std::max(plan_workspace(plan_gemm(M, N, K, *info), M, N),
-                  plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N));
+  return std::max({plan_workspace(plan_gemm(M, N, K, *info), M, N),
+                   plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N),
+                   plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kRowScaled), M, N)});
 }
 
 const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
@@ -959,6 +1051,22 @@ fp8bs_status fp8bs_fp8_gemm_f32(const uint8_t* a, const float* a_s, const uint8_
     return run_gemm_bs(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream),
                        true);
   return run_gemm(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream), true);
+}
+
+fp8bs_status fp8bs_fp8_gemm_rowwise(const uint8_t* a, const float* a_s, const uint8_t* b,
+                                    const float* b_s, int64_t M, int64_t N, int64_t K,
+                                    fp8bs_scale_fmt fmt, void* y, fp8bs_dtype y_dtype,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fp8bs::fail(FP8BS_ERR_INVALID_ARG, "scale format %d", (int)fmt);
+  if (y_dtype != FP8BS_DTYPE_BF16 && y_dtype != FP8BS_DTYPE_F32)
+    return fp8bs::fail(FP8BS_ERR_INVALID_ARG, "y_dtype");
+  const bool f32 = y_dtype == FP8BS_DTYPE_F32;
+  if (fmt == FP8BS_SCALE_FMT_UE8M0)
+    return run_gemm_bs(a, a_s, b, b_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream),
+                       f32, true);
+  return run_gemm(a, a_s, b, b_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream), f32,
+                  true);
 }
 
 fp8bs_status fp8bs_fp8_linear_ue8m0(const uint16_t* x, int64_t M, int64_t K, const uint8_t* w,

@@ -182,9 +182,9 @@ struct Cfg {
   static constexpr int kTmemCols = 512;
   static constexpr int kCtrlBytes = 512;
   // Scale ring: per K block the tile's 128 activation scales and its
-  // (BN / 128) weight scales.
+  // (BN / 128) weight scales, or with row scales on W its BN column scales.
   static constexpr int kScaleSlots = 4;   // >= kAccBufs; slot b goes with TMEM buffer b
-  static constexpr int kScaleSlotBytes = 4 * (BM + 4);
+  static constexpr int kScaleSlotBytes = 4 * (BM + BN);
   static constexpr int kScaleBytes = kScaleSlots * kScaleSlotBytes;
   // grouped mode: per-group m-tile prefix (int)
   static constexpr int kGroupBytes = 4 * kGroupTableInts;
@@ -205,6 +205,7 @@ struct Ctrl {
   uint64_t empty[kStages];
   uint64_t tfull[4];     // TMEM partial buffer and its scale slot ready for the epilogue
   uint64_t tempty[4];    // TMEM partial buffer drained and its scale slot read
+  uint64_t sempty[4];    // row scales on W: the epilogue is done with scale slot b
   uint64_t flush[2];     // per MMA issuer: all of its MMAs complete
   uint32_t tmem_base;
   int abort_flag;
@@ -318,7 +319,13 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   return t;
 }
 
-template <int BN, bool GROUPED, int ARows = 128>
+// BROW: one scale per row of W (W column of y) and K block, w_s [N, K/128],
+// as both operands of the weight-gradient GEMM carry (dense mode only).  The
+// scale producer then fills the slot with the tile's BN column scales, the
+// epilogue multiplies a_s[row] by each column's scale before its FMA, and
+// since those reads outlast the TMEM buffer's release, the slot has its own
+// release barrier (sempty) that the producer waits on instead of tempty.
+template <int BN, bool GROUPED, int ARows = 128, bool BROW = false>
 __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w,
@@ -335,7 +342,9 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
   uint64_t* empty = ctrl->empty;
   uint64_t* tfull = ctrl->tfull;
   uint64_t* tempty = ctrl->tempty;
+  uint64_t* sempty = ctrl->sempty;
   uint64_t* flush = ctrl->flush;
+  static_assert(!(BROW && GROUPED), "row scales on W are a dense-mode variant");
   volatile int* abort_flag = &ctrl->abort_flag;
   float* scale_slots =
       reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kCtrlBytes);
@@ -360,6 +369,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&tfull[b], 2);
       mbar_init(&tempty[b], C::kEpiWarps);
+      mbar_init(&sempty[b], C::kEpiWarps);
     }
     mbar_init(&flush[0], 1);
     mbar_init(&flush[1], 1);
@@ -487,11 +497,17 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     // memory writes of step i.  Step i uses the slot of its TMEM buffer,
     // i % kAccBufs, once the epilogue has released that buffer (tempty), and
     // then arrives on its tfull: a_s of the tile's 128 rows (0 past the last
-    // row) and w_s of the weight blocks the tile touches (0 past the last).
-    constexpr int kAhead = 4;
+    // row) and w_s of the weight blocks the tile touches (0 past the last),
+    // or with BROW the scales of the tile's BN columns (0 past the last), in
+    // which case the slot is reused once the epilogue has read it (sempty).
+    // With BROW the ring holds BN / 32 more values per step; two steps ahead
+    // (over a microsecond of MMA work) keep it within the producer's registers.
+    constexpr int kAhead = BROW ? 2 : 4;
     constexpr int kNbPerTile = C::kNbSpan;
+    constexpr int kWRegs = BROW ? BN / 32 : 1;
+    uint64_t* slot_free = BROW ? sempty : tempty;
     struct Cursor {
-      int u, kb, kb1, group, nb0;
+      int u, kb, kb1, group, nb0, n0;
       int64_t row0, row_end;
       bool valid;
     };
@@ -504,6 +520,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         c.kb1 = t.kb1;
         c.group = t.group;
         c.nb0 = (t.n_tile * BN) / 128;
+        c.n0 = t.n_tile * BN;
         c.row0 = t.row0;
         c.row_end = t.row_end;
       }
@@ -511,18 +528,26 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     auto next = [&](Cursor& c) {
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
-    auto load = [&](const Cursor& c, float (&va)[4], float& vw) {
+    auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWRegs]) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
         va[j] = (c.valid && row < c.row_end) ? __ldg(p.sa + row * p.kbn + c.kb) : 0.0f;
       }
-      const int nb = c.nb0 + lane;
-      vw = (c.valid && lane < kNbPerTile && nb < p.nbn)
-               ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
-               : 0.0f;
+      if (BROW) {
+#pragma unroll
+        for (int j = 0; j < kWRegs; ++j) {
+          const int64_t col = c.n0 + lane + 32 * j;
+          vw[j] = (c.valid && col < p.N) ? __ldg(p.sw + col * p.kbn + c.kb) : 0.0f;
+        }
+      } else {
+        const int nb = c.nb0 + lane;
+        vw[0] = (c.valid && lane < kNbPerTile && nb < p.nbn)
+                    ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
+                    : 0.0f;
+      }
     };
-    float ra[kAhead][4], rw[kAhead];
+    float ra[kAhead][4], rw[kAhead][kWRegs];
     Cursor ahead, cur;
     begin(ahead, unit_start);
     begin(cur, unit_start);
@@ -537,12 +562,17 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
 #pragma unroll
       for (int ph = 0; ph < kAhead; ++ph) {
         if (!cur.valid) break;
-        const bool ok = mbar_wait(&tempty[slot], sphase ^ 1u, abort_flag);
+        const bool ok = mbar_wait(&slot_free[slot], sphase ^ 1u, abort_flag);
         if (!__all_sync(0xFFFFFFFFu, ok)) goto scales_done;
         float* dst = scale_slots + slot * (C::kScaleSlotBytes / 4);
 #pragma unroll
         for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = ra[ph][j];
-        if (lane < kNbPerTile) dst[BM + lane] = rw[ph];
+        if (BROW) {
+#pragma unroll
+          for (int j = 0; j < kWRegs; ++j) dst[BM + lane + 32 * j] = rw[ph][j];
+        } else if (lane < kNbPerTile) {
+          dst[BM + lane] = rw[ph][0];
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&tfull[slot]);
         load(ahead, ra[ph], rw[ph]);
@@ -594,6 +624,9 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         float scale_nb[C::kNbSpan];
 #pragma unroll
         for (int i = 0; i < C::kNbSpan; ++i) scale_nb[i] = sa_row * src[BM + i];
+        // BROW: this warp's column scales (the slot stays valid until sempty).
+        const float* sb_col = src + BM + g * CPW;
+        const float2 sa2 = make_float2(sa_row, sa_row);
         const uint32_t col_addr = lane_addr + static_cast<uint32_t>(tb * BN + g * CPW);
         if (C::kOneBatch) {
           // All of this warp's columns in one batch, then hand the buffer back
@@ -614,7 +647,9 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
             for (int j = 0; j < 16; ++j)
               acc[c * 16 + j] = __ffma2_rn(
                   make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1])),
-                  scale2, acc[c * 16 + j]);
+                  BROW ? __fmul2_rn(sa2, *reinterpret_cast<const float2*>(sb_col + 32 * c + 2 * j))
+                       : scale2,
+                  acc[c * 16 + j]);
           }
         } else {
           // Two register buffers: the load of chunk c+1 is in flight while the
@@ -639,9 +674,16 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
             for (int j = 0; j < 16; ++j)
               acc[c * 16 + j] = __ffma2_rn(
                   make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])),
-                  scale2, acc[c * 16 + j]);
+                  BROW ? __fmul2_rn(sa2, *reinterpret_cast<const float2*>(sb_col + 32 * c + 2 * j))
+                       : scale2,
+                  acc[c * 16 + j]);
             if (c + 1 < NCH) tmem_ld_wait(nxt);
           }
+        }
+        if (BROW) {
+          // Done with this K block's column scales: the producer may refill the slot.
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sempty[tb]);
         }
         if (++tb == C::kAccBufs) {
           tb = 0;

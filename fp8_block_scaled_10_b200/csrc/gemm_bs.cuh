@@ -85,12 +85,16 @@ __device__ __forceinline__ uint32_t ue8m0_byte(float v, bool* bad) {
   return e;
 }
 
-template <int BN, bool GROUPED>
+// BROW: one scale per row of W and K block (w_s [N, K/128], dense mode), the
+// second operand of the weight-gradient GEMM; the W atoms then hold a scale
+// per row, laid out like A's, instead of one block scale repeated.
+template <int BN, bool GROUPED, bool BROW = false>
 __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     fp8_gemm_bs_kernel(const __grid_constant__ CUtensorMap tmap_a,
                        const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_y, const Params p) {
   using C = BsCfg<BN>;
+  static_assert(!(BROW && GROUPED), "row scales on W are a dense-mode variant");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -198,8 +202,11 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     // Walks the same (unit, K block) sequence as the TMA producer; a second
     // cursor runs four steps ahead and loads the scales into a ring of
     // registers, so the loads of step i+4 overlap the atoms of step i.
+    // W values per lane and step: one block scale per 128-row atom, or with
+    // BROW the lane's four rows of each atom.
+    constexpr int kWVals = BROW ? BN / 32 : BN / 128;
     struct Cursor {
-      int u, kb, kb1, group, nb0;
+      int u, kb, kb1, group, nb0, n0;
       int64_t row0, row_end;
       bool valid;
     };
@@ -212,6 +219,7 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
         c.kb1 = t.kb1;
         c.group = t.group;
         c.nb0 = (t.n_tile * BN) / 128;
+        c.n0 = t.n_tile * BN;
         c.row0 = t.row0;
         c.row_end = t.row_end;
       }
@@ -219,21 +227,30 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     auto next = [&](Cursor& c) {
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
-    auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[BN / 128]) {
+    auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWVals]) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
         va[j] = (c.valid && row < c.row_end) ? __ldg(p.sa + row * p.kbn + c.kb) : 1.0f;
       }
+      if (BROW) {
+        // value 4a + j: row 128a + lane + 32j of the tile's W rows
 #pragma unroll
-      for (int a = 0; a < BN / 128; ++a) {
-        const int nb = c.nb0 + a;
-        vw[a] = (c.valid && nb < p.nbn)
-                    ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
-                    : 1.0f;
+        for (int i = 0; i < kWVals; ++i) {
+          const int64_t n = c.n0 + 128 * (i / 4) + lane + 32 * (i % 4);
+          vw[i] = (c.valid && n < p.N) ? __ldg(p.sw + n * p.kbn + c.kb) : 1.0f;
+        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < BN / 128; ++a) {
+          const int nb = c.nb0 + a;
+          vw[a] = (c.valid && nb < p.nbn)
+                      ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
+                      : 1.0f;
+        }
       }
     };
-    float ra[4][4], rw[4][BN / 128];
+    float ra[4][4], rw[4][kWVals];
     Cursor ahead, cur;
     begin(ahead, unit_start);
     begin(cur, unit_start);
@@ -260,8 +277,17 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
         *reinterpret_cast<uint4*>(atoms + 16 * lane) = v;
 #pragma unroll
         for (int a = 0; a < BN / 128; ++a) {
-          const uint32_t e = ue8m0_byte(rw[ph][a], &bad) * 0x01010101u;
-          *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = make_uint4(e, e, e, e);
+          if (BROW) {
+            uint4 w;
+            w.x = ue8m0_byte(rw[ph][4 * a + 0], &bad) * 0x01010101u;
+            w.y = ue8m0_byte(rw[ph][4 * a + 1], &bad) * 0x01010101u;
+            w.z = ue8m0_byte(rw[ph][4 * a + 2], &bad) * 0x01010101u;
+            w.w = ue8m0_byte(rw[ph][4 * a + 3], &bad) * 0x01010101u;
+            *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = w;
+          } else {
+            const uint32_t e = ue8m0_byte(rw[ph][a], &bad) * 0x01010101u;
+            *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = make_uint4(e, e, e, e);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();

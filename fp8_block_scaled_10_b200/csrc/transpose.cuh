@@ -1,0 +1,195 @@
+// Operand transposes for the training GEMMs of an FP8 linear layer
+// ("DeepSeek-V3: How Selective FP8 Stays Stable", "Lower precision is a
+// constrained budget": the forward, activation-gradient and weight-gradient
+// GEMMs all run in FP8).  The tensor core reads both operands K-major, so:
+//
+//  * the activation-gradient GEMM dx = dy W contracts over W's rows: it runs
+//    as fp8_gemm(dy, W^T), and fp8_transpose_kernel makes W^T from W (codes
+//    and 128x128 block scales alike, exactly);
+//  * the weight-gradient GEMM dW = dy^T x contracts over the tokens: both
+//    operands are quantized in 128 x 1 blocks along the tokens and stored
+//    transposed, which act_quant_transposed_kernel does in one pass.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "quant.cuh"
+
+namespace fp8bs {
+
+// ---------------------------------------------------------------------------
+// FP8 transpose: qT[c, r] = q[r, c] on 128 x 128 byte tiles (rows and columns
+// multiples of 16), and sT = s^T for the block scales.
+//
+// A tile goes global -> shared memory A (16-byte loads, row pitch 36 words so
+// that the 4-byte column reads below are conflict-free) -> 4 x 4 byte blocks
+// transposed in registers (byte permutes) -> shared memory T (row pitch 32
+// words, word w of row j stored at w ^ key(j) with key(j) = ((j >> 2) ^ j) &
+// 31, which keeps both the transposing writes and the row reads of the store
+// phase free of bank conflicts) -> global (16-byte stores).  Each thread owns
+// four 16-byte chunks per phase.
+// ---------------------------------------------------------------------------
+constexpr int kTrThreads = 256;
+constexpr int kTrApitch = 36;   // words per row of A
+constexpr int kTrSmemBytes = 128 * kTrApitch * 4 + 128 * 32 * 4;
+
+__device__ __forceinline__ uint32_t tr_key(uint32_t j) { return ((j >> 2) ^ j) & 31u; }
+
+__global__ void __launch_bounds__(kTrThreads)
+    fp8_transpose_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
+                         uint8_t* __restrict__ qt, float* __restrict__ st, int64_t R, int64_t C,
+                         int64_t sr, int64_t sc) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __align__(16) uint32_t smA[128 * kTrApitch];
+  __shared__ __align__(16) uint32_t smT[128 * 32];
+  const int t = threadIdx.x;
+  // block scales: sT[j][i] = s[i][j]
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kTrThreads + t; i < sr * sc;
+       i += static_cast<int64_t>(gridDim.x) * kTrThreads) {
+    const int64_t a = i / sc, b = i - a * sc;
+    st[b * sr + a] = s[i];
+  }
+  const int64_t tiles_r = (R + 127) / 128, tiles_c = (C + 127) / 128;
+  for (int64_t tile = blockIdx.x; tile < tiles_r * tiles_c; tile += gridDim.x) {
+    const int64_t row0 = (tile / tiles_c) * 128, col0 = (tile % tiles_c) * 128;
+    // 1. 128 rows x 8 chunks of 16 bytes
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = u * 32 + (t >> 3), sg = t & 7;
+      const int64_t gr = row0 + r, gc = col0 + 16 * sg;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (gr < R && gc < C) v = __ldcs(reinterpret_cast<const uint4*>(q + gr * C + gc));
+      *reinterpret_cast<uint4*>(&smA[r * kTrApitch + 4 * sg]) = v;
+    }
+    __syncthreads();
+    // 2. 32 x 32 blocks of 4 x 4 bytes: block (br, bc) holds rows 4br.. and
+    //    columns 4bc..; its transpose is rows 4bc.. of T at word br.
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = t + kTrThreads * u;
+      const int br = b >> 5, bc = b & 31;
+      const uint32_t w0 = smA[(4 * br + 0) * kTrApitch + bc];
+      const uint32_t w1 = smA[(4 * br + 1) * kTrApitch + bc];
+      const uint32_t w2 = smA[(4 * br + 2) * kTrApitch + bc];
+      const uint32_t w3 = smA[(4 * br + 3) * kTrApitch + bc];
+      const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), hi01 = __byte_perm(w0, w1, 0x7362);
+      const uint32_t lo23 = __byte_perm(w2, w3, 0x5140), hi23 = __byte_perm(w2, w3, 0x7362);
+      const uint32_t o[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                             __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t j = 4 * bc + c;
+        smT[j * 32 + (static_cast<uint32_t>(br) ^ tr_key(j))] = o[c];
+      }
+    }
+    __syncthreads();
+    // 3. output rows = input columns, 16-byte chunks of input rows
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = u * 32 + (t >> 3), sg = t & 7;
+      const int64_t orow = col0 + j, ocol = row0 + 16 * sg;
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = smT[j * 32 + ((4 * sg + i) ^ tr_key(j))];
+      if (orow < C && ocol < R)
+        __stcs(reinterpret_cast<uint4*>(qt + orow * R + ocol), make_uint4(w[0], w[1], w[2], w[3]));
+    }
+    __syncthreads();
+  }
+}
+
+// Any shape: one byte per thread-step.
+__global__ void __launch_bounds__(256)
+    fp8_transpose_any_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s,
+                             uint8_t* __restrict__ qt, float* __restrict__ st, int64_t R,
+                             int64_t C, int64_t sr, int64_t sc) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < sr * sc; i += stride) {
+    const int64_t a = i / sc, b = i - a * sc;
+    st[b * sr + a] = s[i];
+  }
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < R * C; i += stride) {
+    const int64_t j = i / R, r = i - j * R;   // output element (j, r) = input (r, j)
+    qt[i] = q[r * C + j];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// act_quant in 128 x 1 column blocks, written transposed: for x [R, C]
+// (R % 128 == 0, C % 8 == 0), qT [C, R] and sT [C, R / 128] are act_quant of
+// x^T.  One 128 x 128 tile per step: thread t owns the 8 x 8 block of rows
+// 8 (t / 16).. and columns 8 (t % 16)..; per column, the amax of its 8 rows
+// goes to shared memory, 128 threads take each column's maximum over the 16
+// row groups and its scale (block_scale, the act_quant rule), and every
+// thread then quantizes its block column by column (the quotient as in
+// act_quant) and stores 8 codes of one output row.
+// ---------------------------------------------------------------------------
+constexpr int kAqtThreads = 256;
+
+template <typename T, bool UE8M0>
+__global__ void __launch_bounds__(kAqtThreads)
+    act_quant_transposed_kernel(const T* __restrict__ x, uint8_t* __restrict__ qt,
+                                float* __restrict__ st, int64_t R, int64_t C) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __align__(16) float red[16][128];
+  __shared__ __align__(16) float scol[128];
+  const int t = threadIdx.x;
+  const int cg = t & 15, rg = t >> 4;
+  const int64_t nrb = R / 128, tiles_c = (C + 127) / 128;
+  for (int64_t tile = blockIdx.x; tile < nrb * tiles_c; tile += gridDim.x) {
+    const int64_t tr = tile / tiles_c;
+    const int64_t row0 = tr * 128, col0 = (tile % tiles_c) * 128;
+    const int64_t gc = col0 + 8 * cg;
+    const bool col_ok = gc < C;
+    float v[8][8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (col_ok) {
+        load8(x + (row0 + 8 * rg + k) * C + gc, v[k]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[k][c] = 0.0f;
+      }
+    }
+    float pm[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      pm[c] = fabsf(v[0][c]);
+#pragma unroll
+      for (int k = 1; k < 8; ++k) pm[c] = fmaxf(pm[c], fabsf(v[k][c]));
+    }
+    *reinterpret_cast<float4*>(&red[rg][8 * cg]) = make_float4(pm[0], pm[1], pm[2], pm[3]);
+    *reinterpret_cast<float4*>(&red[rg][8 * cg + 4]) = make_float4(pm[4], pm[5], pm[6], pm[7]);
+    __syncthreads();
+    if (t < 128) {
+      float amax = red[0][t];
+#pragma unroll
+      for (int i = 1; i < 16; ++i) amax = fmaxf(amax, red[i][t]);
+      const float sc = block_scale(amax, UE8M0);
+      scol[t] = sc;
+      if (col0 + t < C) st[(col0 + t) * nrb + tr] = sc;
+    }
+    __syncthreads();
+    if (col_ok) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float sc = scol[8 * cg + c];
+        const float r = __frcp_rn(sc);
+        float col[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) col[k] = v[k][c];
+        const uint2 codes = quantize8<UE8M0>(col, sc, r);
+        __stcs(reinterpret_cast<uint2*>(qt + (gc + c) * R + row0 + 8 * rg), codes);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace fp8bs

@@ -30,6 +30,10 @@
  *        b, b_s), scaling fused into the matrix product); "DeepSeek-V3: How
  *        Selective FP8 Stays Stable", "Learning outcomes" (1x128 activation
  *        tiles, 128x128 weight blocks, FP32 promotion of partial sums).
+ *  [TRAIN] "DeepSeek-V3: How Selective FP8 Stays Stable", "Lower precision is
+ *        a constrained budget" (forward, activation-gradient and
+ *        weight-gradient GEMMs in FP8, outputs BF16 or FP32, weight gradients
+ *        FP32).
  *  [STATIC] "Understanding Dynamic and Static Activation Quantization Schemes
  *        in DeepSeek-V3", "How Static Activation Quantization Differs"
  *        (precomputed scales; static_dequant multiplies the codes by them).
@@ -308,6 +312,66 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_f32(const uint8_t *a, const float *a_s, co
                                           const float *w_s, int64_t M, int64_t N, int64_t K,
                                           fp8bs_scale_fmt fmt, float *y, void *workspace,
                                           size_t workspace_bytes, void *stream);
+
+/*
+ * act_quant_transposed: quantization in block x 1 column blocks, written
+ * transposed ([TRAIN]): the K-major operand layout of the weight-gradient
+ * GEMM, which contracts over the rows of x (the tokens).  By definition
+ *   (qt, st) = act_quant(x^T, block, fmt)
+ * i.e. for column c and row block rb the amax of x[rb*block .. +block, c],
+ * the act_quant scale rule, and qt[c, r] = e4m3fn_rne_satfinite(x[r, c] / s).
+ *   x      device, [rows, cols], bf16 or fp32; rows % block == 0 (else
+ *          FP8BS_ERR_INVALID_ARG), cols % 8 == 0 (else FP8BS_ERR_UNSUPPORTED)
+ *   qt     device, [cols, rows] uint8, written
+ *   st     device, [cols, rows / block] fp32, written
+ * block is 128 (others: FP8BS_ERR_UNSUPPORTED).  rows == 0 is a no-op.
+ */
+FP8BS_API fp8bs_status fp8bs_act_quant_transposed(const void *x, fp8bs_dtype x_dtype,
+                                                  int64_t rows, int64_t cols, int64_t block,
+                                                  fp8bs_scale_fmt fmt, uint8_t *qt, float *st,
+                                                  void *stream);
+
+/*
+ * fp8_transpose: the transposed FP8 matrix and its transposed block scales,
+ * exactly ([TRAIN]: the activation-gradient GEMM dx = dy W contracts over W's
+ * rows, so it runs as fp8_gemm(dy, W^T)):
+ *   qt[c, r] = q[r, c],  st[j, i] = s[i, j]
+ *   q      device, [R, C] uint8;  s  device, [cdiv(R,block), cdiv(C,block)] fp32
+ *   qt     device, [C, R] uint8, written (not aliasing q)
+ *   st     device, [cdiv(C,block), cdiv(R,block)] fp32, written
+ * block (32, 64, 128 or 256) only sizes the scale tables.  Any R and C; the
+ * tiled path needs R and C multiples of 16, other shapes take a slower
+ * element-wise kernel.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_transpose(const uint8_t *q, const float *s, int64_t R,
+                                           int64_t C, int64_t block, uint8_t *qt, float *st,
+                                           void *stream);
+
+/*
+ * fp8_gemm_rowwise: the GEMM whose two operands both carry one scale per row
+ * and 128-wide K block, the form of the weight-gradient GEMM of a linear
+ * layer ([TRAIN]: all three GEMMs of a linear layer run in FP8, and weight
+ * gradients stay FP32):
+ *   y[m, n] = sum_kb a_s[m, kb] * b_s[n, kb] * sum_{k in kb} a[m, k] * b[n, k]
+ * For dW = dy^T x over T tokens: a = dy^T and b = x^T, both quantized in
+ * 128 x 1 blocks along the tokens, as fp8bs_act_quant_transposed writes them
+ * (a: [N_out, T], b: [K_in, T], K = T).
+ *   a      device, [M, K] e4m3fn codes;  a_s  device, [M, K / 128] fp32
+ *   b      device, [N, K] e4m3fn codes;  b_s  device, [N, K / 128] fp32
+ *   fmt    FP8BS_SCALE_FMT_NONE (any positive fp32 scales: per-K-block FP32
+ *          promotion with a scale per column) or FP8BS_SCALE_FMT_UE8M0 (all
+ *          scales positive normal powers of two: the block-scaled MMA, with
+ *          the FP8BS_ERR_SCALE report of fp8bs_fp8_gemm_ue8m0)
+ *   y      device, [M, N], fp32 (y_dtype = F32) or bf16, written
+ *   workspace: fp8bs_gemm_workspace_size(M, N, K) bytes suffice
+ * K % 128 == 0, ragged M and N; errors as for fp8bs_fp8_gemm, plus
+ * FP8BS_ERR_INVALID_ARG for an unknown fmt or y_dtype.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_gemm_rowwise(const uint8_t *a, const float *a_s,
+                                              const uint8_t *b, const float *b_s, int64_t M,
+                                              int64_t N, int64_t K, fp8bs_scale_fmt fmt, void *y,
+                                              fp8bs_dtype y_dtype, void *workspace,
+                                              size_t workspace_bytes, void *stream);
 
 /*
  * fp8_linear_ue8m0: act_quant(x, 128, UE8M0) followed by fp8_gemm_ue8m0 on
