@@ -75,6 +75,7 @@ def lib():
         "fp8bs_act_quant_transposed": (i32, [p, i32, i64, i64, i64, i32, p, p, p]),
         "fp8bs_fp8_transpose": (i32, [p, p, i64, i64, i64, p, p, p]),
         "fp8bs_fp8_gemm_rowwise": (i32, [p, p, p, p, i64, i64, i64, i32, p, i32, p, sz, p]),
+        "fp8bs_gemm_rowwise_workspace_size": (sz, [i64, i64, i64]),
         "fp8bs_act_dequant": (i32, [p, p, i64, i64, i64, i64, p, i32, p]),
         "fp8bs_gemm_workspace_size": (sz, [i64, i64, i64]),
         "fp8bs_gemm_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
@@ -306,7 +307,8 @@ def fp8_gemm_rowwise(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.float32):
     if b.shape[1] != K or tuple(a_s.shape) != (M, K // 128) or tuple(b_s.shape) != (N, K // 128):
         raise ValueError("a [M,K], a_s [M,K/128], b [N,K], b_s [N,K/128] expected")
     y = torch.empty(M, N, dtype=out_dtype, device=a.device)
-    ws, nws = _workspace(M, N, K, a.device)
+    nws = int(lib().fp8bs_gemm_rowwise_workspace_size(M, N, K))
+    ws = torch.empty(nws, dtype=torch.uint8, device=a.device) if nws else None
     dt = DTYPE_F32 if out_dtype == torch.float32 else DTYPE_BF16
     _check(lib().fp8bs_fp8_gemm_rowwise(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K,
                                         _scale_fmt(scale_fmt), _ptr(y), dt, _ptr(ws), nws,

@@ -218,7 +218,7 @@ fp8bs_status make_tmap_out(CUtensorMap* map, const void* y, const void* ws, int6
 // start early), which overlaps launch latency and prologues across the
 // act_quant -> GEMM -> split-K reduction chain.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -227,7 +227,7 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, 
   attr[n].val.programmaticStreamSerializationAllowed = 1;
   ++n;
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -388,6 +388,12 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
   return best;
 }
 
+// Bytes of the K-block-major copies of the two scale tables that the
+// row-scaled GEMM stages in its workspace.
+size_t rowwise_stage_bytes(int64_t M, int64_t N, int64_t K) {
+  return static_cast<size_t>(M + N) * static_cast<size_t>(K / 128) * sizeof(float);
+}
+
 size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   if (pl.tail_splits > 0)
     return static_cast<size_t>(pl.tail_tiles) * pl.tail_splits * 128 * pl.bn * sizeof(float);
@@ -447,7 +453,11 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
   const Plan pl = plan_gemm(M, N, K, *info, w_rowwise ? GemmKind::kRowScaled : GemmKind::kPromotion);
-  const size_t need = plan_workspace(pl, M, N);
+  // Row scales on W: both scale tables are staged K-block-major after the
+  // split-K area of the workspace.
+  const size_t split_bytes = plan_workspace(pl, M, N);
+  const size_t stage_off = (split_bytes + 255) & ~static_cast<size_t>(255);
+  const size_t need = w_rowwise ? stage_off + rowwise_stage_bytes(M, N, K) : split_bytes;
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
 
@@ -461,6 +471,17 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma, out_f32)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
+  if (w_rowwise) {
+    float* sa_t = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + stage_off);
+    float* sw_t = sa_t + M * (K / 128);
+    const int64_t tiles = ((M + 31) / 32 + (N + 31) / 32) * ((K / 128 + 31) / 32);
+    const cudaError_t se = launch(scale_tables_kmajor_kernel, grid_for(tiles, 1, info->sms * 8),
+                                  dim3(32, 8), 0, st, a_s, sa_t, M, w_s, sw_t, N,
+                                  static_cast<int>(K / 128));
+    if (se != cudaSuccess) return cuda_fail(se, "scale staging launch");
+    p.sa = sa_t;
+    p.sw = sw_t;
+  }
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
@@ -532,7 +553,11 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
   const Plan pl = plan_gemm(M, N, K, *info, GemmKind::kBlockScaled);
-  const size_t need = plan_workspace(pl, M, N);
+  // Row scales on W: both scale tables are staged K-block-major after the
+  // split-K area of the workspace.
+  const size_t split_bytes = plan_workspace(pl, M, N);
+  const size_t stage_off = (split_bytes + 255) & ~static_cast<size_t>(255);
+  const size_t need = w_rowwise ? stage_off + rowwise_stage_bytes(M, N, K) : split_bytes;
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
   CUtensorMap ta, tw, ty;
@@ -542,6 +567,17 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   if ((r = make_tmap_out(&ty, y, ws, M, N, pl.splits, &p.y_tma, out_f32)) != FP8BS_OK) return r;
   p.sa = a_s;
   p.sw = w_s;
+  if (w_rowwise) {
+    float* sa_t = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + stage_off);
+    float* sw_t = sa_t + M * (K / 128);
+    const int64_t tiles = ((M + 31) / 32 + (N + 31) / 32) * ((K / 128 + 31) / 32);
+    const cudaError_t se = launch(scale_tables_kmajor_kernel, grid_for(tiles, 1, info->sms * 8),
+                                  dim3(32, 8), 0, st, a_s, sa_t, M, w_s, sw_t, N,
+                                  static_cast<int>(K / 128));
+    if (se != cudaSuccess) return cuda_fail(se, "scale staging launch");
+    p.sa = sa_t;
+    p.sw = sw_t;
+  }
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
@@ -591,6 +627,18 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
     if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
   }
   return FP8BS_OK;
+}
+
+// CTAs of `kernel` that fit on one SM at once (at least 1): persistent
+// kernels that loop over tiles are launched with that many per SM.
+template <typename K>
+int resident_ctas(K kernel, int threads, size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 1;
+  }
+  return n > 0 ? n : 1;
 }
 
 // y = decode(q) * scale over an M x N code matrix, the scale of (row, col)
@@ -769,8 +817,9 @@ fp8bs_status fp8bs_fp8_transpose(const uint8_t* q, const float* s, int64_t R, in
   cudaError_t e;
   if (R % 16 == 0 && C % 16 == 0) {
     const int64_t tiles = ((R + 127) / 128) * ((C + 127) / 128);
-    e = launch(fp8_transpose_kernel, grid_for(tiles, 1, info->sms * 6), kTrThreads, 0, stm, q, s,
-               qt, st, R, C, sr, sc);
+    const int per_sm = resident_ctas(fp8_transpose_kernel, kTrThreads, 0);
+    e = launch(fp8_transpose_kernel, grid_for(tiles, 1, info->sms * per_sm), kTrThreads, 0, stm,
+               q, s, qt, st, R, C, sr, sc);
   } else {
     e = launch(fp8_transpose_any_kernel, grid_for(R * C, 256, info->sms * 8), 256, 0, stm, q, s,
                qt, st, R, C, sr, sc);
@@ -803,7 +852,11 @@ fp8bs_status fp8bs_act_quant_transposed(const void* x, fp8bs_dtype x_dtype, int6
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
   const int64_t tiles = (rows / 128) * ((cols + 127) / 128);
-  const int grid = grid_for(tiles, 1, info->sms * 4);
+  const int per_sm =
+      x_dtype == FP8BS_DTYPE_BF16
+          ? resident_ctas(act_quant_transposed_kernel<__nv_bfloat16, false>, kAqtThreads, 0)
+          : resident_ctas(act_quant_transposed_kernel<float, false>, kAqtThreads, 0);
+  const int grid = grid_for(tiles, 1, info->sms * per_sm);
   cudaStream_t stm = as_stream(stream);
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   cudaError_t e;
@@ -957,6 +1010,17 @@ size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   return std::max({plan_workspace(plan_gemm(M, N, K, *info), M, N),
                    plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N),
                    plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kRowScaled), M, N)});
+}
+
+size_t fp8bs_gemm_rowwise_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  int dev;
+  DeviceInfo* info;
+  if (device_setup(&dev, &info) != FP8BS_OK) return 0;
+  const size_t split = std::max(
+      plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kRowScaled), M, N),
+      plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N));
+  return ((split + 255) & ~static_cast<size_t>(255)) + rowwise_stage_bytes(M, N, K);
 }
 
 const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {

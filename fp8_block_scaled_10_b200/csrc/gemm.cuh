@@ -319,8 +319,10 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
   return t;
 }
 
-// BROW: one scale per row of W (W column of y) and K block, w_s [N, K/128],
-// as both operands of the weight-gradient GEMM carry (dense mode only).  The
+// BROW: one scale per row of W (W column of y) and K block, as both operands
+// of the weight-gradient GEMM carry (dense mode only).  Both scale tables are
+// then read K-block-major, sa [K/128][M] and sw [K/128][N] (the host stages
+// them so), which makes the scale producer's loads coalesced.  The
 // scale producer then fills the slot with the tile's BN column scales, the
 // epilogue multiplies a_s[row] by each column's scale before its FMA, and
 // since those reads outlast the TMEM buffer's release, the slot has its own
@@ -532,13 +534,17 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
-        va[j] = (c.valid && row < c.row_end) ? __ldg(p.sa + row * p.kbn + c.kb) : 0.0f;
+        va[j] = (c.valid && row < c.row_end)
+                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
+                    : 0.0f;
       }
       if (BROW) {
+        // K-block-major tables (sa [kbn][M], sw [kbn][N]): lanes read
+        // consecutive rows / columns, one coalesced load per 32 values.
 #pragma unroll
         for (int j = 0; j < kWRegs; ++j) {
           const int64_t col = c.n0 + lane + 32 * j;
-          vw[j] = (c.valid && col < p.N) ? __ldg(p.sw + col * p.kbn + c.kb) : 0.0f;
+          vw[j] = (c.valid && col < p.N) ? __ldg(p.sw + c.kb * static_cast<int64_t>(p.N) + col) : 0.0f;
         }
       } else {
         const int nb = c.nb0 + lane;
@@ -644,12 +650,21 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
             const float sc = C::kNbSpan == 1 ? scale_nb[0] : (nb_of[c] ? scale_nb[C::kNbSpan - 1] : scale_nb[0]);
             const float2 scale2 = make_float2(sc, sc);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
+            for (int j = 0; j < 16; j += 2) {
+              // BROW: four column scales per 16-byte (broadcast) read
+              float2 s_lo = scale2, s_hi = scale2;
+              if (BROW) {
+                const float4 sb4 = *reinterpret_cast<const float4*>(sb_col + 32 * c + 2 * j);
+                s_lo = __fmul2_rn(sa2, make_float2(sb4.x, sb4.y));
+                s_hi = __fmul2_rn(sa2, make_float2(sb4.z, sb4.w));
+              }
               acc[c * 16 + j] = __ffma2_rn(
                   make_float2(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1])),
-                  BROW ? __fmul2_rn(sa2, *reinterpret_cast<const float2*>(sb_col + 32 * c + 2 * j))
-                       : scale2,
-                  acc[c * 16 + j]);
+                  s_lo, acc[c * 16 + j]);
+              acc[c * 16 + j + 1] = __ffma2_rn(
+                  make_float2(__uint_as_float(v[c][2 * j + 2]), __uint_as_float(v[c][2 * j + 3])),
+                  s_hi, acc[c * 16 + j + 1]);
+            }
           }
         } else {
           // Two register buffers: the load of chunk c+1 is in flight while the
@@ -671,12 +686,20 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
             const float sc = C::kNbSpan == 1 ? scale_nb[0] : (nb_of[c] ? scale_nb[C::kNbSpan - 1] : scale_nb[0]);
             const float2 scale2 = make_float2(sc, sc);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
+            for (int j = 0; j < 16; j += 2) {
+              float2 s_lo = scale2, s_hi = scale2;
+              if (BROW) {
+                const float4 sb4 = *reinterpret_cast<const float4*>(sb_col + 32 * c + 2 * j);
+                s_lo = __fmul2_rn(sa2, make_float2(sb4.x, sb4.y));
+                s_hi = __fmul2_rn(sa2, make_float2(sb4.z, sb4.w));
+              }
               acc[c * 16 + j] = __ffma2_rn(
                   make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])),
-                  BROW ? __fmul2_rn(sa2, *reinterpret_cast<const float2*>(sb_col + 32 * c + 2 * j))
-                       : scale2,
-                  acc[c * 16 + j]);
+                  s_lo, acc[c * 16 + j]);
+              acc[c * 16 + j + 1] = __ffma2_rn(
+                  make_float2(__uint_as_float(cur[2 * j + 2]), __uint_as_float(cur[2 * j + 3])),
+                  s_hi, acc[c * 16 + j + 1]);
+            }
             if (c + 1 < NCH) tmem_ld_wait(nxt);
           }
         }

@@ -85,9 +85,11 @@ __device__ __forceinline__ uint32_t ue8m0_byte(float v, bool* bad) {
   return e;
 }
 
-// BROW: one scale per row of W and K block (w_s [N, K/128], dense mode), the
-// second operand of the weight-gradient GEMM; the W atoms then hold a scale
-// per row, laid out like A's, instead of one block scale repeated.
+// BROW: one scale per row of W and K block (dense mode), the second operand
+// of the weight-gradient GEMM; the W atoms then hold a scale per row, laid
+// out like A's, instead of one block scale repeated.  Both scale tables are
+// then read K-block-major, sa [K/128][M] and sw [K/128][N], as the host
+// stages them.
 template <int BN, bool GROUPED, bool BROW = false>
 __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
     fp8_gemm_bs_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -231,14 +233,17 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
-        va[j] = (c.valid && row < c.row_end) ? __ldg(p.sa + row * p.kbn + c.kb) : 1.0f;
+        va[j] = (c.valid && row < c.row_end)
+                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
+                    : 1.0f;
       }
       if (BROW) {
-        // value 4a + j: row 128a + lane + 32j of the tile's W rows
+        // value 4a + j: row 128a + lane + 32j of the tile's W rows, from the
+        // K-block-major table sw [kbn][N] (coalesced across lanes)
 #pragma unroll
         for (int i = 0; i < kWVals; ++i) {
           const int64_t n = c.n0 + 128 * (i / 4) + lane + 32 * (i % 4);
-          vw[i] = (c.valid && n < p.N) ? __ldg(p.sw + n * p.kbn + c.kb) : 1.0f;
+          vw[i] = (c.valid && n < p.N) ? __ldg(p.sw + c.kb * static_cast<int64_t>(p.N) + n) : 1.0f;
         }
       } else {
 #pragma unroll

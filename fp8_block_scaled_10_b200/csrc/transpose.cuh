@@ -53,17 +53,29 @@ __global__ void __launch_bounds__(kTrThreads)
     st[b * sr + a] = s[i];
   }
   const int64_t tiles_r = (R + 127) / 128, tiles_c = (C + 127) / 128;
-  for (int64_t tile = blockIdx.x; tile < tiles_r * tiles_c; tile += gridDim.x) {
+  const int64_t ntiles = tiles_r * tiles_c;
+  // 1. 128 rows x 8 chunks of 16 bytes per tile, loaded one tile ahead into
+  //    registers so that the loads of the next tile overlap this one's work.
+  uint4 pre[4];
+  auto load_tile = [&](int64_t tile) {
     const int64_t row0 = (tile / tiles_c) * 128, col0 = (tile % tiles_c) * 128;
-    // 1. 128 rows x 8 chunks of 16 bytes
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = u * 32 + (t >> 3), sg = t & 7;
       const int64_t gr = row0 + r, gc = col0 + 16 * sg;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (gr < R && gc < C) v = __ldcs(reinterpret_cast<const uint4*>(q + gr * C + gc));
-      *reinterpret_cast<uint4*>(&smA[r * kTrApitch + 4 * sg]) = v;
+      pre[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (gr < R && gc < C) pre[u] = __ldcs(reinterpret_cast<const uint4*>(q + gr * C + gc));
     }
+  };
+  if (static_cast<int64_t>(blockIdx.x) < ntiles) load_tile(blockIdx.x);
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t row0 = (tile / tiles_c) * 128, col0 = (tile % tiles_c) * 128;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = u * 32 + (t >> 3), sg = t & 7;
+      *reinterpret_cast<uint4*>(&smA[r * kTrApitch + 4 * sg]) = pre[u];
+    }
+    if (tile + gridDim.x < ntiles) load_tile(tile + gridDim.x);
     __syncthreads();
     // 2. 32 x 32 blocks of 4 x 4 bytes: block (br, bc) holds rows 4br.. and
     //    columns 4bc..; its transpose is rows 4bc.. of T at word br.
@@ -120,6 +132,42 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
+// Scale staging for the row-scaled GEMM: the two per-row scale tables
+// a_s [Ma, kbn] and b_s [Mb, kbn] transposed to K-block-major [kbn, Ma] and
+// [kbn, Mb], 32 x 32 tiles through shared memory (tiles of a_s first, then
+// of b_s, over one grid-stride loop).  Block 32 x 8 threads.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    scale_tables_kmajor_kernel(const float* __restrict__ a_s, float* __restrict__ a_t, int64_t Ma,
+                               const float* __restrict__ b_s, float* __restrict__ b_t, int64_t Mb,
+                               int kbn) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float tile[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int64_t ntc = (kbn + 31) / 32;
+  const int64_t ta = ((Ma + 31) / 32) * ntc, tb = ((Mb + 31) / 32) * ntc;
+  for (int64_t i = blockIdx.x; i < ta + tb; i += gridDim.x) {
+    const bool is_a = i < ta;
+    const int64_t ti = is_a ? i : i - ta;
+    const float* in = is_a ? a_s : b_s;
+    float* out = is_a ? a_t : b_t;
+    const int64_t rows = is_a ? Ma : Mb;
+    const int64_t r0 = (ti / ntc) * 32, c0 = (ti % ntc) * 32;
+    for (int k = ty; k < 32; k += 8) {
+      const int64_t r = r0 + k, c = c0 + tx;
+      tile[k][tx] = (r < rows && c < kbn) ? in[r * kbn + c] : 0.0f;
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+      const int64_t c = c0 + k, r = r0 + tx;
+      if (c < kbn && r < rows) out[c * rows + r] = tile[tx][k];
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // act_quant in 128 x 1 column blocks, written transposed: for x [R, C]
 // (R % 128 == 0, C % 8 == 0), qT [C, R] and sT [C, R / 128] are act_quant of
 // x^T.  One 128 x 128 tile per step: thread t owns the 8 x 8 block of rows
@@ -142,19 +190,47 @@ __global__ void __launch_bounds__(kAqtThreads)
   const int t = threadIdx.x;
   const int cg = t & 15, rg = t >> 4;
   const int64_t nrb = R / 128, tiles_c = (C + 127) / 128;
-  for (int64_t tile = blockIdx.x; tile < nrb * tiles_c; tile += gridDim.x) {
+  const int64_t ntiles = nrb * tiles_c;
+  // bf16 input: the thread's 8 x 16 bytes of the next tile are loaded into
+  // registers while this tile is processed (fp32 input, twice the registers,
+  // is loaded when it is needed).
+  constexpr bool kPrefetch = sizeof(T) == 2;
+  uint4 pre[kPrefetch ? 8 : 1];
+  auto load_raw = [&](int64_t tile) {
+    const int64_t gc = (tile % tiles_c) * 128 + 8 * cg;
+    const int64_t row0 = (tile / tiles_c) * 128;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      pre[k] = gc < C ? __ldcs(reinterpret_cast<const uint4*>(x + (row0 + 8 * rg + k) * C + gc))
+                      : make_uint4(0u, 0u, 0u, 0u);
+  };
+  if (kPrefetch && static_cast<int64_t>(blockIdx.x) < ntiles) load_raw(blockIdx.x);
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int64_t tr = tile / tiles_c;
     const int64_t row0 = tr * 128, col0 = (tile % tiles_c) * 128;
     const int64_t gc = col0 + 8 * cg;
     const bool col_ok = gc < C;
     float v[8][8];
+    if constexpr (kPrefetch) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (col_ok) {
-        load8(x + (row0 + 8 * rg + k) * C + gc, v[k]);
-      } else {
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t w[4] = {pre[k].x, pre[k].y, pre[k].z, pre[k].w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[k][c] = 0.0f;
+        for (int j = 0; j < 4; ++j) {
+          v[k][2 * j] = __uint_as_float(w[j] << 16);
+          v[k][2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+      if (tile + gridDim.x < ntiles) load_raw(tile + gridDim.x);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (col_ok) {
+          load8(x + (row0 + 8 * rg + k) * C + gc, v[k]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[k][c] = 0.0f;
+        }
       }
     }
     float pm[8];

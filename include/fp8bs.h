@@ -363,10 +363,14 @@ FP8BS_API fp8bs_status fp8bs_fp8_transpose(const uint8_t *q, const float *s, int
  *          scales positive normal powers of two: the block-scaled MMA, with
  *          the FP8BS_ERR_SCALE report of fp8bs_fp8_gemm_ue8m0)
  *   y      device, [M, N], fp32 (y_dtype = F32) or bf16, written
- *   workspace: fp8bs_gemm_workspace_size(M, N, K) bytes suffice
+ *   workspace: fp8bs_gemm_rowwise_workspace_size(M, N, K) bytes (the split-K
+ *          partials and K-block-major copies of a_s and b_s, which make the
+ *          kernels' scale loads coalesced)
  * K % 128 == 0, ragged M and N; errors as for fp8bs_fp8_gemm, plus
  * FP8BS_ERR_INVALID_ARG for an unknown fmt or y_dtype.
  */
+FP8BS_API size_t fp8bs_gemm_rowwise_workspace_size(int64_t M, int64_t N, int64_t K);
+
 FP8BS_API fp8bs_status fp8bs_fp8_gemm_rowwise(const uint8_t *a, const float *a_s,
                                               const uint8_t *b, const float *b_s, int64_t M,
                                               int64_t N, int64_t K, fp8bs_scale_fmt fmt, void *y,
