@@ -854,7 +854,7 @@ fp8bs_status fp8bs_act_quant_transposed(const void* x, fp8bs_dtype x_dtype, int6
   const int64_t tiles = (rows / 128) * ((cols + 127) / 128);
   const int per_sm =
       x_dtype == FP8BS_DTYPE_BF16
-          ? resident_ctas(act_quant_transposed_kernel<__nv_bfloat16, false>, kAqtThreads, 0)
+          ? resident_ctas(act_quant_transposed_bf16_kernel<false, kAqtPrefetch>, kAqtThreads, 0)
           : resident_ctas(act_quant_transposed_kernel<float, false>, kAqtThreads, 0);
   const int grid = grid_for(tiles, 1, info->sms * per_sm);
   cudaStream_t stm = as_stream(stream);
@@ -862,10 +862,10 @@ fp8bs_status fp8bs_act_quant_transposed(const void* x, fp8bs_dtype x_dtype, int6
   cudaError_t e;
   if (x_dtype == FP8BS_DTYPE_BF16) {
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
-    e = ue ? launch(act_quant_transposed_kernel<__nv_bfloat16, true>, grid, kAqtThreads, 0, stm, xb,
-                    qt, st, rows, cols)
-           : launch(act_quant_transposed_kernel<__nv_bfloat16, false>, grid, kAqtThreads, 0, stm,
-                    xb, qt, st, rows, cols);
+    e = ue ? launch(act_quant_transposed_bf16_kernel<true, kAqtPrefetch>, grid, kAqtThreads, 0,
+                    stm, xb, qt, st, rows, cols)
+           : launch(act_quant_transposed_bf16_kernel<false, kAqtPrefetch>, grid, kAqtThreads, 0,
+                    stm, xb, qt, st, rows, cols);
   } else {
     const auto* xf = static_cast<const float*>(x);
     e = ue ? launch(act_quant_transposed_kernel<float, true>, grid, kAqtThreads, 0, stm, xf, qt,

@@ -19,6 +19,25 @@
 
 namespace fp8bs {
 
+// Tile order of the transposing kernels: groups of kBandGroup row bands
+// (128 rows each) advance together across the columns, so that the CTAs in
+// flight at once read a few KB of each input row and write a KB of each output
+// row (a column-first order writes 128 bytes per output row and moves on).
+constexpr int64_t kBandGroup = 8;
+__device__ __forceinline__ void tile_coords(int64_t tile, int64_t bands, int64_t tiles_c,
+                                            int64_t& tr, int64_t& tc) {
+  const int64_t full = (bands / kBandGroup) * kBandGroup * tiles_c;
+  if (tile < full) {
+    const int64_t grp = tile / (kBandGroup * tiles_c), in = tile % (kBandGroup * tiles_c);
+    tr = grp * kBandGroup + in % kBandGroup;
+    tc = in / kBandGroup;
+  } else {
+    const int64_t rest = bands % kBandGroup, in = tile - full;
+    tr = (bands / kBandGroup) * kBandGroup + in % rest;
+    tc = in / rest;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // FP8 transpose: qT[c, r] = q[r, c] on 128 x 128 byte tiles (rows and columns
 // multiples of 16), and sT = s^T for the block scales.
@@ -58,7 +77,9 @@ __global__ void __launch_bounds__(kTrThreads)
   //    registers so that the loads of the next tile overlap this one's work.
   uint4 pre[4];
   auto load_tile = [&](int64_t tile) {
-    const int64_t row0 = (tile / tiles_c) * 128, col0 = (tile % tiles_c) * 128;
+    int64_t tr, tc;
+    tile_coords(tile, tiles_r, tiles_c, tr, tc);
+    const int64_t row0 = tr * 128, col0 = tc * 128;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = u * 32 + (t >> 3), sg = t & 7;
@@ -69,7 +90,9 @@ __global__ void __launch_bounds__(kTrThreads)
   };
   if (static_cast<int64_t>(blockIdx.x) < ntiles) load_tile(blockIdx.x);
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t row0 = (tile / tiles_c) * 128, col0 = (tile % tiles_c) * 128;
+    int64_t tr, tc;
+    tile_coords(tile, tiles_r, tiles_c, tr, tc);
+    const int64_t row0 = tr * 128, col0 = tc * 128;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = u * 32 + (t >> 3), sg = t & 7;
@@ -178,6 +201,33 @@ __global__ void __launch_bounds__(256)
 // act_quant) and stores 8 codes of one output row.
 // ---------------------------------------------------------------------------
 constexpr int kAqtThreads = 256;
+constexpr bool kAqtPrefetch = false;
+
+
+// The codes of a tile go through shared memory so that the global stores are
+// whole 128-byte runs of output rows: thread (cg, rg) puts the 8 codes of
+// output row 8cg + c (input rows 8rg..) in 8-byte unit rg of that row,
+// stored at unit rg ^ (row / 8 mod 16), a swizzle that spreads the 16
+// different rows one warp instruction writes over all banks; then each
+// group of 8 lanes copies one output row to global memory, 16 bytes each.
+__device__ __forceinline__ void stage_codes(uint2* smq, int cg, int rg, int c, uint2 codes) {
+  const int row = 8 * cg + c;
+  smq[row * 16 + (rg ^ (cg & 15))] = codes;
+}
+
+__device__ __forceinline__ void store_staged_codes(const uint2* smq, uint8_t* __restrict__ qt,
+                                                   int64_t R, int64_t C, int64_t row0,
+                                                   int64_t col0, int t) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int j = u * 32 + (t >> 3), h = t & 7;
+    const int key = (j >> 3) & 15;
+    const uint2 lo = smq[j * 16 + ((2 * h) ^ key)], hi = smq[j * 16 + ((2 * h + 1) ^ key)];
+    if (col0 + j < C)
+      __stcs(reinterpret_cast<uint4*>(qt + (col0 + j) * R + row0 + 16 * h),
+             make_uint4(lo.x, lo.y, hi.x, hi.y));
+  }
+}
 
 template <typename T, bool UE8M0>
 __global__ void __launch_bounds__(kAqtThreads)
@@ -187,13 +237,13 @@ __global__ void __launch_bounds__(kAqtThreads)
   pdl_wait();
   __shared__ __align__(16) float red[16][128];
   __shared__ __align__(16) float scol[128];
+  __shared__ __align__(16) uint2 smq[128 * 16];
   const int t = threadIdx.x;
   const int cg = t & 15, rg = t >> 4;
   const int64_t nrb = R / 128, tiles_c = (C + 127) / 128;
   const int64_t ntiles = nrb * tiles_c;
-  // bf16 input: the thread's 8 x 16 bytes of the next tile are loaded into
-  // registers while this tile is processed (fp32 input, twice the registers,
-  // is loaded when it is needed).
+  // (bf16 input takes act_quant_transposed_bf16_kernel; this path prefetches
+  // only if instantiated for a 2-byte type.)
   constexpr bool kPrefetch = sizeof(T) == 2;
   uint4 pre[kPrefetch ? 8 : 1];
   auto load_raw = [&](int64_t tile) {
@@ -260,11 +310,105 @@ __global__ void __launch_bounds__(kAqtThreads)
         float col[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) col[k] = v[k][c];
-        const uint2 codes = quantize8<UE8M0>(col, sc, r);
-        __stcs(reinterpret_cast<uint2*>(qt + (gc + c) * R + row0 + 8 * rg), codes);
+        stage_codes(smq, cg, rg, c, quantize8<UE8M0>(col, sc, r));
       }
     }
     __syncthreads();
+    store_staged_codes(smq, qt, R, C, row0, col0, t);
+  }
+}
+
+// bf16 input, the same tile walk with the tile kept packed: each thread holds
+// its 8 rows x 8 columns as 32 words of bf16 pairs, takes the column amax
+// with 16-bit SIMD maxima of the sign-cleared halves (a non-negative bf16
+// orders like its bit pattern) and unpacks a value only to quantize it.  The
+// smaller register footprint lets more CTAs share an SM, which keeps more
+// loads in flight.  PREFETCH additionally loads the next tile's words while
+// this tile is processed.
+template <bool UE8M0, bool PREFETCH>
+__global__ void __launch_bounds__(kAqtThreads)
+    act_quant_transposed_bf16_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ qt,
+                                     float* __restrict__ st, int64_t R, int64_t C) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __align__(16) float red[16][128];
+  __shared__ __align__(16) float scol[128];
+  __shared__ __align__(16) uint2 smq[128 * 16];
+  const int t = threadIdx.x;
+  const int cg = t & 15, rg = t >> 4;
+  const int64_t nrb = R / 128, tiles_c = (C + 127) / 128;
+  const int64_t ntiles = nrb * tiles_c;
+  uint4 cur[8], nxt[PREFETCH ? 8 : 1];
+  auto load_words = [&](int64_t tile, uint4 (&w)[PREFETCH ? 8 : 1], uint4 (&w8)[8], bool to_next) {
+    int64_t tr, tc;
+    tile_coords(tile, nrb, tiles_c, tr, tc);
+    const int64_t gc = tc * 128 + 8 * cg;
+    const int64_t row0 = tr * 128;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 v = gc < C ? __ldcs(reinterpret_cast<const uint4*>(x + (row0 + 8 * rg + k) * C + gc))
+                             : make_uint4(0u, 0u, 0u, 0u);
+      if (PREFETCH && to_next) w[PREFETCH ? k : 0] = v; else w8[k] = v;
+    }
+  };
+  if (PREFETCH && static_cast<int64_t>(blockIdx.x) < ntiles) load_words(blockIdx.x, nxt, cur, true);
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    int64_t tr, tc;
+    tile_coords(tile, nrb, tiles_c, tr, tc);
+    const int64_t row0 = tr * 128, col0 = tc * 128;
+    const int64_t gc = col0 + 8 * cg;
+    const bool col_ok = gc < C;
+    if (PREFETCH) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cur[k] = nxt[PREFETCH ? k : 0];
+      if (tile + gridDim.x < ntiles) load_words(tile + gridDim.x, nxt, cur, true);
+    } else {
+      load_words(tile, nxt, cur, false);
+    }
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      m[0] = __vmaxu2(m[0], cur[k].x & 0x7FFF7FFFu);
+      m[1] = __vmaxu2(m[1], cur[k].y & 0x7FFF7FFFu);
+      m[2] = __vmaxu2(m[2], cur[k].z & 0x7FFF7FFFu);
+      m[3] = __vmaxu2(m[3], cur[k].w & 0x7FFF7FFFu);
+    }
+    *reinterpret_cast<float4*>(&red[rg][8 * cg]) =
+        make_float4(__uint_as_float(m[0] << 16), __uint_as_float(m[0] & 0xFFFF0000u),
+                    __uint_as_float(m[1] << 16), __uint_as_float(m[1] & 0xFFFF0000u));
+    *reinterpret_cast<float4*>(&red[rg][8 * cg + 4]) =
+        make_float4(__uint_as_float(m[2] << 16), __uint_as_float(m[2] & 0xFFFF0000u),
+                    __uint_as_float(m[3] << 16), __uint_as_float(m[3] & 0xFFFF0000u));
+    __syncthreads();
+    if (t < 128) {
+      float amax = red[0][t];
+#pragma unroll
+      for (int i = 1; i < 16; ++i) amax = fmaxf(amax, red[i][t]);
+      const float sc = block_scale(amax, UE8M0);
+      scol[t] = sc;
+      if (col0 + t < C) st[(col0 + t) * nrb + tr] = sc;
+    }
+    __syncthreads();
+    if (col_ok) {
+      const float4 s_lo = *reinterpret_cast<const float4*>(&scol[8 * cg]);
+      const float4 s_hi = *reinterpret_cast<const float4*>(&scol[8 * cg + 4]);
+      const float sc8[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float sc = sc8[c];
+        const float r = __frcp_rn(sc);
+        float col[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t w = (c >> 1) == 0 ? cur[k].x : (c >> 1) == 1 ? cur[k].y
+                           : (c >> 1) == 2 ? cur[k].z : cur[k].w;
+          col[k] = __uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
+        }
+        stage_codes(smq, cg, rg, c, quantize8<UE8M0>(col, sc, r));
+      }
+    }
+    __syncthreads();
+    store_staged_codes(smq, qt, R, C, row0, col0, t);
   }
 }
 
