@@ -50,7 +50,7 @@ FP8_OVER_BF16 = 2.0     # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLO
 # DRAM bytes (read + write) of one prefill GEMM launch from the ncu capture
 # summarised in profiles/fp8_gemm_prefill_M4096_N18432_K7168.md.  It belongs
 # to the kernel as captured; reset it to None whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES = 165.936128e6 + 134.464768e6
+GEMM_TRAFFIC_BYTES = 166.597376e6 + 132.455424e6
 
 
 def parse_args():
@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the per-workload parts")
+    ap.add_argument("--parts", choices=["all", "training"], default="all",
+                    help="which per-workload parts to run: all, or only the training GEMMs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -254,7 +256,7 @@ def time_events(fn, iters, flush=None, rounds=3):
     return statistics.median(means)
 
 
-def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
+def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
     """Per-workload kernel measurements (outside the step's timed region)."""
     parts = {}
     L = fp8bs.lib()
@@ -268,6 +270,9 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
         # the next timed launch) and leaves only clean, unrelated lines in L2.
         scratch.zero_()
         scratch_rd.sum()
+
+    if which == "training":
+        return run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush)
 
     # act_quant, x bf16 [16384, 7168] with 0.1% entries x100
     R, C = 16384, 7168
@@ -448,6 +453,65 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream):
     parts["experts_grouped_ue8m0_bs"] = {"rows": Mt, "us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
                                          "frac_fp8": fl / ms / 1e9 / fp8_peak,
                                          "kernel": "block-scaled MMA"}
+    del qa, sa, wg, sg, yg, offs
+    parts.update(run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush))
+    return parts
+
+
+def run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush):
+    """The training GEMMs of the dense up-projection over 4096 tokens (x [4096,
+    7168], W [18432, 7168], dy [4096, 18432]): W^T for the activation-gradient
+    GEMM dx = dy W (fp8_transpose, then the forward kernel at K=18432,
+    N=7168), the transposing quantizer of dy and x, and the weight-gradient
+    GEMM dW = dy^T x [18432, 7168] fp32 over K = 4096 tokens (fp8_gemm_rowwise)."""
+    parts = {}
+    L = fp8bs.lib()
+    T, N, K = 4096, 18432, 7168
+    qw = wl.e4m3_codes(N, K, seed=30, device="cuda")
+    sw = wl.uniform((N // 128, K // 128), 1e-5, 1e-3, seed=31, device="cuda")
+    qwt = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    swt = torch.empty(K // 128, N // 128, dtype=torch.float32, device="cuda")
+    f = lambda: L.fp8bs_fp8_transpose(vp(qw), vp(sw), N, K, 128, vp(qwt), vp(swt), stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10, flush)
+    nb = 2 * N * K + 2 * sw.numel() * 4
+    parts["fp8_transpose_W_18432x7168"] = {"us": ms * 1e3, "GB/s": nb / ms / 1e6,
+                                           "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
+    del qw, sw, qwt, swt
+    for rows, cols, name in ((T, K, "x"), (T, N, "dy")):
+        x = wl.heavy_tailed_channels(rows, cols, seed=40, device="cuda")
+        qt = torch.empty(cols, rows, dtype=torch.uint8, device="cuda")
+        st_ = torch.empty(cols, rows // 128, dtype=torch.float32, device="cuda")
+        f = lambda: L.fp8bs_act_quant_transposed(vp(x), 0, rows, cols, 128, 0, vp(qt), vp(st_),
+                                                 stream)
+        for _ in range(3):
+            f()
+        ms = time_events(f, 10, flush)
+        nb = rows * cols * 3 + st_.numel() * 4
+        parts["act_quant_transposed_%s_%dx%d" % (name, rows, cols)] = {
+            "us": ms * 1e3, "GB/s": nb / ms / 1e6, "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
+        del x, qt, st_
+    fl = 2 * N * K * T
+    for fmt, fname in ((0, "none"), (1, "ue8m0")):
+        a = wl.normal_with_outliers(N, T, seed=41, frac=0.001, factor=20.0, device="cuda")
+        b = wl.normal_with_outliers(K, T, seed=42, frac=0.001, factor=20.0, device="cuda")
+        qa, sa = fp8bs.act_quant(a, 128, "ue8m0" if fmt else None)
+        qb, sb = fp8bs.act_quant(b, 128, "ue8m0" if fmt else None)
+        del a, b
+        qa, qb = qa.view(torch.uint8), qb.view(torch.uint8)
+        dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+        nws = int(L.fp8bs_gemm_rowwise_workspace_size(N, K, T))
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
+        f = lambda: L.fp8bs_fp8_gemm_rowwise(vp(qa), vp(sa), vp(qb), vp(sb), N, K, T, fmt, vp(dw),
+                                             1, vp(ws), nws, stream)
+        for _ in range(3):
+            f()
+        ms = time_events(f, 10)
+        parts["wgrad_M18432_N7168_K4096_%s" % fname] = {
+            "us": ms * 1e3, "TFLOP/s": fl / ms / 1e9, "frac_fp8": fl / ms / 1e9 / fp8_peak,
+            "out": "fp32", "kernel": "block-scaled MMA" if fmt else "promotion, per-column scales"}
+        del qa, sa, qb, sb, dw, ws
     return parts
 
 
@@ -581,7 +645,7 @@ def ours(args, dist):
     del x_host, y_host, lin
     torch.cuda.empty_cache()
     if not args.quick:
-        result["parts"] = run_parts(fp8bs, wl, hbm, fp8_peak, stream)
+        result["parts"] = run_parts(fp8bs, wl, hbm, fp8_peak, stream, args.parts)
         result["parts_note"] = "each part: median over 3 rounds of the mean of 10 event-timed launches, after 3 warm-ups; memory-bound parts and decode GEMMs flush L2 before each launch (memset of 4x L2 size, then a read of 2x L2 size so no dirty lines are written back inside the timed launch); GB/s of algorithmic bytes vs %s HBM %.1f GB/s" % (peak_kind, hbm)
     if dist.rank == 0:
         rows, run, _ = cpu_baseline(args.cpu_seconds)
