@@ -60,8 +60,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the per-workload parts")
-    ap.add_argument("--parts", choices=["all", "training"], default="all",
-                    help="which per-workload parts to run: all, or only the training GEMMs")
+    ap.add_argument("--parts", choices=["all", "training", "experts"], default="all",
+                    help="which per-workload parts to run: all, only the training GEMMs, or only the grouped expert GEMMs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -273,6 +273,8 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
 
     if which == "training":
         return run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush)
+    if which == "experts":
+        return run_expert_parts(fp8bs, wl, fp8_peak, stream)
 
     # act_quant, x bf16 [16384, 7168] with 0.1% entries x100
     R, C = 16384, 7168
@@ -414,7 +416,16 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
             "gemm_then_act_quant_us": ms_s * 1e3,
             "note": "fp8bs_fp8_gemm_quant vs fp8bs_fp8_gemm + fp8bs_act_quant of the bf16 y"}
     del lin, q_out, s_out
-    # expert-batched grouped GEMM: 32 x W [2048, 7168], 65536 routed rows
+    parts.update(run_expert_parts(fp8bs, wl, fp8_peak, stream))
+    parts.update(run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush))
+    return parts
+
+
+def run_expert_parts(fp8bs, wl, fp8_peak, stream):
+    """The expert-batched grouped GEMM: 32 x W [2048, 7168], 65536 routed rows,
+    with fp32 scales (promotion kernel) and ue8m0 scales (block-scaled MMA)."""
+    parts = {}
+    L = fp8bs.lib()
     counts = wl.expert_counts(wl.EXPERT_TOKENS * wl.EXPERT_TOPK, wl.EXPERTS, seed=70)
     offs = torch.cat([torch.zeros(1, dtype=torch.int64), counts.cumsum(0)]).cuda()
     Mt = int(counts.sum())
@@ -453,8 +464,6 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
     parts["experts_grouped_ue8m0_bs"] = {"rows": Mt, "us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
                                          "frac_fp8": fl / ms / 1e9 / fp8_peak,
                                          "kernel": "block-scaled MMA"}
-    del qa, sa, wg, sg, yg, offs
-    parts.update(run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush))
     return parts
 
 

@@ -281,7 +281,23 @@ struct Plan {
   int grid;   // persistent CTAs
   // Split tail (see gemm::Params): 0 = none.
   int full_units = 0, tail_tiles = 0, tail_splits = 0, tail_kbps = 0;
+  int n_group = 1;   // band width of the tile order (gemm::tile_mn)
 };
+
+// Band width of the dense tile order for one K split.  m fastest (width 1)
+// reads each W tile once and A once per n tile, from L2 when A fits there
+// beside the W tiles in flight (up to kAResidentBytes).  A larger A would
+// come from HBM once per n tile; a band of n tiles whose W fits in
+// kWBandBytes of L2 then reads A once per band instead.  (Measured on B200:
+// the weight-gradient shape M = 18432, N = 7168, K = 4096 read 1.7 GB per
+// launch m-fastest, against 0.64 GB of operands and output.)
+constexpr int64_t kAResidentBytes = 40ll << 20;
+constexpr int64_t kWBandBytes = 20ll << 20;
+int choose_n_group(int64_t M, int64_t K, int bn, int n_tiles) {
+  if (M * K <= kAResidentBytes) return 1;
+  const int64_t g = kWBandBytes / (static_cast<int64_t>(bn) * K);
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, n_tiles)));
+}
 
 // The split tail's FP32 partials are kept within this many bytes, so that
 // every prefill plan also fits the library's static scratch array.
@@ -385,6 +401,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
       if (better) best = cand;
     }
   }
+  if (best.splits == 1 && compute_bound) best.n_group = choose_n_group(M, K, best.bn, best.n_tiles);
   return best;
 }
 
@@ -492,6 +509,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.nbn = static_cast<int>((N + 127) / 128);
   p.m_tiles = pl.m_tiles;
   p.n_tiles = pl.n_tiles;
+  p.n_group = pl.n_group;
   p.splits = pl.splits;
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
@@ -511,12 +529,12 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
     e = out_f32
             ? launch(gemm::tail_reduce_kernel<float>, grid_for(items, 256, info->sms * 8), 256, 0,
                      st, static_cast<const float*>(ws), static_cast<float*>(y), M,
-                     static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles,
-                     pl.tail_splits, pl.bn)
+                     static_cast<int>(N), pl.m_tiles, pl.n_tiles, pl.n_group, pl.full_units,
+                     pl.tail_tiles, pl.tail_splits, pl.bn)
             : launch(gemm::tail_reduce_kernel<__nv_bfloat16>, grid_for(items, 256, info->sms * 8),
                      256, 0, st, static_cast<const float*>(ws),
                      reinterpret_cast<__nv_bfloat16*>(y), M, static_cast<int>(N), pl.m_tiles,
-                     pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
+                     pl.n_tiles, pl.n_group, pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
     if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
   }
   if (pl.splits > 1) {
@@ -588,6 +606,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   p.nbn = static_cast<int>((N + 127) / 128);
   p.m_tiles = pl.m_tiles;
   p.n_tiles = pl.n_tiles;
+  p.n_group = pl.n_group;
   p.splits = pl.splits;
   p.kb_per_split = pl.kb_per_split;
   p.num_units = pl.units;
@@ -608,12 +627,12 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
     e = out_f32
             ? launch(gemm::tail_reduce_kernel<float>, grid_for(items, 256, info->sms * 8), 256, 0,
                      st, static_cast<const float*>(ws), static_cast<float*>(y), M,
-                     static_cast<int>(N), pl.m_tiles, pl.full_units, pl.tail_tiles,
-                     pl.tail_splits, pl.bn)
+                     static_cast<int>(N), pl.m_tiles, pl.n_tiles, pl.n_group, pl.full_units,
+                     pl.tail_tiles, pl.tail_splits, pl.bn)
             : launch(gemm::tail_reduce_kernel<__nv_bfloat16>, grid_for(items, 256, info->sms * 8),
                      256, 0, st, static_cast<const float*>(ws),
                      reinterpret_cast<__nv_bfloat16*>(y), M, static_cast<int>(N), pl.m_tiles,
-                     pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
+                     pl.n_tiles, pl.n_group, pl.full_units, pl.tail_tiles, pl.tail_splits, pl.bn);
     if (e != cudaSuccess) return cuda_fail(e, "split-tail reduce launch");
   }
   if (pl.splits > 1) {
@@ -1034,9 +1053,9 @@ const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
   const Plan pl = plan_gemm(M, N, K, *info);
   snprintf(buf, sizeof(buf),
            "bn=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d sms=%d "
-           "tail_tiles=%d tail_splits=%d",
+           "tail_tiles=%d tail_splits=%d n_group=%d",
            pl.bn, pl.m_tiles, pl.n_tiles, pl.splits, pl.kb_per_split, pl.units, pl.grid,
-           info->sms, pl.tail_tiles, pl.tail_splits);
+           info->sms, pl.tail_tiles, pl.tail_splits, pl.n_group);
   return buf;
 }
 
@@ -1181,6 +1200,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
   p.nbn = static_cast<int>((N + 127) / 128);
   p.m_tiles = 0;
   p.n_tiles = static_cast<int>((N + bn - 1) / bn);
+  p.n_group = 1;
   p.splits = 1;
   p.kb_per_split = p.kbn;
   p.num_units = 0;
@@ -1244,6 +1264,7 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   p.nbn = static_cast<int>((N + 127) / 128);
   p.m_tiles = 0;
   p.n_tiles = static_cast<int>((N + bn - 1) / bn);
+  p.n_group = 1;
   p.splits = 1;
   p.kb_per_split = p.kbn;
   p.num_units = 0;
@@ -1311,6 +1332,7 @@ fp8bs_status fp8bs_fp8_gemm_quant(const uint8_t* a, const float* a_s, const uint
   p.nbn = static_cast<int>((N + 127) / 128);
   p.m_tiles = m_tiles;
   p.n_tiles = n_tiles;
+  p.n_group = choose_n_group(M, K, bn, n_tiles);
   p.splits = 1;
   p.kb_per_split = p.kbn;
   p.num_units = static_cast<int>(units);

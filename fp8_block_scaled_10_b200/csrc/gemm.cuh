@@ -71,6 +71,8 @@ struct Params {
   int kbn;                  // K / 128
   int nbn;                  // cdiv(N, 128)
   int m_tiles;              // dense mode: tiles of kUnitRows rows
+  int n_group;              // dense mode, one split: tiles walk bands of n_group
+                            // n tiles, m fastest inside a band (see tile_mn)
   int n_tiles;
   int splits;
   int kb_per_split;
@@ -225,6 +227,21 @@ struct Unit {
 
 // Dense units: m tile fastest, so the CTAs running at the same time share W
 // tiles (and sweep all of A, which stays in L2).
+// Tile t of a dense problem with one K split: bands of g = n_group n tiles
+// (the last band narrower) are walked one after the other, and inside a band
+// the m tile changes slowest, so the CTAs running at once share the band's
+// W tiles (which stay in L2) while A streams once per band.  n_group = 1 is
+// the m-fastest order (each W tile read once, A once per n tile), which suits
+// an A small enough to stay in L2; a wide band suits a large A and a small W.
+__host__ __device__ __forceinline__ void tile_mn(int tile, int m_tiles, int n_tiles, int g,
+                                                 int& m_tile, int& n_tile) {
+  const int band = tile / (m_tiles * g);
+  const int width = min(g, n_tiles - band * g);
+  const int rem = tile - band * m_tiles * g;
+  m_tile = rem / width;
+  n_tile = band * g + rem % width;
+}
+
 template <int kUnitRows>
 __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   Unit t;
@@ -236,19 +253,26 @@ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
     const int tt = r % p.tail_tiles;
     const int tile = p.full_units + tt;
     t.split = r / p.tail_tiles;
-    t.n_tile = tile / p.m_tiles;
+    int m_tile;
+    tile_mn(tile, p.m_tiles, p.n_tiles, p.n_group, m_tile, t.n_tile);
     t.group = 0;
-    t.row0 = static_cast<int64_t>(tile % p.m_tiles) * kUnitRows;
+    t.row0 = static_cast<int64_t>(m_tile) * kUnitRows;
     t.row_end = p.M;
     t.kb0 = t.split * p.tail_kbps;
     t.kb1 = min(p.kbn, t.kb0 + p.tail_kbps);
     t.tail_slot = tt * p.tail_splits + t.split;
     return t;
   }
-  const int m_tile = u % p.m_tiles;
-  const int rest = u / p.m_tiles;
-  t.split = rest % p.splits;
-  t.n_tile = rest / p.splits;
+  int m_tile;
+  if (p.splits == 1) {
+    t.split = 0;
+    tile_mn(u, p.m_tiles, p.n_tiles, p.n_group, m_tile, t.n_tile);
+  } else {
+    m_tile = u % p.m_tiles;
+    const int rest = u / p.m_tiles;
+    t.split = rest % p.splits;
+    t.n_tile = rest / p.splits;
+  }
   t.group = 0;
   t.row0 = static_cast<int64_t>(m_tile) * kUnitRows;
   t.row_end = p.M;
@@ -864,7 +888,8 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
 template <typename OutT>
 __global__ void __launch_bounds__(256)
     tail_reduce_kernel(const float* __restrict__ ws, OutT* __restrict__ y, int64_t M,
-                       int N, int m_tiles, int full_units, int tail_tiles, int splits, int bn) {
+                       int N, int m_tiles, int n_tiles, int n_group, int full_units,
+                       int tail_tiles, int splits, int bn) {
   pdl_trigger();
   pdl_wait();
   const int groups = bn / 4;
@@ -874,9 +899,10 @@ __global__ void __launch_bounds__(256)
     const int tt = static_cast<int>(i / (BM * groups));
     const int rem = static_cast<int>(i - static_cast<int64_t>(tt) * BM * groups);
     const int r = rem / groups, c = (rem - r * groups) * 4;
-    const int tile = full_units + tt;
-    const int64_t row = static_cast<int64_t>(tile % m_tiles) * BM + r;
-    const int64_t col = static_cast<int64_t>(tile / m_tiles) * bn + c;
+    int m_tile, n_tile;
+    tile_mn(full_units + tt, m_tiles, n_tiles, n_group, m_tile, n_tile);
+    const int64_t row = static_cast<int64_t>(m_tile) * BM + r;
+    const int64_t col = static_cast<int64_t>(n_tile) * bn + c;
     if (row >= M || col >= N) continue;
     float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int sp = 0; sp < splits; ++sp) {
