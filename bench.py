@@ -50,7 +50,7 @@ FP8_OVER_BF16 = 2.0     # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLO
 # DRAM bytes (read + write) of one prefill GEMM launch from the ncu capture
 # summarised in profiles/fp8_gemm_prefill_M4096_N18432_K7168.md.  It belongs
 # to the kernel as captured; reset it to None whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES = 166.597376e6 + 132.455424e6
+GEMM_TRAFFIC_BYTES = 169.671168e6 + 135.812096e6
 
 
 def parse_args():
