@@ -211,7 +211,8 @@ class Linear:
         assert st == 0, self.L.fp8bs_last_error_message()
 
     def gemm_bs(self, stream):
-        """The block-scaled (ue8m0) GEMM; needs fmt=1 (power-of-two scales)."""
+        """The ue8m0 entry point (block-scaled MMA, or for decode-sized M the
+        promotion kernel); needs fmt=1 (power-of-two scales)."""
         st = self.L.fp8bs_fp8_gemm_ue8m0(vp(self.q), vp(self.s), vp(self.qw), vp(self.sw), self.m,
                                          self.n, self.k, vp(self.y), vp(self.ws), self.nws, stream)
         assert st == 0, self.L.fp8bs_last_error_message()
@@ -359,7 +360,7 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
                 else _resize(lin, fp8bs, wl, mm)
             lin.act_quant(stream)
             nbytes = nn * kk + 4 * (-(-nn // 128)) * (kk // 128) + mm * kk + 4 * mm * (kk // 128) + 2 * mm * nn
-            for tag, f in (("", lambda: lin.gemm(stream)), ("_bs", lambda: lin.gemm_bs(stream))):
+            for tag, f in (("", lambda: lin.gemm(stream)), ("_ue8m0", lambda: lin.gemm_bs(stream))):
                 for _ in range(3):
                     f()
                 ms = time_events(f, 10, flush)
@@ -367,7 +368,9 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
                     "us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / hbm,
                     "TFLOP/s": 2 * mm * nn * kk / ms / 1e9, "splitk_workspace": lin.nws,
                     "plan": fp8bs.gemm_plan(mm, nn, kk),
-                    "kernel": "block-scaled MMA" if tag else "promotion"}
+                    "kernel": ("fp8bs_fp8_gemm_ue8m0: promotion kernel with the power-of-two check"
+                               if mm <= 64 else "fp8bs_fp8_gemm_ue8m0: block-scaled MMA")
+                              if tag else "fp8bs_fp8_gemm: promotion"}
         del lin
     # prefill shapes: fused act_quant + GEMM per call, and the GEMM alone
     for kk, nn in wl.PREFILL_KN:

@@ -101,7 +101,18 @@ struct Params {
   // split: ws = y, y_tma 2 maps y as a single split; several: the reduction
   // writes FP32).  p.y is unused then.
   int out_f32;
+  // The caller promised power-of-two scales (a *_ue8m0 entry routed to this
+  // kernel): the scale producer checks every scale it loads and reports one
+  // that is not a positive normal power of two (device error 6).
+  int check_pow2;
 };
+
+// Nonzero unless v is a positive normal power of two.
+__device__ __forceinline__ uint32_t not_pow2(float v) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t e = (b >> 23) & 0xFFu;
+  return (b & 0x807FFFFFu) | static_cast<uint32_t>(e == 0u) | static_cast<uint32_t>(e == 0xFFu);
+}
 
 // Output staging for TMA stores of bf16 y: each epilogue warp owns one box of
 // 32 rows x 32 columns (2 KB) in shared memory, laid out in the 64-byte
@@ -554,13 +565,14 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     auto next = [&](Cursor& c) {
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
+    uint32_t bad = 0;
     auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWRegs]) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
-        va[j] = (c.valid && row < c.row_end)
-                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
-                    : 0.0f;
+        const bool ok = c.valid && row < c.row_end;
+        va[j] = ok ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb) : 0.0f;
+        if (ok && p.check_pow2) bad |= not_pow2(va[j]);
       }
       if (BROW) {
         // K-block-major tables (sa [kbn][M], sw [kbn][N]): lanes read
@@ -572,9 +584,10 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         }
       } else {
         const int nb = c.nb0 + lane;
-        vw[0] = (c.valid && lane < kNbPerTile && nb < p.nbn)
-                    ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
-                    : 0.0f;
+        const bool ok = c.valid && lane < kNbPerTile && nb < p.nbn;
+        vw[0] = ok ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
+                   : 0.0f;
+        if (ok && p.check_pow2) bad |= not_pow2(vw[0]);
       }
     };
     float ra[kAhead][4], rw[kAhead][kWRegs];
@@ -615,7 +628,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
       }
     }
   scales_done:
-    __syncwarp();
+    if (__any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) report_error(6);
   }
   } else {
     if (C::kSplitRegs) reg_acquire<C::kEpiRegs>();

@@ -284,7 +284,10 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t *a, const flo
  * arguments, layouts, workspace and result as fp8bs_fp8_gemm, but every a_s
  * and w_s entry must be a positive normal power of two, which the tensor core
  * then applies itself (tcgen05.mma kind::mxf8f6f4.block_scale with ue8m0
- * scale factors, one FP32 accumulation over all of K).  A scale that is not
+ * scale factors, one FP32 accumulation over all of K).  Decode-sized M (up
+ * to 64 rows), where the weight stream decides the time, runs the
+ * per-K-block promotion kernel instead, which is faster there and gives a
+ * result within the same tolerance.  On either path a scale that is not
  * such a power of two is reported through the device error word
  * (FP8BS_ERR_SCALE) and makes the output meaningless.
  */

@@ -109,10 +109,21 @@ def test_grouped_ue8m0_expert_config_sampled():
         assert_gemm_close(y[torch.from_numpy(rows).cuda()], y_ref, bnd, "ue8m0 expert %d" % g)
 
 
-def test_gemm_ue8m0_reports_non_power_of_two_scales():
-    x, qa, sa, qw, sw = _case(128, 256, 256, seed=7)
-    sa = sa.copy()
-    sa[5, 1] *= np.float32(1.5)                      # no longer a power of two
-    fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw), scale_fmt="ue8m0")
+@pytest.mark.parametrize("M", [128, 8])
+def test_gemm_ue8m0_reports_non_power_of_two_scales(M):
+    """M = 128 runs the block-scaled MMA, decode-sized M = 8 the promotion
+    kernel; both check the scales' form (an activation scale, then a weight
+    scale, no longer a power of two)."""
+    x, qa, sa, qw, sw = _case(M, 256, 256, seed=7)
+    bad_a = sa.copy()
+    bad_a[5, 1] *= np.float32(1.5)                   # no longer a power of two
+    fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(bad_a), cuda_codes(qw), cuda_f32(sw), scale_fmt="ue8m0")
     assert fp8bs.device_error() == fp8bs.ERR_SCALE
     assert fp8bs.device_error() == 0                 # read-and-clear
+    bad_w = sw.copy()
+    bad_w[1, 0] = np.float32(3e-3)
+    fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(bad_w), scale_fmt="ue8m0")
+    assert fp8bs.device_error() == fp8bs.ERR_SCALE
+    # power-of-two scales raise nothing on either path
+    fp8bs.fp8_gemm(cuda_codes(qa), cuda_f32(sa), cuda_codes(qw), cuda_f32(sw), scale_fmt="ue8m0")
+    assert fp8bs.device_error() == 0
