@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(kAqtThreads)
   pdl_wait();
   __shared__ __align__(16) float red[16][128];
   __shared__ __align__(16) float scol[128];
+  __shared__ __align__(16) float rcol[128];   // RN(1 / scol)
   __shared__ __align__(16) uint2 smq[128 * 16];
   const int t = threadIdx.x;
   const int cg = t & 15, rg = t >> 4;
@@ -386,17 +387,21 @@ __global__ void __launch_bounds__(kAqtThreads)
       for (int i = 1; i < 16; ++i) amax = fmaxf(amax, red[i][t]);
       const float sc = block_scale(amax, UE8M0);
       scol[t] = sc;
+      rcol[t] = __frcp_rn(sc);
       if (col0 + t < C) st[(col0 + t) * nrb + tr] = sc;
     }
     __syncthreads();
     if (col_ok) {
       const float4 s_lo = *reinterpret_cast<const float4*>(&scol[8 * cg]);
       const float4 s_hi = *reinterpret_cast<const float4*>(&scol[8 * cg + 4]);
+      const float4 r_lo = *reinterpret_cast<const float4*>(&rcol[8 * cg]);
+      const float4 r_hi = *reinterpret_cast<const float4*>(&rcol[8 * cg + 4]);
       const float sc8[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
+      const float r8[8] = {r_lo.x, r_lo.y, r_lo.z, r_lo.w, r_hi.x, r_hi.y, r_hi.z, r_hi.w};
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const float sc = sc8[c];
-        const float r = __frcp_rn(sc);
+        const float r = r8[c];
         float col[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
