@@ -59,10 +59,10 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G, int AR = 128, bool BROW = false>
+template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false>
 fp8bs_status setup_gemm_kernel() {
   using C = gemm::Cfg<BN, AR>;
-  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR, BROW>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -123,6 +123,10 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_bs_kernel<128, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<128, false, 128, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 16, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 16, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 64, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 64, false, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, false, 128, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, false, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, false, true>()) != FP8BS_OK)
@@ -417,12 +421,12 @@ size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
   return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
 }
 
-template <int BN, bool G, int AR = 128, bool BROW = false>
+template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                         const gemm::Params& p, int grid, cudaStream_t st) {
   using C = gemm::Cfg<BN, AR>;
-  return launch(gemm::fp8_gemm_kernel<BN, G, AR, BROW>, grid, C::kThreads, C::smem_bytes(G), st,
-                ta, tw, ty, p);
+  return launch(gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK>, grid, C::kThreads,
+                C::smem_bytes(G), st, ta, tw, ty, p);
 }
 
 // Rows of A one pipeline stage loads: all 128 rows of a tile, or for
@@ -502,7 +506,6 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.y = reinterpret_cast<__nv_bfloat16*>(y);
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
-  p.check_pow2 = check_pow2 ? 1 : 0;
   p.m_offsets = nullptr;
   p.M = M;
   p.N = static_cast<int>(N);
@@ -520,10 +523,20 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.tail_kbps = pl.tail_kbps;
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   p.groups = 1;
-  cudaError_t e =
-      !w_rowwise ? launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st)
-      : pl.bn == 256 ? launch_gemm<256, false, 128, true>(ta, tw, ty, p, pl.grid, st)
+  cudaError_t e;
+  if (w_rowwise)
+    e = pl.bn == 256 ? launch_gemm<256, false, 128, true>(ta, tw, ty, p, pl.grid, st)
                      : launch_gemm<128, false, 128, true>(ta, tw, ty, p, pl.grid, st);
+  else if (check_pow2 && (a_rows == 16 || a_rows == 64))
+    e = a_rows == 16
+            ? (pl.bn == 256 ? launch_gemm<256, false, 16, false, true>(ta, tw, ty, p, pl.grid, st)
+                            : launch_gemm<128, false, 16, false, true>(ta, tw, ty, p, pl.grid, st))
+            : (pl.bn == 256 ? launch_gemm<256, false, 64, false, true>(ta, tw, ty, p, pl.grid, st)
+                            : launch_gemm<128, false, 64, false, true>(ta, tw, ty, p, pl.grid, st));
+  else if (check_pow2)
+    return fail(FP8BS_ERR_UNSUPPORTED, "scale check without decode tiles (M=%lld)", (long long)M);
+  else
+    e = launch_gemm_any<false>(pl.bn, a_rows, ta, tw, ty, p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm launch");
   if (pl.tail_splits > 0) {
     const int64_t items = static_cast<int64_t>(pl.tail_tiles) * 128 * (pl.bn / 4);

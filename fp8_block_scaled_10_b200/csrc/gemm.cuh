@@ -101,10 +101,6 @@ struct Params {
   // split: ws = y, y_tma 2 maps y as a single split; several: the reduction
   // writes FP32).  p.y is unused then.
   int out_f32;
-  // The caller promised power-of-two scales (a *_ue8m0 entry routed to this
-  // kernel): the scale producer checks every scale it loads and reports one
-  // that is not a positive normal power of two (device error 6).
-  int check_pow2;
 };
 
 // Nonzero unless v is a positive normal power of two.
@@ -362,7 +358,12 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
 // epilogue multiplies a_s[row] by each column's scale before its FMA, and
 // since those reads outlast the TMEM buffer's release, the slot has its own
 // release barrier (sempty) that the producer waits on instead of tempty.
-template <int BN, bool GROUPED, int ARows = 128, bool BROW = false>
+// CHECK: the caller promised power-of-two scales (a *_ue8m0 entry routed to
+// this kernel, at decode-sized M): the scale producer checks every scale it
+// writes out and reports one that is not a positive normal power of two
+// (device error 6).  A compile-time switch: the check's code measurably slows
+// the scale producer of the kernels that do not need it.
+template <int BN, bool GROUPED, int ARows = 128, bool BROW = false, bool CHECK = false>
 __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w,
@@ -565,14 +566,17 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     auto next = [&](Cursor& c) {
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
+    // The power-of-two check runs when a step's values are written out, not
+    // here: testing a value where its load is issued would wait for the load
+    // and undo the prefetch.
     uint32_t bad = 0;
     auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWRegs]) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t row = c.row0 + lane + 32 * j;
-        const bool ok = c.valid && row < c.row_end;
-        va[j] = ok ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb) : 0.0f;
-        if (ok && p.check_pow2) bad |= not_pow2(va[j]);
+        va[j] = (c.valid && row < c.row_end)
+                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
+                    : 0.0f;
       }
       if (BROW) {
         // K-block-major tables (sa [kbn][M], sw [kbn][N]): lanes read
@@ -584,10 +588,9 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         }
       } else {
         const int nb = c.nb0 + lane;
-        const bool ok = c.valid && lane < kNbPerTile && nb < p.nbn;
-        vw[0] = ok ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
-                   : 0.0f;
-        if (ok && p.check_pow2) bad |= not_pow2(vw[0]);
+        vw[0] = (c.valid && lane < kNbPerTile && nb < p.nbn)
+                    ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
+                    : 0.0f;
       }
     };
     float ra[kAhead][4], rw[kAhead][kWRegs];
@@ -616,6 +619,12 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         } else if (lane < kNbPerTile) {
           dst[BM + lane] = rw[ph][0];
         }
+        if (CHECK && !BROW) {   // (the row-scaled entry sends ue8m0 elsewhere)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (cur.row0 + lane + 32 * j < cur.row_end) bad |= not_pow2(ra[ph][j]);
+          if (lane < kNbPerTile && cur.nb0 + lane < p.nbn) bad |= not_pow2(rw[ph][0]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&tfull[slot]);
         load(ahead, ra[ph], rw[ph]);
@@ -628,7 +637,8 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
       }
     }
   scales_done:
-    if (__any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) report_error(6);
+    if (CHECK && __any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) report_error(6);
+    __syncwarp();
   }
   } else {
     if (C::kSplitRegs) reg_acquire<C::kEpiRegs>();
