@@ -359,10 +359,12 @@ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_pr
 // since those reads outlast the TMEM buffer's release, the slot has its own
 // release barrier (sempty) that the producer waits on instead of tempty.
 // CHECK: the caller promised power-of-two scales (a *_ue8m0 entry routed to
-// this kernel, at decode-sized M): the scale producer checks every scale it
-// writes out and reports one that is not a positive normal power of two
-// (device error 6).  A compile-time switch: the check's code measurably slows
-// the scale producer of the kernels that do not need it.
+// this kernel, at decode-sized M): the first epilogue warp, before its first
+// wait, reads the scales the CTA's units use and reports one that is not a
+// positive normal power of two (device error 6).  Checked in the scale
+// producer, the values slowed decode by ~5 us; in the TMA warp's spare lanes
+// the divergent check ran ahead of the first TMA issue.  A compile-time
+// switch, so the other instantiations carry none of it.
 template <int BN, bool GROUPED, int ARows = 128, bool BROW = false, bool CHECK = false>
 __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -566,10 +568,6 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     auto next = [&](Cursor& c) {
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
-    // The power-of-two check runs when a step's values are written out, not
-    // here: testing a value where its load is issued would wait for the load
-    // and undo the prefetch.
-    uint32_t bad = 0;
     auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWRegs]) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -619,12 +617,6 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         } else if (lane < kNbPerTile) {
           dst[BM + lane] = rw[ph][0];
         }
-        if (CHECK && !BROW) {   // (the row-scaled entry sends ue8m0 elsewhere)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (cur.row0 + lane + 32 * j < cur.row_end) bad |= not_pow2(ra[ph][j]);
-          if (lane < kNbPerTile && cur.nb0 + lane < p.nbn) bad |= not_pow2(rw[ph][0]);
-        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&tfull[slot]);
         load(ahead, ra[ph], rw[ph]);
@@ -637,7 +629,6 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
       }
     }
   scales_done:
-    if (CHECK && __any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) report_error(6);
     __syncwarp();
   }
   } else {
@@ -650,6 +641,42 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     constexpr int NCH = C::kChunks;
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    if (CHECK && !GROUPED && e == 0) {
+      // Before its first wait, which at decode-sized M comes microseconds
+      // before the first partial: a_s [M, kbn] (small there) is shared out
+      // over the CTAs, and each CTA checks the w_s blocks of its own units,
+      // four independent loads per lane in flight at a time.
+      uint32_t bad = 0;
+      const int64_t na = p.M * p.kbn;
+      const int64_t step_a = static_cast<int64_t>(gridDim.x) * 32;
+      for (int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane; i < na; i += 4 * step_a) {
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = i + j * step_a < na ? __ldg(p.sa + i + j * step_a) : 1.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bad |= not_pow2(v[j]);
+      }
+      for (int u = unit_start; u < num_units; u += unit_step) {
+        const Unit t = unit_of(u);
+        const int nb0 = (t.n_tile * BN) / 128;
+        const int nkb = t.kb1 - t.kb0;
+        const int cnt = C::kNbSpan * nkb;
+        for (int i = lane; i < cnt; i += 4 * 32) {
+          float v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int el = i + 32 * j;
+            const int nb = nb0 + el / nkb;
+            v[j] = (el < cnt && nb < p.nbn)
+                       ? __ldg(p.sw + static_cast<int64_t>(nb) * p.kbn + t.kb0 + el % nkb)
+                       : 1.0f;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) bad |= not_pow2(v[j]);
+        }
+      }
+      if (__any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) report_error(6);
+    }
     const bool vec_store = (p.N % 8) == 0;
     int tb = 0;
     uint32_t tphase = 0;
