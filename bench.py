@@ -418,7 +418,17 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
             "fused_us": ms_q * 1e3, "fused_TFLOP/s": fl / ms_q / 1e9,
             "gemm_then_act_quant_us": ms_s * 1e3,
             "note": "fp8bs_fp8_gemm_quant vs fp8bs_fp8_gemm + fp8bs_act_quant of the bf16 y"}
-    del lin, q_out, s_out
+    # FP32 output (the unrounded accumulator), same shape
+    y32 = torch.empty(mm, nn, dtype=torch.float32, device="cuda")
+    f = lambda: L.fp8bs_fp8_gemm_f32(vp(lin.q), vp(lin.s), vp(lin.qw), vp(lin.sw), mm, nn, kk, 0,
+                                     vp(y32), vp(lin.ws), lin.nws, stream)
+    for _ in range(3):
+        f()
+    ms = time_events(f, 10)
+    parts["prefill_K7168_N18432_fp32_output"] = {
+        "gemm_us": ms * 1e3, "gemm_TFLOP/s": fl / ms / 1e9, "gemm_frac_fp8": fl / ms / 1e9 / fp8_peak,
+        "note": "fp8bs_fp8_gemm_f32, scale_fmt None"}
+    del lin, q_out, s_out, y32
     parts.update(run_expert_parts(fp8bs, wl, fp8_peak, stream))
     parts.update(run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush))
     return parts
