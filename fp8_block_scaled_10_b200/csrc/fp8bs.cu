@@ -450,6 +450,13 @@ cudaError_t launch_gemm_any(int bn, int a_rows, const CUtensorMap& ta, const CUt
                      : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
 }
 
+// Work units and tile indices are 32-bit in the kernels: the number of
+// 128 x 128 output tiles (the most any plan has before a K split, which the
+// planner caps at 16) must stay below 2^26.
+bool gemm_too_large(int64_t M, int64_t N) {
+  return ((M + 127) / 128) * ((N + 127) / 128) >= (int64_t(1) << 26);
+}
+
 fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8_t* w,
                                  const float* w_s, const void* y, int64_t N, int64_t K) {
   if (!a || !a_s || !w || !w_s || !y) return fail(FP8BS_ERR_INVALID_ARG, "null operand pointer");
@@ -469,6 +476,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (gemm_too_large(M, N)) return fail(FP8BS_ERR_INVALID_ARG, "M x N too large (tile count)");
   if (M == 0) return FP8BS_OK;
   int dev;
   DeviceInfo* info;
@@ -580,6 +588,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (gemm_too_large(M, N)) return fail(FP8BS_ERR_INVALID_ARG, "M x N too large (tile count)");
   if (M == 0) return FP8BS_OK;
   int dev;
   DeviceInfo* info;
@@ -1233,6 +1242,8 @@ fp8bs_status fp8bs_fp8_gemm_grouped_ue8m0(int64_t G, const int64_t* m_offsets, i
   p.num_units = 0;
   p.groups = static_cast<int>(G);
   const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
+  if (max_units >= (int64_t(1) << 26))
+    return fail(FP8BS_ERR_INVALID_ARG, "M_total x N too large (tile count)");
   const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
   cudaError_t e = bn == 256 ? launch_gemm_bs<256, true>(ta, tw, ty, p, grid, as_stream(stream))
                             : launch_gemm_bs<128, true>(ta, tw, ty, p, grid, as_stream(stream));
@@ -1298,6 +1309,8 @@ fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t
   p.groups = static_cast<int>(G);
   // Units are only known on the device; an upper bound sizes the grid.
   const int64_t max_units = ((M_total + 127) / 128 + G) * p.n_tiles;
+  if (max_units >= (int64_t(1) << 26))
+    return fail(FP8BS_ERR_INVALID_ARG, "M_total x N too large (tile count)");
   const int grid = static_cast<int>(std::min<int64_t>(max_units, info->sms));
   cudaError_t e = launch_gemm_any<true>(bn, 128, ta, tw, ty, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_grouped launch");
@@ -1323,6 +1336,7 @@ fp8bs_status fp8bs_fp8_gemm_quant(const uint8_t* a, const float* a_s, const uint
     return fail(FP8BS_ERR_INVALID_ARG, "s_out must be a 4-byte aligned device pointer");
   if (y != nullptr && !aligned16(y)) return fail(FP8BS_ERR_INVALID_ARG, "y must be 16-byte aligned");
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (gemm_too_large(M, N)) return fail(FP8BS_ERR_INVALID_ARG, "M x N too large (tile count)");
   if (M == 0) return FP8BS_OK;
   int dev;
   DeviceInfo* info;

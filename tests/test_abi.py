@@ -97,6 +97,9 @@ def test_host_side_argument_errors_without_gpu(L):
     assert L.fp8bs_act_dequant(dummy, dummy, 1, 4, 256, 128, dummy, 0, None) == fp8bs.ERR_INVALID_ARG
     assert L.fp8bs_act_dequant(dummy, dummy, 0, 4, 256, 128, dummy, 7, None) == fp8bs.ERR_INVALID_ARG
     assert L.fp8bs_act_dequant(dummy, dummy, 0, 4, 256, 512, dummy, 0, None) == fp8bs.ERR_UNSUPPORTED
+    # a tile count past the kernels' 32-bit unit indices is refused
+    st = L.fp8bs_fp8_gemm(dummy, dummy, dummy, dummy, 1 << 31, 1 << 30, 128, dummy, None, 0, None)
+    assert st == fp8bs.ERR_INVALID_ARG and b"too large" in L.fp8bs_last_error_message()
     # empty problems are successful no-ops
     assert L.fp8bs_act_quant_static(None, 0, 0, 256, 128, None, 0, None, None, None) == fp8bs.OK
     assert L.fp8bs_act_dequant(None, None, 2, 0, 256, 128, None, 0, None) == fp8bs.OK
