@@ -131,6 +131,11 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_bs_kernel<128, false, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<256, false, true>()) != FP8BS_OK)
       return r;
+    for (auto k : {act_quant_transposed_tma_kernel<false>, act_quant_transposed_tma_kernel<true>}) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               2 * kAqtStageBytes + 1024);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (act_quant_transposed)");
+    }
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -907,21 +912,31 @@ fp8bs_status fp8bs_act_quant_transposed(const void* x, fp8bs_dtype x_dtype, int6
   fp8bs_status r = device_setup(&dev, &info);
   if (r != FP8BS_OK) return r;
   const int64_t tiles = (rows / 128) * ((cols + 127) / 128);
-  const int per_sm =
-      x_dtype == FP8BS_DTYPE_BF16
-          ? resident_ctas(act_quant_transposed_bf16_kernel<false, kAqtPrefetch>, kAqtThreads, 0)
-          : resident_ctas(act_quant_transposed_kernel<float, false>, kAqtThreads, 0);
-  const int grid = grid_for(tiles, 1, info->sms * per_sm);
   cudaStream_t stm = as_stream(stream);
   const bool ue = fmt == FP8BS_SCALE_FMT_UE8M0;
   cudaError_t e;
   if (x_dtype == FP8BS_DTYPE_BF16) {
-    const auto* xb = static_cast<const __nv_bfloat16*>(x);
-    e = ue ? launch(act_quant_transposed_bf16_kernel<true, kAqtPrefetch>, grid, kAqtThreads, 0,
-                    stm, xb, qt, st, rows, cols)
-           : launch(act_quant_transposed_bf16_kernel<false, kAqtPrefetch>, grid, kAqtThreads, 0,
-                    stm, xb, qt, st, rows, cols);
+    // TMA-fed kernel: 128 x 128 bf16 boxes of x (columns past cols read as 0)
+    CUtensorMap tx;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+    const cuuint32_t box[2] = {128u, 128u};
+    const cuuint32_t elem[2] = {1u, 1u};
+    const CUresult cr = g_encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x),
+                                 dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (x) failed (%d)", (int)cr);
+    const size_t smem = 2 * kAqtStageBytes + 1024;
+    const int per_sm = resident_ctas(act_quant_transposed_tma_kernel<false>, kAqtThreads, smem);
+    const int grid = grid_for(tiles, 1, info->sms * per_sm);
+    e = ue ? launch(act_quant_transposed_tma_kernel<true>, grid, kAqtThreads, smem, stm, tx, qt,
+                    st, rows, cols)
+           : launch(act_quant_transposed_tma_kernel<false>, grid, kAqtThreads, smem, stm, tx, qt,
+                    st, rows, cols);
   } else {
+    const int per_sm = resident_ctas(act_quant_transposed_kernel<float, false>, kAqtThreads, 0);
+    const int grid = grid_for(tiles, 1, info->sms * per_sm);
     const auto* xf = static_cast<const float*>(x);
     e = ue ? launch(act_quant_transposed_kernel<float, true>, grid, kAqtThreads, 0, stm, xf, qt,
                     st, rows, cols)
