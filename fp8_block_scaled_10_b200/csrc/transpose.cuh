@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// act_quant in 128 x 1 column blocks, written transposed: for x [R, C]
+// act_quant in 128 x 1 column blocks, written transposed (fp32 input; bf16
+// input has the TMA-fed kernel below): for x [R, C]
 // (R % 128 == 0, C % 8 == 0), qT [C, R] and sT [C, R / 128] are act_quant of
 // x^T.  One 128 x 128 tile per step: thread t owns the 8 x 8 block of rows
 // 8 (t / 16).. and columns 8 (t % 16)..; per column, the amax of its 8 rows
@@ -241,45 +242,20 @@ __global__ void __launch_bounds__(kAqtThreads)
   const int cg = t & 15, rg = t >> 4;
   const int64_t nrb = R / 128, tiles_c = (C + 127) / 128;
   const int64_t ntiles = nrb * tiles_c;
-  // (bf16 input takes act_quant_transposed_bf16_kernel; this path prefetches
-  // only if instantiated for a 2-byte type.)
-  constexpr bool kPrefetch = sizeof(T) == 2;
-  uint4 pre[kPrefetch ? 8 : 1];
-  auto load_raw = [&](int64_t tile) {
-    const int64_t gc = (tile % tiles_c) * 128 + 8 * cg;
-    const int64_t row0 = (tile / tiles_c) * 128;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      pre[k] = gc < C ? __ldcs(reinterpret_cast<const uint4*>(x + (row0 + 8 * rg + k) * C + gc))
-                      : make_uint4(0u, 0u, 0u, 0u);
-  };
-  if (kPrefetch && static_cast<int64_t>(blockIdx.x) < ntiles) load_raw(blockIdx.x);
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t tr = tile / tiles_c;
-    const int64_t row0 = tr * 128, col0 = (tile % tiles_c) * 128;
+    int64_t tr, tc;
+    tile_coords(tile, nrb, tiles_c, tr, tc);
+    const int64_t row0 = tr * 128, col0 = tc * 128;
     const int64_t gc = col0 + 8 * cg;
     const bool col_ok = gc < C;
     float v[8][8];
-    if constexpr (kPrefetch) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t w[4] = {pre[k].x, pre[k].y, pre[k].z, pre[k].w};
+    for (int k = 0; k < 8; ++k) {
+      if (col_ok) {
+        load8(x + (row0 + 8 * rg + k) * C + gc, v[k]);
+      } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[k][2 * j] = __uint_as_float(w[j] << 16);
-          v[k][2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-      }
-      if (tile + gridDim.x < ntiles) load_raw(tile + gridDim.x);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (col_ok) {
-          load8(x + (row0 + 8 * rg + k) * C + gc, v[k]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) v[k][c] = 0.0f;
-        }
+        for (int c = 0; c < 8; ++c) v[k][c] = 0.0f;
       }
     }
     float pm[8];
