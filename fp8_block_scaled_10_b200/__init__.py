@@ -339,8 +339,9 @@ def fp8_gemm(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.bfloat16):
     a: [..., K] e4m3fn, a_s: [..., K/128] float32, b: [N, K] e4m3fn,
     b_s: [cdiv(N,128), K/128] float32 -> y: [..., N] of out_dtype
     (torch.bfloat16, or torch.float32 for the unrounded FP32 accumulator).
-    scale_fmt="ue8m0" promises that every scale is a power of two and uses
-    the tensor core's block-scaled MMA."""
+    scale_fmt="ue8m0" promises that every scale is a power of two: the tensor
+    core's block-scaled MMA applies them (at decode-sized M, up to 64 rows, the
+    promotion kernel runs instead, with a check of the scales)."""
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
     a, b = _codes(a), _codes(b)
@@ -389,7 +390,8 @@ def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,
 
     x: [..., K] bfloat16, weight: [N, K] e4m3fn, weight_scale: [cdiv(N,128), K/128].
     With scale_fmt="ue8m0" and weight_scale_fmt="ue8m0" (power-of-two weight
-    scales) the GEMM runs on the block-scaled MMA."""
+    scales) the GEMM is the ue8m0 entry (block-scaled MMA; promotion kernel at
+    decode-sized M)."""
     w = _codes(weight)
     _need_cuda(x, w, weight_scale)
     if x.dtype != torch.bfloat16:
