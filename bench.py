@@ -60,8 +60,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the per-workload parts")
-    ap.add_argument("--parts", choices=["all", "training", "experts"], default="all",
-                    help="which per-workload parts to run: all, only the training GEMMs, or only the grouped expert GEMMs")
+    ap.add_argument("--parts", choices=["all", "memory", "decode", "training", "experts"],
+                    default="all",
+                    help="which per-workload parts to run: all, or only one group (memory-bound "
+                         "quantizers and dequant, decode GEMMs, training GEMMs, grouped experts)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -276,6 +278,8 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
         return run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush)
     if which == "experts":
         return run_expert_parts(fp8bs, wl, fp8_peak, stream)
+    if which == "decode":
+        return run_gemm_parts(fp8bs, wl, hbm, fp8_peak, stream, flush, parts, which)
 
     # act_quant, x bf16 [16384, 7168] with 0.1% entries x100
     R, C = 16384, 7168
@@ -352,6 +356,14 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
     parts["weight_quant_f32"] = {"shape": [R, C], "us": ms * 1e3, "GB/s": nb / ms / 1e6,
                                  "frac_hbm": nb / ms / 1e6 / hbm, "bytes": nb}
     del wf, qo, so
+    if which == "memory":
+        return parts
+    return run_gemm_parts(fp8bs, wl, hbm, fp8_peak, stream, flush, parts, which)
+
+
+def run_gemm_parts(fp8bs, wl, hbm, fp8_peak, stream, flush, parts, which):
+    """The GEMM parts: decode, prefill, FP8/FP32 output, experts, training."""
+    L = fp8bs.lib()
     # decode GEMMs (ue8m0 scales), bytes = W + w_s + A + a_s + y
     for kk, nn in wl.DECODE_KN:
         lin = None
@@ -372,6 +384,8 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
                                if mm <= 64 else "fp8bs_fp8_gemm_ue8m0: block-scaled MMA")
                               if tag else "fp8bs_fp8_gemm: promotion"}
         del lin
+    if which == "decode":
+        return parts
     # prefill shapes: fused act_quant + GEMM per call, and the GEMM alone
     for kk, nn in wl.PREFILL_KN:
         for fmt in (0, 1):
