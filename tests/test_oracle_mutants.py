@@ -1,0 +1,116 @@
+"""Planted mistakes: each test takes an oracle result, plants a plausible slip
+in it (on the CPU, in numpy), and checks that the reference comparison the
+corresponding pin in test_oracle_pins.py relies on rejects the slipped
+result while accepting the oracle's own.  This shows that the pins of the
+static scheme, the transposing quantizer, the FP8 transpose and the
+row-scaled GEMM discriminate the slips they are meant to catch."""
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+
+BLOCK = 128
+
+
+def _bf16(x):
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _torch_codes(y):
+    return y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_static_scale_indexed_by_row_is_caught():
+    """The static scale of element (r, c) is s[c // block]; a slip that reads
+    s[r % nblk] instead is rejected by the x = 1, s[b] = 2^-b check."""
+    rows, nblk = 5, 7
+    x = np.ones((rows, nblk * BLOCK), np.float32)
+    s = np.exp2(-np.arange(nblk, dtype=np.float32)).astype(np.float32)
+    want = np.broadcast_to(np.repeat(_torch_codes(torch.from_numpy(1.0 / s)), BLOCK),
+                           (rows, nblk * BLOCK))
+    good = oracle.act_quant_static(x, s)
+    assert np.array_equal(good, want)
+    slip = np.stack([oracle.act_quant_static(x[r:r + 1], np.full(nblk, s[r % nblk], np.float32))[0]
+                     for r in range(rows)])
+    assert not np.array_equal(slip, want)
+
+
+def test_static_dequant_without_scale_is_caught():
+    """static_dequant multiplies by the block's scale; dropping it (or
+    dividing) fails the page-formula comparison."""
+    g = torch.Generator().manual_seed(3)
+    codes = torch.randint(0, 254, (4, 2 * BLOCK), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8)
+    s = torch.tensor([0.25, 3.0], dtype=torch.float32)
+    ref = (codes.view(torch.float8_e4m3fn).float().reshape(4, 2, BLOCK) * s.unsqueeze(-1)).reshape(4, -1)
+    good = oracle.act_dequant(codes.numpy(), s.numpy(), out="f32")
+    assert np.array_equal(good, ref.numpy())
+    for slip in (good / np.repeat(s.numpy(), BLOCK) ** 2, codes.view(torch.float8_e4m3fn).float().numpy()):
+        assert not np.array_equal(slip.astype(np.float32), ref.numpy())
+
+
+def test_transposed_quantizer_with_row_blocks_is_caught():
+    """act_quant_transposed takes 128 x 1 column blocks; transposing the codes
+    of ordinary 1 x 128 row blocks instead fails the column-block comparison."""
+    g = torch.Generator().manual_seed(5)
+    R, C = 2 * BLOCK, 2 * BLOCK
+    x = torch.randn(R, C, generator=g) * 3
+    x[torch.rand(x.shape, generator=g) < 0.02] *= 40
+    arr = _bf16(x)
+    xf = torch.from_numpy(oracle.bf16_bits_to_f32(arr).copy())
+    amax = xf.abs().reshape(R // BLOCK, BLOCK, C).amax(dim=1)
+    s = (torch.clamp(amax, min=float(np.float32(1e-4))) / torch.tensor(448.0)).numpy()
+    want = _torch_codes(xf / torch.from_numpy(s).repeat_interleave(BLOCK, dim=0)).T
+    good, _ = oracle.act_quant_transposed(arr)
+    assert np.array_equal(good, want)
+    slip = oracle.act_quant(arr)[0].T
+    assert not np.array_equal(slip, want)
+
+
+def test_fp8_transpose_without_scale_transpose_is_caught():
+    """Transposing the codes with a scale grid of the right shape but its
+    blocks in the wrong places fails the dequant-commutes check."""
+    g = torch.Generator().manual_seed(7)
+    codes = torch.randint(0, 254, (300, 200), generator=g)
+    codes = (codes + (codes >= 0x7F).long()).to(torch.uint8).numpy()
+    s = (torch.rand(3, 2, generator=g) + 0.01).numpy().astype(np.float32)
+    y = oracle.weight_dequant(codes, s, out="f32")
+    qt, st = oracle.fp8_transpose(codes, s)
+    assert np.array_equal(oracle.weight_dequant(qt, st, out="f32"), y.T)
+    flipped = np.ascontiguousarray(s[::-1, ::-1].T)   # right shape, wrong blocks
+    assert not np.array_equal(oracle.weight_dequant(qt, flipped, out="f32"), y.T)
+
+
+def test_row_scaled_gemm_with_block_scales_is_caught():
+    """The row-scaled GEMM takes b_s[n, kb]; reading the scale of n's
+    128-row block instead (b_s[n // 128 * 128, kb]) breaks exact arithmetic."""
+    g = torch.Generator().manual_seed(9)
+    M, N, K = 2, 130, 256
+    qa = (torch.randint(0, 126, (M, K), generator=g)).to(torch.uint8).numpy()
+    qb = (torch.randint(0, 126, (N, K), generator=g)).to(torch.uint8).numpy()
+    sa = (torch.rand(M, K // 128, generator=g) + 0.5).numpy().astype(np.float32)
+    sb = (torch.rand(N, K // 128, generator=g) + 0.5).numpy().astype(np.float32)
+    y, _ = oracle.gemm(qa, sa, qb, sb, w_scales="row")
+    table = oracle.e4m3_table()
+
+    def exact(scales_for_row):
+        out = np.zeros((M, N), dtype=object)
+        for m in range(M):
+            for n in range(N):
+                acc = Fraction(0)
+                for kb in range(K // 128):
+                    sl = slice(kb * 128, (kb + 1) * 128)
+                    p = sum(Fraction(float(a)) * Fraction(float(b))
+                            for a, b in zip(table[qa[m, sl]], table[qb[n, sl]]))
+                    acc += Fraction(float(sa[m, kb])) * Fraction(float(scales_for_row(n)[kb])) * p
+                out[m, n] = acc
+        return out
+
+    ex = exact(lambda n: sb[n])
+    assert all(abs(Fraction(float(y[m, n])) - ex[m, n]) <= abs(ex[m, n]) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+               for m in range(M) for n in range(N))
+    slip = exact(lambda n: sb[(n // 128) * 128])
+    assert any(abs(Fraction(float(y[m, n])) - slip[m, n]) > abs(slip[m, n]) * Fraction(1, 2 ** 20)
+               for m in range(M) for n in range(N))
