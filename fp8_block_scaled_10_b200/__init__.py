@@ -144,6 +144,43 @@ def _scale_fmt(scale_fmt):
     raise ValueError("scale_fmt must be None or 'ue8m0'")
 
 
+def _io_dtype(dtype, what):
+    """DTYPE_BF16 / DTYPE_F32 for a bfloat16 / float32 tensor dtype."""
+    if dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError("%s must be torch.bfloat16 or torch.float32, got %s" % (what, dtype))
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def _scales_like(s, shape, what):
+    """Raise unless s is a float32 tensor of exactly ``shape``: the kernels read
+    scales through raw pointers, so a short table would be read past its end."""
+    if s.dtype != torch.float32:
+        raise TypeError("%s must be float32, got %s" % (what, s.dtype))
+    if tuple(s.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (what, tuple(shape), tuple(s.shape)))
+
+
+def _gemm_operands(a, a_s, b, b_s):
+    """Shape checks of fp8_gemm's operands -> (M, N, K)."""
+    if b.dim() != 2:
+        raise ValueError("b must be 2-D [N, K]")
+    K = a.shape[-1]
+    if b.shape[1] != K:
+        raise ValueError("a [..., K] and b [N, K] disagree on K (%d vs %d)" % (K, b.shape[1]))
+    if K <= 0 or K % 128 != 0:
+        raise ValueError("K=%d must be a positive multiple of 128" % K)
+    N = b.shape[0]
+    _scales_like(a_s, tuple(a.shape[:-1]) + (K // 128,), "a_s")
+    _scales_like(b_s, (_cdiv(N, 128), K // 128), "b_s")
+    return a.numel() // K, N, K
+
+
 def act_quant(x, block_size=128, scale_fmt=None):
     """Dynamic 1 x block_size quantization of the last dimension.
 
@@ -219,7 +256,7 @@ def act_dequant(q, s, block_size=128, out_dtype=torch.float32):
         raise ValueError("last dimension must be a multiple of block_size")
     stride = _act_scales(s, q.shape[:-1], cols, block_size)
     rows = q.numel() // cols if cols else 0
-    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[out_dtype]
+    dt = _io_dtype(out_dtype, "out_dtype")
     y = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     _check(lib().fp8bs_act_dequant(_ptr(q), _ptr(s), stride, rows, cols, block_size, _ptr(y), dt,
                                    _stream(q.device)))
@@ -239,7 +276,7 @@ def weight_dequant(x, s, block_size=128, out_dtype=torch.bfloat16):
     M, N = x.shape
     if tuple(s.shape) != (-(-M // block_size), -(-N // block_size)) or s.dtype != torch.float32:
         raise ValueError("s must be float32 of shape (cdiv(M, block), cdiv(N, block))")
-    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[out_dtype]
+    dt = _io_dtype(out_dtype, "out_dtype")
     y = torch.empty(M, N, dtype=out_dtype, device=x.device)
     _check(lib().fp8bs_weight_dequant(_ptr(x), _ptr(s), M, N, block_size, _ptr(y), dt,
                                       _stream(x.device)))
@@ -251,7 +288,7 @@ def weight_quant(w, block_size=128, scale_fmt=None):
     _need_cuda(w)
     if w.dim() != 2:
         raise ValueError("weight_quant expects a 2-D weight")
-    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[w.dtype]
+    dt = _io_dtype(w.dtype, "w")
     M, N = w.shape
     q = torch.empty(M, N, dtype=torch.float8_e4m3fn, device=w.device)
     s = torch.empty(-(-M // block_size), -(-N // block_size), dtype=torch.float32, device=w.device)
@@ -269,7 +306,7 @@ def act_quant_transposed(x, block_size=128, scale_fmt=None):
     _need_cuda(x)
     if x.dim() != 2:
         raise ValueError("act_quant_transposed expects a 2-D x")
-    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[x.dtype]
+    dt = _io_dtype(x.dtype, "x")
     rows, cols = x.shape
     q = torch.empty(cols, rows, dtype=torch.float8_e4m3fn, device=x.device)
     s = torch.empty(cols, rows // block_size, dtype=torch.float32, device=x.device)
@@ -301,11 +338,15 @@ def fp8_gemm_rowwise(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.float32):
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
     a, b = _codes(a), _codes(b)
-    _need_cuda(a, a_s, b, b_s)
+    if a.dim() != 2 or b.dim() != 2 or b.shape[1] != a.shape[1]:
+        raise ValueError("a [M,K], a_s [M,K/128], b [N,K], b_s [N,K/128] expected")
     M, K = a.shape
     N = b.shape[0]
-    if b.shape[1] != K or tuple(a_s.shape) != (M, K // 128) or tuple(b_s.shape) != (N, K // 128):
-        raise ValueError("a [M,K], a_s [M,K/128], b [N,K], b_s [N,K/128] expected")
+    if K <= 0 or K % 128 != 0:
+        raise ValueError("K=%d must be a positive multiple of 128" % K)
+    _scales_like(a_s, (M, K // 128), "a_s")
+    _scales_like(b_s, (N, K // 128), "b_s")
+    _need_cuda(a, a_s, b, b_s)
     y = torch.empty(M, N, dtype=out_dtype, device=a.device)
     nws = int(lib().fp8bs_gemm_rowwise_workspace_size(M, N, K))
     ws = torch.empty(nws, dtype=torch.uint8, device=a.device) if nws else None
@@ -345,13 +386,11 @@ def fp8_gemm(a, a_s, b, b_s, scale_fmt=None, out_dtype=torch.bfloat16):
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
     a, b = _codes(a), _codes(b)
+    M, N, K = _gemm_operands(a, a_s, b, b_s)
+    fmt = _scale_fmt(scale_fmt)
     _need_cuda(a, a_s, b, b_s)
-    K = a.shape[-1]
-    M = a.numel() // K if K else 0
-    N = b.shape[0]
     y = torch.empty(*a.shape[:-1], N, dtype=out_dtype, device=a.device)
     ws, nws = _workspace(M, N, K, a.device)
-    fmt = _scale_fmt(scale_fmt)
     if out_dtype == torch.float32:
         _check(lib().fp8bs_fp8_gemm_f32(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K, fmt,
                                         _ptr(y), _ptr(ws), nws, _stream(a.device)))
@@ -369,13 +408,12 @@ def fp8_gemm_quant(a, a_s, b, b_s, out_scale_fmt=None, return_y=False):
     Returns (q e4m3fn [..., N], s float32 [..., N/128]), plus the bf16 y when
     return_y.  N must be a multiple of 128."""
     a, b = _codes(a), _codes(b)
+    M, N, K = _gemm_operands(a, a_s, b, b_s)
+    if N % 128 != 0:
+        raise ValueError("N=%d must be a multiple of 128 for an FP8 output" % N)
     _need_cuda(a, a_s, b, b_s)
-    K = a.shape[-1]
-    M = a.numel() // K if K else 0
-    N = b.shape[0]
     q = torch.empty(*a.shape[:-1], N, dtype=torch.uint8, device=a.device)
-    s = torch.empty(*a.shape[:-1], N // 128 if N % 128 == 0 else 1, dtype=torch.float32,
-                    device=a.device)
+    s = torch.empty(*a.shape[:-1], N // 128, dtype=torch.float32, device=a.device)
     y = torch.empty(*a.shape[:-1], N, dtype=torch.bfloat16, device=a.device) if return_y else None
     _check(lib().fp8bs_fp8_gemm_quant(_ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), M, N, K,
                                       _scale_fmt(out_scale_fmt), _ptr(q), _ptr(s), _ptr(y),
@@ -393,12 +431,17 @@ def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,
     scales) the GEMM is the ue8m0 entry (block-scaled MMA; promotion kernel at
     decode-sized M)."""
     w = _codes(weight)
-    _need_cuda(x, w, weight_scale)
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bfloat16")
+    if w.dim() != 2 or w.shape[1] != x.shape[-1]:
+        raise ValueError("weight must be [N, K] with K = x.shape[-1]")
     K = x.shape[-1]
-    M = x.numel() // K if K else 0
+    if K <= 0 or K % 128 != 0:
+        raise ValueError("K=%d must be a positive multiple of 128" % K)
     N = w.shape[0]
+    _scales_like(weight_scale, (_cdiv(N, 128), K // 128), "weight_scale")
+    _need_cuda(x, w, weight_scale)
+    M = x.numel() // K
     y = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
     q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
     s = torch.empty(*x.shape[:-1], K // 128, dtype=torch.float32, device=x.device)
@@ -420,11 +463,19 @@ def fp8_gemm_grouped(a, a_s, w, w_s, m_offsets, scale_fmt=None):
     a: [M_total, K] e4m3fn, a_s: [M_total, K/128], w: [G, N, K] e4m3fn,
     w_s: [G, cdiv(N,128), K/128], m_offsets: [G+1] int64 on the device."""
     a, w = _codes(a), _codes(w)
-    _need_cuda(a, a_s, w, w_s, m_offsets)
     if m_offsets.dtype != torch.int64:
         raise TypeError("m_offsets must be int64")
+    if a.dim() != 2 or w.dim() != 3 or w.shape[2] != a.shape[1]:
+        raise ValueError("a [M_total, K] and w [G, N, K] expected")
     G, N, K = w.shape
     M = a.shape[0]
+    if K <= 0 or K % 128 != 0:
+        raise ValueError("K=%d must be a positive multiple of 128" % K)
+    if tuple(m_offsets.shape) != (G + 1,):
+        raise ValueError("m_offsets must have shape (G + 1,) = (%d,)" % (G + 1))
+    _scales_like(a_s, (M, K // 128), "a_s")
+    _scales_like(w_s, (G, _cdiv(N, 128), K // 128), "w_s")
+    _need_cuda(a, a_s, w, w_s, m_offsets)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
     fn = lib().fp8bs_fp8_gemm_grouped_ue8m0 if _scale_fmt(scale_fmt) else lib().fp8bs_fp8_gemm_grouped
     _check(fn(G, _ptr(m_offsets), M, _ptr(a), _ptr(a_s), _ptr(w), _ptr(w_s), N, K, _ptr(y),
