@@ -125,6 +125,9 @@ def _need_cuda(*ts):
             raise ValueError("fp8bs runs on CUDA tensors only (got a %s tensor)" % t.device)
         if not t.is_contiguous():
             raise ValueError("fp8bs expects contiguous tensors")
+        if t.device != ts[0].device:
+            raise ValueError("all operands must be on one device (%s and %s)"
+                             % (ts[0].device, t.device))
 
 
 def _codes(t):

@@ -110,3 +110,20 @@ def test_fp8_gemm_grouped_shapes():
 def test_dtype_errors_are_type_errors():
     with pytest.raises(TypeError, match="out_dtype"):
         fp8bs._io_dtype(torch.float16, "out_dtype")
+
+
+def test_operands_on_two_devices_are_refused():
+    """Operands on different GPUs are refused before the kernel could take a
+    peer pointer for a local one (checked with stand-in device objects)."""
+    class Fake:
+        is_cuda = True
+
+        def __init__(self, dev):
+            self.device = torch.device("cuda", dev)
+
+        def is_contiguous(self):
+            return True
+
+    fp8bs._need_cuda(Fake(0), Fake(0))
+    with pytest.raises(ValueError, match="one device"):
+        fp8bs._need_cuda(Fake(0), Fake(1))
