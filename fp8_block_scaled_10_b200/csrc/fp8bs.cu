@@ -1163,6 +1163,8 @@ fp8bs_status fp8bs_fp8_gemm_static_scratch(const uint8_t* a, const float* a_s, c
                        "scratch holds %zu bytes (use fp8bs_fp8_gemm with a workspace)",
                        (long long)M, (long long)N, (long long)K, need,
                        (size_t)FP8BS_STATIC_SCRATCH_BYTES);
+  // An empty problem is validated and returns before the scratch is looked up.
+  if (M == 0) return fp8bs_fp8_gemm(a, a_s, w, w_s, M, N, K, y, nullptr, 0, stream);
   void* scratch = nullptr;
   const fp8bs_status r = static_scratch_address(&scratch);
   if (r != FP8BS_OK) return r;

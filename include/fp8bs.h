@@ -264,9 +264,11 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm(const uint8_t *a, const float *a_s, const 
  * FP8BS_STATIC_SCRATCH_BYTES (fp8bs_gemm_workspace_size(M, N, K) is larger)
  * are rejected with FP8BS_ERR_WORKSPACE before anything is launched.
  *
- * The first call on a device looks up the scratch array's device address
- * (cudaGetSymbolAddress, once per device, on the current device); make that
- * first call before any stream capture.  All calls share the one array and
+ * An empty problem (M == 0) is validated like fp8bs_fp8_gemm and returns
+ * FP8BS_OK without touching the device.  The first call with M > 0 on a
+ * device looks up the scratch array's device address (cudaGetSymbolAddress,
+ * once per device, on the current device); make that first call before any
+ * stream capture.  All calls share the one array and
  * every call writes the partials it reads, so nothing needs clearing between
  * calls, but calls that overlap on the GPU (other streams, other threads)
  * race on the array: serialise them.

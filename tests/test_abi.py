@@ -116,3 +116,27 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         fp8bs.act_quant(torch.zeros(4, 128, dtype=torch.bfloat16))
+
+
+def test_every_entry_point_treats_an_empty_problem_as_a_no_op(L):
+    """Zero rows (or an empty matrix) return OK before any device work, so
+    these calls succeed on a host without a GPU."""
+    dummy = _p(4096)
+    OK = fp8bs.OK
+    assert L.fp8bs_weight_quant(None, 0, 0, 256, 128, 0, None, None, None) == OK
+    assert L.fp8bs_fp8_transpose(None, None, 0, 256, 128, None, None, None) == OK
+    assert L.fp8bs_fp8_transpose(None, None, 256, 0, 128, None, None, None) == OK
+    assert L.fp8bs_act_quant_transposed(None, 0, 0, 256, 128, 0, None, None, None) == OK
+    assert L.fp8bs_fp8_gemm_ue8m0(dummy, dummy, dummy, dummy, 0, 256, 128, dummy, None, 0,
+                                  None) == OK
+    assert L.fp8bs_fp8_gemm_static_scratch(dummy, dummy, dummy, dummy, 0, 256, 128, dummy,
+                                           None) == OK
+    for fmt in (0, 1):
+        assert L.fp8bs_fp8_gemm_rowwise(dummy, dummy, dummy, dummy, 0, 256, 128, fmt, dummy, 1,
+                                        None, 0, None) == OK
+    assert L.fp8bs_fp8_linear(None, 0, 256, 0, dummy, dummy, 128, dummy, dummy, dummy, None, 0,
+                              None) == OK
+    assert L.fp8bs_fp8_linear_ue8m0(None, 0, 256, dummy, dummy, 128, dummy, dummy, dummy, None, 0,
+                                    None) == OK
+    for fn in (L.fp8bs_fp8_gemm_grouped, L.fp8bs_fp8_gemm_grouped_ue8m0):
+        assert fn(4, dummy, 0, dummy, dummy, dummy, dummy, 256, 128, dummy, None) == OK
