@@ -339,6 +339,33 @@ def test_weight_quant_tiles_and_ragged_edges():
             assert np.array_equal(q[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128], ref)
 
 
+@pytest.mark.parametrize("block", [32, 64, 128, 256])
+def test_weight_quant_block_sizes_and_ue8m0_match_library_ops(block):
+    """Per block x block tile (ragged at the bottom and right edges): amax by
+    torch, the clamp and /448 in fp32, the ue8m0 round-up as an exact
+    power-of-two ceiling, then torch's division and torch's e4m3 cast."""
+    rows, cols = 2 * block + 9, 3 * block - 5
+    g = torch.Generator().manual_seed(300 + block)
+    w = torch.randn(rows, cols, generator=g) * 0.02
+    w[torch.rand(w.shape, generator=g) < 0.01] *= 30
+    w[block:2 * block, :block] = 0.0                      # an all-zero tile
+    rb, cb = -(-rows // block), -(-cols // block)
+    pad = torch.zeros(rb * block, cb * block)
+    pad[:rows, :cols] = w.abs()
+    amax = pad.reshape(rb, block, cb, block).amax(dim=(1, 3))
+    s_none = (torch.clamp(amax, min=float(f32(CLAMP))) / torch.tensor(448.0)).numpy()
+    for fmt in (None, "ue8m0"):
+        q, s = oracle.weight_quant(w.numpy(), block=block, scale_fmt=fmt)
+        sref = s_none.astype(np.float32)
+        if fmt == "ue8m0":
+            sref = np.array([_exact_pow2_ceil(v) for v in sref.ravel()],
+                            dtype=np.float32).reshape(sref.shape)
+        assert np.array_equal(s.view(np.uint32), sref.view(np.uint32)), fmt
+        st = torch.from_numpy(s).repeat_interleave(block, 0)[:rows].repeat_interleave(block, 1)[:, :cols]
+        ref = (w / st).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(q, ref), fmt
+
+
 # --------------------------------------------------------------------------
 # weight_dequant
 # --------------------------------------------------------------------------
