@@ -140,3 +140,24 @@ def test_every_entry_point_treats_an_empty_problem_as_a_no_op(L):
                                     None) == OK
     for fn in (L.fp8bs_fp8_gemm_grouped, L.fp8bs_fp8_gemm_grouped_ue8m0):
         assert fn(4, dummy, 0, dummy, dummy, dummy, dummy, 256, 128, dummy, None) == OK
+
+
+def test_plain_c_client_builds_and_runs(L, tmp_path):
+    """The header compiles as strict C99 and a C program links against the
+    library and gets the documented host-side results (no Python involved)."""
+    import os
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    libdir = os.path.dirname(fp8bs.LIB_PATH)
+    exe = str(tmp_path / "abi_c_client")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"), os.path.join(here, "abi_c_client.c"),
+                    "-L", libdir, "-lfp8bs", "-Wl,-rpath," + libdir, "-o", exe],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "abi c client ok"
