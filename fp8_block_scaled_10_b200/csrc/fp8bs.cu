@@ -1,7 +1,9 @@
 // C ABI of libfp8bs.so (declared in include/fp8bs.h): argument checks, launch
 // configuration, TMA descriptors and the per-device error word.  The kernels
 // live in quant.cuh (act_quant, weight_dequant, weight_quant, split-K
-// reduction) and gemm.cuh (block-scaled FP8 GEMM).
+// reduction), gemm.cuh (FP8 GEMM with FP32 promotion), gemm_bs.cuh (FP8 GEMM
+// on the block-scaled MMA) and transpose.cuh (FP8 transpose, transposing
+// quantizer); plan.h plans the dense GEMM launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -15,6 +17,7 @@
 #include "fp8bs.h"
 #include "gemm.cuh"
 #include "gemm_bs.cuh"
+#include "plan.h"
 #include "quant.cuh"
 #include "sm100.cuh"
 #include "transpose.cuh"
@@ -279,152 +282,6 @@ int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, max_ctas)));
 }
 
-// ---------------------------------------------------------------------------
-// GEMM planning: tile width BN and split-K factor.
-// ---------------------------------------------------------------------------
-struct Plan {
-  int bn;
-  int m_tiles, n_tiles;
-  int splits, kb_per_split;
-  int units;
-  int grid;   // persistent CTAs
-  // Split tail (see gemm::Params): 0 = none.
-  int full_units = 0, tail_tiles = 0, tail_splits = 0, tail_kbps = 0;
-  int n_group = 1;   // band width of the tile order (gemm::tile_mn)
-};
-
-// Band width of the dense tile order for one K split.  m fastest (width 1)
-// reads each W tile once and A once per n tile, from L2 when A fits there
-// beside the W tiles in flight (up to kAResidentBytes).  A larger A would
-// come from HBM once per n tile; a band of n tiles whose W fits in
-// kWBandBytes of L2 then reads A once per band instead.  (Measured on B200:
-// the weight-gradient shape M = 18432, N = 7168, K = 4096 read 1.7 GB per
-// launch m-fastest, against 0.64 GB of operands and output.)
-constexpr int64_t kAResidentBytes = 40ll << 20;
-constexpr int64_t kWBandBytes = 20ll << 20;
-int choose_n_group(int64_t M, int64_t K, int bn, int n_tiles) {
-  if (M * K <= kAResidentBytes) return 1;
-  const int64_t g = kWBandBytes / (static_cast<int64_t>(bn) * K);
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, n_tiles)));
-}
-
-// The split tail's FP32 partials are kept within this many bytes, so that
-// every prefill plan also fits the library's static scratch array.
-constexpr size_t kTailWorkspaceCap = FP8BS_STATIC_SCRATCH_BYTES;
-
-double wave_efficiency(int64_t units, int slots) {
-  const int64_t waves = (units + slots - 1) / slots;
-  return static_cast<double>(units) / static_cast<double>(waves * slots);
-}
-
-// The two GEMM kernels the planner serves.
-// kRowScaled: the promotion kernel with one scale per row of W (per column of
-// y) and K block, whose epilogue multiplies each column's scale in.
-enum class GemmKind { kPromotion, kBlockScaled, kRowScaled };
-
-// Time per K block of one 128-row work unit, in microseconds, measured on
-// B200 at M = 4096 with every SM busy.
-//   promotion kernel: 128 x 256 tile ~0.55, 128 x 192 ~0.48, 128 x 128
-//     ~0.36 (the tensor core and the epilogue's FP32 promotion overlap; the
-//     wider tile moves fewer operand bytes per FLOP);
-//   block-scaled kernel: 128 x 256 ~0.5, 128 x 128 ~1/3 (operand feed).
-double kb_time_us(GemmKind kind, int bn) {
-  if (kind == GemmKind::kPromotion) return bn == 256 ? 0.55 : (bn == 192 ? 0.48 : 0.36);
-  if (kind == GemmKind::kRowScaled) return bn == 256 ? 0.62 : 0.40;
-  return bn == 256 ? 0.5 : 1.0 / 3.0;
-}
-
-// Chooses tile width and K split.
-//
-// M > 128 (several 128-row tiles share each W tile): the estimated time is
-// waves of work units x K blocks per unit x kb_time_us, plus, for a K split,
-// the FP32 partials' round trip through HBM and the reduction launch.  When
-// the tiles fill the GPU but their last wave would keep at most half of the
-// SMs busy, the plan can split only the tiles of that wave along
-// K ("split tail", both kernels): the whole waves run unchanged and the
-// tail's partials, a few MB, are summed by a small reduction.
-//
-// M <= 128 (decode): the weight stream from HBM bounds every tile width
-// alike; the score is the fraction of persistent slots kept busy, with a
-// small cost per split, preferring wider tiles.
-Plan plan_gemm(int64_t M, int64_t N, int64_t K, const DeviceInfo& d,
-               GemmKind kind = GemmKind::kPromotion) {
-  Plan best{};
-  double best_score = -1.0;
-  double best_time = 1e30;
-  const int kbn = static_cast<int>(K / 128);
-  const bool compute_bound = M > 128;
-  const int slots = d.sms;
-  for (int bn : {256, 192, 128}) {
-    if (bn == 192 && (kind != GemmKind::kPromotion || !compute_bound)) continue;
-    const int m_tiles = static_cast<int>((M + 127) / 128);
-    const int n_tiles = static_cast<int>((N + bn - 1) / bn);
-    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
-    // Split K only when the tiles alone cannot fill the GPU.
-    const int max_split = tiles >= slots ? 1 : std::min(16, std::max(1, kbn / 4));
-    for (int s = 1; s <= max_split; ++s) {
-      const int per = (kbn + s - 1) / s;
-      const int splits = (kbn + per - 1) / per;
-      if (splits != s) continue;
-      const int64_t units = tiles * splits;
-      bool better;
-      Plan cand{bn, m_tiles, n_tiles, splits, per, static_cast<int>(units),
-                static_cast<int>(std::min<int64_t>(units, slots))};
-      if (compute_bound) {
-        const double kb_us = kb_time_us(kind, bn);
-        const double waves = static_cast<double>((units + slots - 1) / slots);
-        double t = waves * per * kb_us;
-        if (splits > 1)   // partials written and read back (HBM ~5 TB/s), bf16 out, launch
-          t += (8.0 * splits + 2.0) * static_cast<double>(M) * N / 5.0e6 + 5.0;
-        const int64_t tail = tiles % slots;
-        if (splits == 1 && tiles > slots && tail > 0 && 2 * tail <= slots) {
-          const size_t tile_bytes = static_cast<size_t>(128) * bn * sizeof(float);
-          const int64_t by_ws = static_cast<int64_t>(kTailWorkspaceCap / (tail * tile_bytes));
-          const int ts = static_cast<int>(std::min<int64_t>({slots / tail, kbn / 4, by_ws}));
-          if (ts >= 2) {
-            const int tkb = (kbn + ts - 1) / ts;
-            const double t_tail = static_cast<double>(tiles / slots) * per * kb_us +
-                                  tkb * kb_us + 3.0;   // + the reduction launch
-            if (t_tail < t) {
-              t = t_tail;
-              cand.full_units = static_cast<int>(tiles - tail);
-              cand.tail_tiles = static_cast<int>(tail);
-              cand.tail_splits = (kbn + tkb - 1) / tkb;
-              cand.tail_kbps = tkb;
-              cand.units = cand.full_units + cand.tail_tiles * cand.tail_splits;
-              cand.grid = slots;
-            }
-          }
-        }
-        better = t < best_time - 1e-9;
-        if (better) best_time = t;
-      } else {
-        const double eff = wave_efficiency(units, slots);
-        const double fill = static_cast<double>(std::min<int64_t>(M, 128)) / 128;
-        const double feed = bn == 128 ? 0.97 : 1.0;
-        const double split_cost = splits > 1 ? 0.95 - 0.002 * splits : 1.0;
-        const double score = eff * feed * split_cost * (fill + 0.5 * (1 - fill));
-        better = score > best_score + 1e-9;
-        if (better) best_score = score;
-      }
-      if (better) best = cand;
-    }
-  }
-  if (best.splits == 1 && compute_bound) best.n_group = choose_n_group(M, K, best.bn, best.n_tiles);
-  return best;
-}
-
-// Bytes of the K-block-major copies of the two scale tables that the
-// row-scaled GEMM stages in its workspace.
-size_t rowwise_stage_bytes(int64_t M, int64_t N, int64_t K) {
-  return static_cast<size_t>(M + N) * static_cast<size_t>(K / 128) * sizeof(float);
-}
-
-size_t plan_workspace(const Plan& pl, int64_t M, int64_t N) {
-  if (pl.tail_splits > 0)
-    return static_cast<size_t>(pl.tail_tiles) * pl.tail_splits * 128 * pl.bn * sizeof(float);
-  return pl.splits > 1 ? static_cast<size_t>(pl.splits) * M * N * sizeof(float) : 0;
-}
 
 template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
@@ -486,7 +343,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const Plan pl = plan_gemm(M, N, K, *info, w_rowwise ? GemmKind::kRowScaled : GemmKind::kPromotion);
+  const Plan pl = plan_gemm(M, N, K, info->sms, w_rowwise ? GemmKind::kRowScaled : GemmKind::kPromotion);
   // Row scales on W: both scale tables are staged K-block-major after the
   // split-K area of the workspace.
   const size_t split_bytes = plan_workspace(pl, M, N);
@@ -520,22 +377,8 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
   p.m_offsets = nullptr;
-  p.M = M;
-  p.N = static_cast<int>(N);
-  p.kbn = static_cast<int>(K / 128);
-  p.nbn = static_cast<int>((N + 127) / 128);
-  p.m_tiles = pl.m_tiles;
-  p.n_tiles = pl.n_tiles;
-  p.n_group = pl.n_group;
-  p.splits = pl.splits;
-  p.kb_per_split = pl.kb_per_split;
-  p.num_units = pl.units;
-  p.full_units = pl.full_units;
-  p.tail_tiles = pl.tail_tiles;
-  p.tail_splits = pl.tail_splits;
-  p.tail_kbps = pl.tail_kbps;
+  set_schedule(p, pl, M, N, K);
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
-  p.groups = 1;
   cudaError_t e;
   if (w_rowwise)
     e = pl.bn == 256 ? launch_gemm<256, false, 128, true>(ta, tw, ty, p, pl.grid, st)
@@ -598,7 +441,7 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   int dev;
   DeviceInfo* info;
   if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
-  const Plan pl = plan_gemm(M, N, K, *info, GemmKind::kBlockScaled);
+  const Plan pl = plan_gemm(M, N, K, info->sms, GemmKind::kBlockScaled);
   // Row scales on W: both scale tables are staged K-block-major after the
   // split-K area of the workspace.
   const size_t split_bytes = plan_workspace(pl, M, N);
@@ -628,22 +471,8 @@ fp8bs_status run_gemm_bs(const uint8_t* a, const float* a_s, const uint8_t* w, c
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
   p.m_offsets = nullptr;
-  p.M = M;
-  p.N = static_cast<int>(N);
-  p.kbn = static_cast<int>(K / 128);
-  p.nbn = static_cast<int>((N + 127) / 128);
-  p.m_tiles = pl.m_tiles;
-  p.n_tiles = pl.n_tiles;
-  p.n_group = pl.n_group;
-  p.splits = pl.splits;
-  p.kb_per_split = pl.kb_per_split;
-  p.num_units = pl.units;
-  p.full_units = pl.full_units;
-  p.tail_tiles = pl.tail_tiles;
-  p.tail_splits = pl.tail_splits;
-  p.tail_kbps = pl.tail_kbps;
+  set_schedule(p, pl, M, N, K);
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
-  p.groups = 1;
   cudaError_t e = w_rowwise
                       ? (pl.bn == 256 ? launch_gemm_bs<256, false, true>(ta, tw, ty, p, pl.grid, st)
                                       : launch_gemm_bs<128, false, true>(ta, tw, ty, p, pl.grid, st))
@@ -1077,9 +906,9 @@ size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   DeviceInfo* info;
   if (device_setup(&dev, &info) != FP8BS_OK) return 0;
   // One size serves both GEMM entry points (their plans may differ).
-  return std::max({plan_workspace(plan_gemm(M, N, K, *info), M, N),
-                   plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N),
-                   plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kRowScaled), M, N)});
+  return std::max({plan_workspace(plan_gemm(M, N, K, info->sms), M, N),
+                   plan_workspace(plan_gemm(M, N, K, info->sms, GemmKind::kBlockScaled), M, N),
+                   plan_workspace(plan_gemm(M, N, K, info->sms, GemmKind::kRowScaled), M, N)});
 }
 
 size_t fp8bs_gemm_rowwise_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -1088,8 +917,8 @@ size_t fp8bs_gemm_rowwise_workspace_size(int64_t M, int64_t N, int64_t K) {
   DeviceInfo* info;
   if (device_setup(&dev, &info) != FP8BS_OK) return 0;
   const size_t split = std::max(
-      plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kRowScaled), M, N),
-      plan_workspace(plan_gemm(M, N, K, *info, GemmKind::kBlockScaled), M, N));
+      plan_workspace(plan_gemm(M, N, K, info->sms, GemmKind::kRowScaled), M, N),
+      plan_workspace(plan_gemm(M, N, K, info->sms, GemmKind::kBlockScaled), M, N));
   return ((split + 255) & ~static_cast<size_t>(255)) + rowwise_stage_bytes(M, N, K);
 }
 
@@ -1101,7 +930,7 @@ const char* fp8bs_gemm_plan_string(int64_t M, int64_t N, int64_t K) {
     snprintf(buf, sizeof(buf), "none");
     return buf;
   }
-  const Plan pl = plan_gemm(M, N, K, *info);
+  const Plan pl = plan_gemm(M, N, K, info->sms);
   snprintf(buf, sizeof(buf),
            "bn=%d m_tiles=%d n_tiles=%d splits=%d kb_per_split=%d units=%d grid=%d sms=%d "
            "tail_tiles=%d tail_splits=%d n_group=%d",

@@ -250,7 +250,7 @@ __host__ __device__ __forceinline__ void tile_mn(int tile, int m_tiles, int n_ti
 }
 
 template <int kUnitRows>
-__device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
+__host__ __device__ __forceinline__ Unit dense_unit(const Params& p, int u) {
   Unit t;
   t.tail_slot = -1;
   if (p.tail_splits > 0 && u >= p.full_units) {
