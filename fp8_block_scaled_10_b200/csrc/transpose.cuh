@@ -24,8 +24,9 @@ namespace fp8bs {
 // flight at once read a few KB of each input row and write a KB of each output
 // row (a column-first order writes 128 bytes per output row and moves on).
 constexpr int64_t kBandGroup = 8;
-__device__ __forceinline__ void tile_coords(int64_t tile, int64_t bands, int64_t tiles_c,
-                                            int64_t& tr, int64_t& tc) {
+__host__ __device__ __forceinline__ void tile_coords(int64_t tile, int64_t bands,
+                                                     int64_t tiles_c, int64_t& tr,
+                                                     int64_t& tc) {
   const int64_t full = (bands / kBandGroup) * kBandGroup * tiles_c;
   if (tile < full) {
     const int64_t grp = tile / (kBandGroup * tiles_c), in = tile % (kBandGroup * tiles_c);

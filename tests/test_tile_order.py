@@ -1,7 +1,8 @@
-"""The GEMM's dense tile order (bands of n tiles, m fastest inside a band),
-checked on the CPU: tests/tile_order_check.cu includes the kernel header and
-runs its __host__ __device__ tile_mn over many shapes and band widths (no GPU
-needed; nvcc compiles the host side)."""
+"""The GEMM's dense tile order (bands of n tiles, m fastest inside a band)
+and the transposing kernels' tile order (groups of 8 row bands), checked on
+the CPU: tests/tile_order_check.cu includes the kernel headers and runs their
+__host__ __device__ tile_mn and tile_coords over many shapes (no GPU needed;
+nvcc compiles the host side)."""
 import os
 import shutil
 import subprocess
