@@ -247,14 +247,6 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Multiplier and shifts of div_invariant for a divisor d >= 1.
-InvariantDiv invariant_div(uint32_t d) {
-  uint32_t l = 0;
-  while (l < 32 && (uint64_t(1) << l) < d) ++l;
-  const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
-  return InvariantDiv{static_cast<uint32_t>(m), l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
-}
-
 // log2 of a supported quantization block size (32, 64, 128 or 256), else -1.
 int block_log2(int64_t block) {
   switch (block) {
@@ -299,17 +291,23 @@ template <bool G>
 cudaError_t launch_gemm_any(int bn, int a_rows, const CUtensorMap& ta, const CUtensorMap& tw,
                             const CUtensorMap& ty, const gemm::Params& p, int grid,
                             cudaStream_t st) {
-  if (!G && a_rows == 16)
-    return bn == 256 ? launch_gemm<256, G, 16>(ta, tw, ty, p, grid, st)
-                     : launch_gemm<128, G, 16>(ta, tw, ty, p, grid, st);
-  if (!G && a_rows == 64)
-    return bn == 256 ? launch_gemm<256, G, 64>(ta, tw, ty, p, grid, st)
-                     : launch_gemm<128, G, 64>(ta, tw, ty, p, grid, st);
-  if (G) return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
-                          : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
-  return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
-         : bn == 192 ? launch_gemm<192, G>(ta, tw, ty, p, grid, st)
+  // Grouped launches use 128-row A stages and 128- or 256-wide tiles only, so
+  // the other variants are not instantiated for them.
+  if constexpr (G) {
+    (void)a_rows;
+    return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
                      : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
+  } else {
+    if (a_rows == 16)
+      return bn == 256 ? launch_gemm<256, G, 16>(ta, tw, ty, p, grid, st)
+                       : launch_gemm<128, G, 16>(ta, tw, ty, p, grid, st);
+    if (a_rows == 64)
+      return bn == 256 ? launch_gemm<256, G, 64>(ta, tw, ty, p, grid, st)
+                       : launch_gemm<128, G, 64>(ta, tw, ty, p, grid, st);
+    return bn == 256 ? launch_gemm<256, G>(ta, tw, ty, p, grid, st)
+           : bn == 192 ? launch_gemm<192, G>(ta, tw, ty, p, grid, st)
+                       : launch_gemm<128, G>(ta, tw, ty, p, grid, st);
+  }
 }
 
 // Work units and tile indices are 32-bit in the kernels: the number of

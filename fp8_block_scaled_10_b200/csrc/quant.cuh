@@ -225,8 +225,20 @@ struct InvariantDiv {
   uint32_t m, sh1, sh2;
 };
 
-__device__ __forceinline__ uint32_t div_invariant(uint32_t n, const InvariantDiv& d) {
+// Multiplier and shifts for a divisor d >= 1 (host side, once per launch).
+inline InvariantDiv invariant_div(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (uint64_t(1) << l) < d) ++l;
+  const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
+  return InvariantDiv{static_cast<uint32_t>(m), l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
+}
+
+__host__ __device__ __forceinline__ uint32_t div_invariant(uint32_t n, const InvariantDiv& d) {
+#ifdef __CUDA_ARCH__
   const uint32_t t = __umulhi(n, d.m);
+#else
+  const uint32_t t = static_cast<uint32_t>((static_cast<uint64_t>(n) * d.m) >> 32);
+#endif
   return (t + ((n - t) >> d.sh1)) >> d.sh2;
 }
 
