@@ -8,10 +8,12 @@ batch: act_quant of x bf16 [4096, 7168] (1x128 blocks, scale_fmt None) and the
 block-scaled FP8 GEMM against W e4m3 [18432, 7168] with 128x128-block scales,
 bf16 out.  ``value`` is whole-job TFLOP/s (2*M*N*K per step per GPU).  The
 JSON line also carries the GEMM kernel's roofline, the per-workload parts
-(act_quant and weight_dequant GB/s at [16384, 7168] / [18432, 7168], decode,
-other prefill shapes, the expert-batched grouped GEMM), an end-to-end number
-through the C ABI with pinned host buffers, the clocks seen during the timed
-region, and the CPU oracle's throughput on a bounded sample.
+(act_quant, the static scheme, weight_quant and weight_dequant GB/s at
+[16384, 7168] / [18432, 7168]; the decode GEMMs; the other prefill shapes;
+the FP8- and FP32-output GEMMs; the expert-batched grouped GEMM; the training
+GEMMs' transposes and weight-gradient GEMM), an end-to-end number through the
+C ABI with pinned host buffers, the clocks seen during the timed region, and
+the CPU oracle's throughput on a bounded sample.
 
 Each rank (torchrun, one per GPU) runs an independent replica of the step;
 the path has no cross-GPU exchange, so there is no collective on the data
@@ -59,7 +61,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--quick", action="store_true", help="skip the per-workload parts")
+    ap.add_argument("--quick", action="store_true",
+                    help="omit the per-workload breakdown ('parts'); the step is timed in full either way")
     ap.add_argument("--parts", choices=["all", "memory", "decode", "training", "experts"],
                     default="all",
                     help="which per-workload parts to run: all, or only one group (memory-bound "
