@@ -161,3 +161,62 @@ def test_plain_c_client_builds_and_runs(L, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "abi c client ok"
+
+
+def _header_prototypes():
+    """name -> list of parameter declarations, from include/fp8bs.h."""
+    import os
+    import re
+    text = open(fp8bs.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"FP8BS_API\s+[^;(]*?\b(fp8bs_\w+)\s*\(([^)]*)\)\s*;", text, re.S):
+        params = [p.strip() for p in m.group(2).split(",")]
+        protos[m.group(1)] = [] if params == ["void"] else params
+    return protos
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every prototype's parameter count, and which parameters are pointers,
+    agree with the ctypes argument types the binding declares."""
+    import ctypes
+    protos = _header_prototypes()
+    assert set(protos) == set(fp8bs.header_symbols())
+    for name, params in protos.items():
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == len(params), (name, params)
+        for decl, ct in zip(params, fn.argtypes):
+            is_ptr = "*" in decl
+            assert is_ptr == (ct in (ctypes.c_void_p, ctypes.c_char_p) or
+                              hasattr(ct, "contents") or
+                              getattr(ct, "__name__", "").startswith("LP_")), (name, decl, ct)
+            if is_ptr:
+                continue
+            # integer widths: int64_t, size_t, and int or an enum (C int)
+            if "int64_t" in decl:
+                want = ctypes.c_int64
+            elif "size_t" in decl:
+                want = ctypes.c_size_t
+            else:
+                assert decl.split()[0] in ("int", "fp8bs_dtype", "fp8bs_scale_fmt",
+                                           "fp8bs_status"), (name, decl)
+                want = ctypes.c_int
+            assert ctypes.sizeof(ct) == ctypes.sizeof(want), (name, decl, ct)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built library the binding raises instead of falling back."""
+    code = ("import fp8_block_scaled_10_b200 as f\n"
+            "f.LIB_PATH = %r\n"
+            "f._lib = None\n"
+            "try:\n"
+            "    f.lib()\n"
+            "except ImportError as e:\n"
+            "    print('raised', e)\n" % str(tmp_path / "absent.so"))
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=root,
+                       timeout=120)
+    assert r.returncode == 0 and r.stdout.startswith("raised"), r.stdout + r.stderr
