@@ -329,7 +329,8 @@ __device__ __forceinline__ void group_table(const Params& p, int* table, int lan
 }
 
 template <int kUnitRows>
-__device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix, int u) {
+__host__ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int* tile_prefix,
+                                                      int u) {
   Unit t;
   const int gm = u / p.n_tiles;
   t.n_tile = u % p.n_tiles;
