@@ -419,7 +419,10 @@ FP8BS_API fp8bs_status fp8bs_fp8_linear(const uint16_t *x, int64_t M, int64_t K,
  *               non-decreasing, m_offsets[G] <= M_total); the host never reads
  *               them, so routing results need no host synchronization.  A group
  *               whose end is below its start is empty; rows outside
- *               [0, M_total) are never read or written.
+ *               [0, M_total) are never read or written.  Offsets that
+ *               decrease break the contract: memory stays safe (each group is
+ *               clamped to [0, M_total)), but a later group may then overlap
+ *               an earlier group's rows, whose y is then unspecified.
  *   a      device, [M_total, K];  a_s  device, [M_total, K / 128]
  *   w      device, [G, N, K];     w_s  device, [G, cdiv(N, 128), K / 128]
  *   y      device, [M_total, N] bf16; rows that belong to no group are left
