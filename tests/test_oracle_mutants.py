@@ -219,3 +219,24 @@ def test_weight_dequant_transposed_scale_index_fails_the_library_pin():
     wrong = flat[(j * 2 + i) % flat.numel()]        # column-major walk of the grid
     slip = (codes.view(torch.float8_e4m3fn).to(torch.float32) * wrong).numpy()
     assert not np.array_equal(slip, ref)
+
+
+def test_weight_quant_with_row_blocks_is_caught():
+    """weight_quant scales each 128 x 128 tile; quantizing in act_quant's
+    1 x 128 row blocks instead fails the per-tile torch comparison."""
+    g = torch.Generator().manual_seed(11)
+    rows, cols = 2 * BLOCK + 9, 3 * BLOCK - 5
+    w = torch.randn(rows, cols, generator=g) * 0.02
+    w[torch.rand(w.shape, generator=g) < 0.01] *= 30
+    rb, cb = -(-rows // BLOCK), -(-cols // BLOCK)
+    pad = torch.zeros(rb * BLOCK, cb * BLOCK)
+    pad[:rows, :cols] = w.abs()
+    amax = pad.reshape(rb, BLOCK, cb, BLOCK).amax(dim=(1, 3))
+    s = torch.clamp(amax, min=float(np.float32(1e-4))) / torch.tensor(448.0)
+    st = s.repeat_interleave(BLOCK, 0)[:rows].repeat_interleave(BLOCK, 1)[:, :cols]
+    want = _torch_codes(w / st)
+    good, _ = oracle.weight_quant(w.numpy())
+    assert np.array_equal(good, want)
+    slip = np.concatenate([oracle.act_quant(np.ascontiguousarray(w[:, j:j + BLOCK].numpy()))[0]
+                           for j in range(0, cols - cols % BLOCK, BLOCK)], axis=1)
+    assert not np.array_equal(slip, want[:, :slip.shape[1]])
