@@ -49,10 +49,29 @@ WORKLOAD = "prefill FP8 linear: act_quant x bf16 [4096,7168] + fp8_gemm W e4m3 [
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0     # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
-# DRAM bytes (read + write) of one prefill GEMM launch from the ncu capture
-# summarised in profiles/fp8_gemm_prefill_M4096_N18432_K7168.md.  It belongs
-# to the kernel as captured; reset it to None whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES = 169.671168e6 + 135.812096e6
+# DRAM bytes (read + write) of one prefill GEMM launch, from one ncu capture
+# of that launch (dram__bytes_read.sum + dram__bytes_write.sum), together with
+# a hash of the kernel sources it was captured from.  The bench line reports
+# the figure only while the sources still hash to the same value, so a kernel
+# change makes `traffic` null until the launch is captured again.
+GEMM_TRAFFIC = {"bytes": 169.671168e6 + 135.812096e6,
+                "sources_sha256": "captured-before-source-hashing"}
+GEMM_SOURCES = ("gemm.cuh", "gemm_bs.cuh", "sm100.cuh", "quant.cuh", "plan.h", "fp8bs.cu")
+
+
+def gemm_sources_sha256():
+    """Hash of the GEMM kernel sources (csrc/), in a fixed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "fp8_block_scaled_10_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic():
+    """The captured DRAM bytes per GEMM launch, or None once the sources differ."""
+    return GEMM_TRAFFIC["bytes"] if GEMM_TRAFFIC["sources_sha256"] == gemm_sources_sha256() else None
 
 
 def parse_args():
@@ -703,8 +722,9 @@ def ours(args, dist):
         "gpu_launches": lin.launches_per_step * args.steps,
         "roofline": {"bound": "tensor", "kernel": "fp8_gemm_kernel",
                      "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp8_peak, "traffic": GEMM_TRAFFIC_BYTES,
-                     "traffic_unit": "bytes per launch (ncu dram read+write)",
+                     "frac": gemm_tflops / fp8_peak, "traffic": gemm_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram read+write); null when the "
+                                     "kernel sources changed since the capture",
                      "peak_note": "%s bf16 burst %.1f TFLOP/s x %.1f (nominal FP8/BF16 dense ratio)"
                                   % (peak_kind, bf16, FP8_OVER_BF16)},
         "gemm_plan": fp8bs.gemm_plan(M, N, K),

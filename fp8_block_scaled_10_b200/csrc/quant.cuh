@@ -87,6 +87,10 @@ __device__ __forceinline__ float2 quotient2(float2 x, float2 r, float2 ns) {
 // Quantizes 8 values of one block and packs the codes (element 0 in the low
 // byte).  For ue8m0, r = 1/s is an exact power of two, so x * r is exactly
 // the correctly rounded x / s; otherwise the quotient comes from quotient2.
+// A block holding an infinity has s = inf and r = 0: the IEEE quotient of a
+// finite x is then a signed zero, which the first estimate x * 0 already is,
+// while the correction steps would compute 0 * inf = NaN.  With ns = 0 each
+// step gives back its input (e = x, q + x * 0 = q), so the estimate stands.
 template <bool UE8M0>
 __device__ __forceinline__ uint2 quantize8(const float (&v)[8], float s, float r) {
   float t[8];
@@ -94,7 +98,8 @@ __device__ __forceinline__ uint2 quantize8(const float (&v)[8], float s, float r
 #pragma unroll
     for (int j = 0; j < 8; ++j) t[j] = v[j] * r;
   } else {
-    const float2 r2 = make_float2(r, r), ns2 = make_float2(-s, -s);
+    const float ns = isinf(s) ? 0.0f : -s;
+    const float2 r2 = make_float2(r, r), ns2 = make_float2(ns, ns);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float2 q = quotient2(make_float2(v[2 * j], v[2 * j + 1]), r2, ns2);

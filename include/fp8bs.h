@@ -17,6 +17,12 @@
  * scratch space take it from a caller-provided workspace whose size the
  * matching *_workspace_size() function returns.
  *
+ * Per-device set-up (kernel attributes, the tensor-map encoder, the static
+ * scratch array's address) is done on the first call that needs it on each
+ * device and kept for the life of the process.  After cudaDeviceReset() of a
+ * device, no entry point of this library may be called on that device again
+ * in the same process: the kept set-up would refer to the destroyed context.
+ *
  * Sources of the operations (page title, then section):
  *  [ACT] "Understanding Dynamic and Static Activation Quantization Schemes in
  *        DeepSeek-V3", "How Dynamic Activation Quantization Works";
@@ -267,8 +273,9 @@ FP8BS_API fp8bs_status fp8bs_fp8_gemm(const uint8_t *a, const float *a_s, const 
  * An empty problem (M == 0) is validated like fp8bs_fp8_gemm and returns
  * FP8BS_OK without touching the device.  The first call with M > 0 on a
  * device looks up the scratch array's device address (cudaGetSymbolAddress,
- * once per device, on the current device); make that first call before any
- * stream capture.  All calls share the one array and
+ * once per device, on the current device) and keeps it for the life of the
+ * process (invalid after cudaDeviceReset(), as all per-device set-up above);
+ * make that first call before any stream capture.  All calls share the one array and
  * every call writes the partials it reads, so nothing needs clearing between
  * calls, but calls that overlap on the GPU (other streams, other threads)
  * race on the array: serialise them.

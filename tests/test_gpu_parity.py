@@ -98,6 +98,38 @@ def test_act_quant_special_blocks(fmt, dtype):
     assert np.array_equal(u8(q), q_ref)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [None, "ue8m0"])
+def test_act_quant_infinite_blocks(fmt, dtype):
+    """A block holding one +-inf: s = inf, every finite element of the block
+    is the IEEE quotient x / inf = +-0 (codes 0x00 / 0x80), and the infinite
+    element itself is inf / inf = NaN, whose sign IEEE leaves open (either
+    NaN code is accepted there).  The other blocks are unaffected."""
+    rows, cols = 64, 1024
+    x = wl.normal_with_outliers(rows, cols, seed=91, frac=0.01, factor=50.0).float().numpy()
+    rng = np.random.default_rng(92)
+    inf_at = []
+    for r in range(rows):
+        for b in rng.choice(cols // 128, size=2, replace=False):
+            c = int(b) * 128 + int(rng.integers(0, 128))
+            x[r, c] = np.inf if rng.random() < 0.5 else -np.inf
+            inf_at.append((r, c))
+    xt = torch.from_numpy(x).to(dtype)
+    q, s = fp8bs.act_quant(xt.cuda(), 128, fmt)
+    q_ref, s_ref = _oracle_act_quant(xt, fmt)
+    assert np.array_equal(f32bits(s.cpu().numpy()), f32bits(s_ref))
+    assert np.isinf(s_ref).sum() == len(inf_at)
+    got = u8(q)
+    nan_mask = np.zeros_like(got, dtype=bool)
+    for r, c in inf_at:
+        nan_mask[r, c] = True
+    assert np.all((got[nan_mask] & 0x7F) == 0x7F) and np.all((q_ref[nan_mask] & 0x7F) == 0x7F)
+    assert np.array_equal(got[~nan_mask], q_ref[~nan_mask])
+    # every finite element of an infinite block encodes a signed zero
+    blk_inf = np.repeat(np.isinf(s_ref), 128, axis=1) & ~nan_mask
+    assert np.all((got[blk_inf] & 0x7F) == 0)
+
+
 def test_act_quant_many_midpoints_fp32():
     """fp32 inputs built as e4m3 midpoint * s: the exact-division fallback runs often."""
     rng = np.random.default_rng(7)

@@ -6,8 +6,11 @@ of a caller workspace.
 
 Checked through the C ABI against fp8bs_fp8_gemm (which is given a torch
 workspace) on a split-K problem, for two calls in a row; the second call
-reuses the array the first one left behind.  Oversize problems must be
-refused before any launch.  This file is collected last on purpose.
+reuses the array the first one left behind.  Both entry points run the same
+plan, kernels and summation order, so their outputs must agree bit for bit;
+both are also held to the GEMM tolerance against the oracle's FP64 product.
+Oversize problems must be refused before any launch.  This file is collected
+last on purpose.
 """
 import ctypes
 
@@ -52,17 +55,20 @@ def test_static_scratch_gemm_matches_workspace_gemm():
     y_ws = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     assert L.fp8bs_fp8_gemm(_vp(a), _vp(a_s), _vp(w), _vp(w_s), M, N, K, _vp(y_ws),
                             _vp(ws), need, _stream()) == fp8bs.OK
-    y_ref = y_ws.float().cpu().numpy().astype(np.float64)
-    _, bound = oracle.gemm(qa, sa, qw, sw)
+    y_ref, bound = oracle.gemm(qa, sa, qw, sw)
     tol = GEMM_REL * np.abs(y_ref) + GEMM_ABS_OF_BOUND * bound
+    err_ws = np.abs(y_ws.float().cpu().numpy().astype(np.float64) - y_ref)
+    assert np.all(err_ws <= tol), "workspace GEMM: %d outputs outside tolerance" % int((err_ws > tol).sum())
 
     for call in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         st = L.fp8bs_fp8_gemm_static_scratch(_vp(a), _vp(a_s), _vp(w), _vp(w_s), M, N, K,
                                              _vp(y), _stream())
         assert st == fp8bs.OK, L.fp8bs_last_error_message()
-        got = y.float().cpu().numpy().astype(np.float64)
-        err = np.abs(got - y_ref)
+        # same plan and summation order as the workspace call: identical bits
+        assert torch.equal(y.view(torch.int16), y_ws.view(torch.int16)), \
+            "call %d: %d outputs differ from fp8bs_fp8_gemm" % (call, int((y.view(torch.int16) != y_ws.view(torch.int16)).sum()))
+        err = np.abs(y.float().cpu().numpy().astype(np.float64) - y_ref)
         assert np.all(err <= tol), "call %d: %d outputs outside tolerance" % (call, int((err > tol).sum()))
     assert fp8bs.device_error() == 0
 
