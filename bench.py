@@ -82,10 +82,16 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true",
                     help="omit the per-workload breakdown ('parts'); the step is timed in full either way")
-    ap.add_argument("--parts", choices=["all", "memory", "decode", "training", "experts"],
+    ap.add_argument("--parts", choices=["all", "memory", "decode", "prefill", "training", "experts"],
                     default="all",
                     help="which per-workload parts to run: all, or only one group (memory-bound "
-                         "quantizers and dequant, decode GEMMs, training GEMMs, grouped experts)")
+                         "quantizers and dequant, decode GEMMs, prefill GEMMs, training GEMMs, "
+                         "grouped experts)")
+    ap.add_argument("--prefill-shape", default=None,
+                    help="with --parts prefill: only this K,N prefill shape (e.g. 7168,576)")
+    ap.add_argument("--parts-only", action="store_true",
+                    help="profiling aid: run only the --parts group (no headline step, no CPU "
+                         "baseline) and print {\"parts\": ...}")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -281,7 +287,7 @@ def time_events(fn, iters, flush=None, rounds=3):
     return statistics.median(means)
 
 
-def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
+def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all", prefill_shape=None):
     """Per-workload kernel measurements (outside the step's timed region)."""
     parts = {}
     L = fp8bs.lib()
@@ -298,6 +304,8 @@ def run_parts(fp8bs, wl, hbm, fp8_peak, stream, which="all"):
 
     if which == "training":
         return run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush)
+    if which == "prefill":
+        return run_prefill_parts(fp8bs, wl, fp8_peak, stream, prefill_shape)
     if which == "experts":
         return run_expert_parts(fp8bs, wl, fp8_peak, stream)
     if which == "decode":
@@ -408,31 +416,7 @@ def run_gemm_parts(fp8bs, wl, hbm, fp8_peak, stream, flush, parts, which):
         del lin
     if which == "decode":
         return parts
-    # prefill shapes: fused act_quant + GEMM per call, and the GEMM alone
-    for kk, nn in wl.PREFILL_KN:
-        for fmt in (0, 1):
-            lin = Linear(fp8bs, wl, wl.PREFILL_M, kk, nn, fmt=fmt, seed=200 + kk + nn)
-            for _ in range(3):
-                lin.act_quant(stream); lin.gemm(stream)
-            ms_g = time_events(lambda: lin.gemm(stream), 10)
-            ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm(stream)), 10)
-            fl = 2 * wl.PREFILL_M * nn * kk
-            parts["prefill_K%d_N%d_%s" % (kk, nn, "ue8m0" if fmt else "none")] = {
-                "plan": fp8bs.gemm_plan(wl.PREFILL_M, nn, kk),
-                "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
-                "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
-                "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
-            if fmt:
-                for _ in range(3):
-                    lin.gemm_bs(stream)
-                ms_g = time_events(lambda: lin.gemm_bs(stream), 10)
-                ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm_bs(stream)), 10)
-                parts["prefill_K%d_N%d_ue8m0_bs" % (kk, nn)] = {
-                    "kernel": "block-scaled MMA",
-                    "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
-                    "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
-                    "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
-            del lin
+    parts.update(run_prefill_parts(fp8bs, wl, fp8_peak, stream))
     # FP8-output GEMM (the epilogue quantizes y for the next layer) against the
     # bf16-output GEMM followed by act_quant of y, prefill K=7168, N=18432
     lin = Linear(fp8bs, wl, wl.PREFILL_M, 7168, 18432, fmt=0, seed=300)
@@ -467,6 +451,39 @@ def run_gemm_parts(fp8bs, wl, hbm, fp8_peak, stream, flush, parts, which):
     del lin, q_out, s_out, y32
     parts.update(run_expert_parts(fp8bs, wl, fp8_peak, stream))
     parts.update(run_training_parts(fp8bs, wl, hbm, fp8_peak, stream, flush))
+    return parts
+
+
+def run_prefill_parts(fp8bs, wl, fp8_peak, stream, shape=None):
+    """The prefill shapes (M = 4096): act_quant + GEMM per call, and the GEMM
+    alone, for both scale formats; `shape` = (K, N) restricts it to one shape."""
+    parts = {}
+    for kk, nn in wl.PREFILL_KN:
+        if shape is not None and (kk, nn) != shape:
+            continue
+        for fmt in (0, 1):
+            lin = Linear(fp8bs, wl, wl.PREFILL_M, kk, nn, fmt=fmt, seed=200 + kk + nn)
+            for _ in range(3):
+                lin.act_quant(stream); lin.gemm(stream)
+            ms_g = time_events(lambda: lin.gemm(stream), 10)
+            ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm(stream)), 10)
+            fl = 2 * wl.PREFILL_M * nn * kk
+            parts["prefill_K%d_N%d_%s" % (kk, nn, "ue8m0" if fmt else "none")] = {
+                "plan": fp8bs.gemm_plan(wl.PREFILL_M, nn, kk),
+                "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
+                "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
+                "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
+            if fmt:
+                for _ in range(3):
+                    lin.gemm_bs(stream)
+                ms_g = time_events(lambda: lin.gemm_bs(stream), 10)
+                ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm_bs(stream)), 10)
+                parts["prefill_K%d_N%d_ue8m0_bs" % (kk, nn)] = {
+                    "kernel": "block-scaled MMA",
+                    "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
+                    "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
+                    "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
+            del lin
     return parts
 
 
@@ -611,6 +628,13 @@ def cpu_baseline(target_s, impl_steps=None):
     return rows, run, times
 
 
+def _prefill_shape(args):
+    if not args.prefill_shape:
+        return None
+    k, n = (int(v) for v in args.prefill_shape.split(","))
+    return (k, n)
+
+
 def ours(args, dist):
     import fp8_block_scaled_10_b200 as fp8bs
     from fp8_block_scaled_10_b200 import build, workloads as wl
@@ -621,6 +645,9 @@ def ours(args, dist):
     fp8_peak = bf16 * FP8_OVER_BF16
     stream_t = torch.cuda.current_stream()
     stream = ctypes.c_void_p(stream_t.cuda_stream)
+    if args.parts_only:
+        return {"parts": run_parts(fp8bs, wl, hbm, fp8_peak, stream, args.parts, _prefill_shape(args)),
+                "note": "--parts-only: a profiling aid, not a bench line"}
 
     lin = Linear(fp8bs, wl, M, K, N, fmt=0, seed=1234 + dist.rank)
     flops = 2.0 * M * N * K
@@ -739,7 +766,8 @@ def ours(args, dist):
     del x_host, y_host, x_dev, y_dev, lin
     torch.cuda.empty_cache()
     if not args.quick:
-        result["parts"] = run_parts(fp8bs, wl, hbm, fp8_peak, stream, args.parts)
+        result["parts"] = run_parts(fp8bs, wl, hbm, fp8_peak, stream, args.parts,
+                                    _prefill_shape(args))
         result["parts_note"] = "each part: median over 3 rounds of the mean of 10 event-timed launches, after 3 warm-ups; memory-bound parts and decode GEMMs flush L2 before each launch (memset of 4x L2 size, then a read of 2x L2 size so no dirty lines are written back inside the timed launch); GB/s of algorithmic bytes vs %s HBM %.1f GB/s" % (peak_kind, hbm)
     if dist.rank == 0:
         rows, run, _ = cpu_baseline(args.cpu_seconds)

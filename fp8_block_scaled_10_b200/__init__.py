@@ -81,6 +81,7 @@ def lib():
         "fp8bs_gemm_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
         "fp8bs_selftest_quotient": (i32, [p, p, p, i64, p]),
         "fp8bs_selftest_block_scale": (i32, [p, p, i64, i32, p]),
+        "fp8bs_selftest_gemm_stall": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, i32, p]),
         "fp8bs_fp8_gemm": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
         "fp8bs_fp8_gemm_static_scratch": (i32, [p, p, p, p, i64, i64, i64, p, p]),
         "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),

@@ -332,7 +332,7 @@ fp8bs_status check_gemm_operands(const uint8_t* a, const float* a_s, const uint8
 fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
                       int64_t M, int64_t N, int64_t K, void* y, void* ws, size_t ws_bytes,
                       cudaStream_t st, bool out_f32 = false,
-                      bool w_rowwise = false, bool check_pow2 = false) {
+                      bool w_rowwise = false, bool check_pow2 = false, int stall_step = 0) {
   fp8bs_status r = check_gemm_operands(a, a_s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
   if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
@@ -375,6 +375,7 @@ fp8bs_status run_gemm(const uint8_t* a, const float* a_s, const uint8_t* w, cons
   p.ws = static_cast<float*>(out_f32 && pl.splits == 1 ? y : ws);
   p.out_f32 = out_f32 ? 1 : 0;
   p.m_offsets = nullptr;
+  p.stall_step = stall_step;
   set_schedule(p, pl, M, N, K);
   p.tail_ws = pl.tail_splits > 0 ? static_cast<float*>(ws) : nullptr;
   cudaError_t e;
@@ -896,6 +897,15 @@ fp8bs_status fp8bs_selftest_block_scale(const float* amax, float* s, int64_t n, 
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "block-scale self-test launch");
   return FP8BS_OK;
+}
+
+fp8bs_status fp8bs_selftest_gemm_stall(const uint8_t* a, const float* a_s, const uint8_t* w,
+                                       const float* w_s, int64_t M, int64_t N, int64_t K,
+                                       uint16_t* y, void* workspace, size_t workspace_bytes,
+                                       int stall_step, void* stream) {
+  if (stall_step < 1) return fail(FP8BS_ERR_INVALID_ARG, "stall_step must be >= 1");
+  return run_gemm(a, a_s, w, w_s, M, N, K, y, workspace, workspace_bytes, as_stream(stream),
+                  false, false, false, stall_step);
 }
 
 size_t fp8bs_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {

@@ -101,6 +101,11 @@ struct Params {
   // split: ws = y, y_tma 2 maps y as a single split; several: the reduction
   // writes FP32).  p.y is unused then.
   int out_f32;
+  // Test of the bounded waits only (0 in every product launch): CTA 0's scale
+  // producer withholds its arrival for its K-block step stall_step - 1
+  // (counted over its units from 0), so the epilogue's wait on that step
+  // cannot complete and must give up.
+  int stall_step;
 };
 
 // Nonzero unless v is a positive normal power of two.
@@ -603,6 +608,9 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     }
     int slot = 0;
     uint32_t sphase = 0;
+    const uint32_t stall_at =
+        (p.stall_step > 0 && blockIdx.x == 0) ? static_cast<uint32_t>(p.stall_step - 1) : 0xFFFFFFFFu;
+    uint32_t step = 0;
     while (cur.valid) {
 #pragma unroll
       for (int ph = 0; ph < kAhead; ++ph) {
@@ -619,7 +627,8 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
           dst[BM + lane] = rw[ph][0];
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tfull[slot]);
+        if (lane == 0 && step != stall_at) mbar_arrive(&tfull[slot]);
+        ++step;
         load(ahead, ra[ph], rw[ph]);
         next(ahead);
         next(cur);

@@ -240,6 +240,27 @@ FP8BS_API fp8bs_status fp8bs_selftest_quotient(const float *x, const float *s, f
 FP8BS_API fp8bs_status fp8bs_selftest_block_scale(const float *amax, float *s, int64_t n,
                                                   int scale_fmt, void *stream);
 
+/*
+ * Self-test of the GEMM's bounded device waits (the pages show no failure
+ * handling; this is the library's own failure path).  Runs fp8bs_fp8_gemm
+ * with one arrival withheld: the first CTA's scale producer does not signal
+ * its K-block step stall_step - 1 (counted over that CTA's work units from
+ * 0), so the epilogue's wait for that step cannot complete.  The wait gives
+ * up after its limit (about 2 s), records FP8BS_ERR_TIMEOUT in the device
+ * error word, and every role of that CTA drains the copies and MMAs it has in
+ * flight, releases its tensor memory and exits; the other CTAs finish
+ * normally.  The context stays usable: fp8bs_get_device_error() then returns
+ * FP8BS_ERR_TIMEOUT, and later calls run normally.  y is left partly
+ * unwritten.  Arguments as for fp8bs_fp8_gemm, plus stall_step >= 1 (else
+ * FP8BS_ERR_INVALID_ARG); a step past the CTA's last one withholds nothing.
+ * For verification only.
+ */
+FP8BS_API fp8bs_status fp8bs_selftest_gemm_stall(const uint8_t *a, const float *a_s,
+                                                 const uint8_t *w, const float *w_s, int64_t M,
+                                                 int64_t N, int64_t K, uint16_t *y,
+                                                 void *workspace, size_t workspace_bytes,
+                                                 int stall_step, void *stream);
+
 /* Launch plan fp8_gemm would use for an M x N x K problem on the current
  * device (tile width, K split, work units, grid), as a
  * NUL-terminated string in thread-local storage; for logs and benchmarks. */
