@@ -240,6 +240,28 @@ class Linear:
                                    self.n, self.k, vp(self.y), vp(self.ws), self.nws, stream)
         assert st == 0, self.L.fp8bs_last_error_message()
 
+    def _linear_ws(self):
+        if not hasattr(self, "lws"):
+            self.nlws = int(self.L.fp8bs_linear_workspace_size(self.m, self.n, self.k))
+            self.lws = torch.empty(max(self.nlws, 16), dtype=torch.uint8, device="cuda")
+
+    def linear(self, stream):
+        """fp8bs_fp8_linear: act_quant and the GEMM in the form the library
+        plans for the shape (the two launches, or the fused launch)."""
+        self._linear_ws()
+        st = self.L.fp8bs_fp8_linear(vp(self.x), self.m, self.k, self.fmt, vp(self.qw), vp(self.sw),
+                                     self.n, vp(self.y), vp(self.q), vp(self.s), vp(self.lws),
+                                     self.nlws, stream)
+        assert st == 0, self.L.fp8bs_last_error_message()
+
+    def linear_fused(self, stream):
+        """fp8bs_fp8_linear_fused: the single-launch form (where one exists)."""
+        self._linear_ws()
+        st = self.L.fp8bs_fp8_linear_fused(vp(self.x), self.m, self.k, self.fmt, vp(self.qw),
+                                           vp(self.sw), self.n, vp(self.y), vp(self.q), vp(self.s),
+                                           vp(self.lws), self.nlws, stream)
+        return st
+
     def gemm_bs(self, stream):
         """The ue8m0 entry point (block-scaled MMA, or for decode-sized M the
         promotion kernel); needs fmt=1 (power-of-two scales)."""
@@ -466,13 +488,28 @@ def run_prefill_parts(fp8bs, wl, fp8_peak, stream, shape=None):
             for _ in range(3):
                 lin.act_quant(stream); lin.gemm(stream)
             ms_g = time_events(lambda: lin.gemm(stream), 10)
-            ms_l = time_events(lambda: (lin.act_quant(stream), lin.gemm(stream)), 10)
+            ms_2 = time_events(lambda: (lin.act_quant(stream), lin.gemm(stream)), 10)
+            for _ in range(3):
+                lin.linear(stream)
+            ms_l = time_events(lambda: lin.linear(stream), 10)
             fl = 2 * wl.PREFILL_M * nn * kk
+            ms_f = None
+            if lin.linear_fused(stream) == 0:
+                for _ in range(3):
+                    lin.linear_fused(stream)
+                ms_f = time_events(lambda: lin.linear_fused(stream), 10)
             parts["prefill_K%d_N%d_%s" % (kk, nn, "ue8m0" if fmt else "none")] = {
                 "plan": fp8bs.gemm_plan(wl.PREFILL_M, nn, kk),
                 "gemm_us": ms_g * 1e3, "gemm_TFLOP/s": fl / ms_g / 1e9,
                 "gemm_frac_fp8": fl / ms_g / 1e9 / fp8_peak,
-                "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9}
+                "linear_plan": fp8bs.linear_plan(wl.PREFILL_M, nn, kk),
+                "linear_us": ms_l * 1e3, "linear_TFLOP/s": fl / ms_l / 1e9,
+                "act_quant_then_gemm_us": ms_2 * 1e3,
+                "fused_linear_us": ms_f * 1e3 if ms_f is not None else None,
+                "note": "linear_us: fp8bs_fp8_linear (the form linear_plan names); "
+                        "act_quant_then_gemm_us: the two launches called separately; "
+                        "fused_linear_us: fp8bs_fp8_linear_fused, one launch (null where "
+                        "the tiles leave no SMs to quantize)"}
             if fmt:
                 for _ in range(3):
                     lin.gemm_bs(stream)

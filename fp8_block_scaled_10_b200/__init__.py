@@ -27,7 +27,8 @@ __all__ = [
     "act_quant", "act_quant_static", "act_dequant", "static_dequant",
     "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
     "fp8_gemm_grouped", "fp8_gemm_quant", "fp8_gemm_rowwise", "act_quant_transposed",
-    "fp8_transpose", "gemm_workspace_size", "gemm_plan", "device_error", "lib", "Fp8bsError",
+    "fp8_transpose", "gemm_workspace_size", "gemm_plan", "linear_plan", "device_error", "lib",
+    "Fp8bsError",
     "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -85,6 +86,9 @@ def lib():
         "fp8bs_fp8_gemm": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
         "fp8bs_fp8_gemm_static_scratch": (i32, [p, p, p, p, i64, i64, i64, p, p]),
         "fp8bs_fp8_linear": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
+        "fp8bs_linear_workspace_size": (sz, [i64, i64, i64]),
+        "fp8bs_fp8_linear_fused": (i32, [p, i64, i64, i32, p, p, i64, p, p, p, p, sz, p]),
+        "fp8bs_linear_plan_string": (ctypes.c_char_p, [i64, i64, i64]),
         "fp8bs_fp8_gemm_ue8m0": (i32, [p, p, p, p, i64, i64, i64, p, p, sz, p]),
         "fp8bs_fp8_gemm_f32": (i32, [p, p, p, p, i64, i64, i64, i32, p, p, sz, p]),
         "fp8bs_fp8_linear_ue8m0": (i32, [p, i64, i64, p, p, i64, p, p, p, p, sz, p]),
@@ -366,6 +370,12 @@ def gemm_workspace_size(M, N, K):
     return int(lib().fp8bs_gemm_workspace_size(M, N, K))
 
 
+def linear_plan(M, N, K):
+    """Which form fp8_linear takes for this shape on the current device
+    (fused act_quant + GEMM in one launch, or the two launches)."""
+    return lib().fp8bs_linear_plan_string(M, N, K).decode()
+
+
 def gemm_plan(M, N, K):
     """The launch plan fp8_gemm uses for an M x N x K problem on this device."""
     return lib().fp8bs_gemm_plan_string(M, N, K).decode()
@@ -449,12 +459,14 @@ def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,
     y = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
     q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
     s = torch.empty(*x.shape[:-1], K // 128, dtype=torch.float32, device=x.device)
-    ws, nws = _workspace(M, N, K, x.device)
     if _scale_fmt(scale_fmt) and _scale_fmt(weight_scale_fmt):
+        ws, nws = _workspace(M, N, K, x.device)
         _check(lib().fp8bs_fp8_linear_ue8m0(_ptr(x), M, K, _ptr(w), _ptr(weight_scale), N,
                                             _ptr(y), _ptr(q), _ptr(s), _ptr(ws), nws,
                                             _stream(x.device)))
     else:
+        nws = int(lib().fp8bs_linear_workspace_size(M, N, K))
+        ws = torch.empty(nws, dtype=torch.uint8, device=x.device) if nws else None
         _check(lib().fp8bs_fp8_linear(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
                                       _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s), _ptr(ws),
                                       nws, _stream(x.device)))

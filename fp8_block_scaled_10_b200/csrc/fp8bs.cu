@@ -62,10 +62,10 @@ EncodeTiledFn g_encode = nullptr;
 // Opts the GEMM kernel into its dynamic shared memory and checks that the
 // registers it is launched with cover its warpgroup register split (a split
 // larger than the launch total would make setmaxnreg.inc wait forever).
-template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false>
+template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false, bool FUSED = false>
 fp8bs_status setup_gemm_kernel() {
   using C = gemm::Cfg<BN, AR>;
-  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK>;
+  auto kernel = gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::smem_bytes(G));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -132,7 +132,10 @@ fp8bs_status device_setup(int* dev_out, DeviceInfo** info_out) {
         (r = setup_gemm_kernel<256, false, 64, false, true>()) != FP8BS_OK ||
         (r = setup_gemm_kernel<256, false, 128, true>()) != FP8BS_OK ||
         (r = setup_gemm_bs_kernel<128, false, true>()) != FP8BS_OK ||
-        (r = setup_gemm_bs_kernel<256, false, true>()) != FP8BS_OK)
+        (r = setup_gemm_bs_kernel<256, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<128, false, 128, false, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<192, false, 128, false, false, true>()) != FP8BS_OK ||
+        (r = setup_gemm_kernel<256, false, 128, false, false, true>()) != FP8BS_OK)
       return r;
     for (auto k : {act_quant_transposed_tma_kernel<false>, act_quant_transposed_tma_kernel<true>}) {
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -275,12 +278,16 @@ int grid_for(int64_t work_items, int64_t per_cta, int max_ctas) {
 }
 
 
-template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false>
+// The x map of fused launches; unused (zero) in every other GEMM launch.
+const CUtensorMap kNoMap{};
+
+template <int BN, bool G, int AR = 128, bool BROW = false, bool CHECK = false, bool FUSED = false>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
-                        const gemm::Params& p, int grid, cudaStream_t st) {
+                        const gemm::Params& p, int grid, cudaStream_t st,
+                        const CUtensorMap& tx = kNoMap) {
   using C = gemm::Cfg<BN, AR>;
-  return launch(gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK>, grid, C::kThreads,
-                C::smem_bytes(G), st, ta, tw, ty, p);
+  return launch(gemm::fp8_gemm_kernel<BN, G, AR, BROW, CHECK, FUSED>, grid, C::kThreads,
+                C::smem_bytes(G), st, ta, tw, ty, tx, p);
 }
 
 // Rows of A one pipeline stage loads: all 128 rows of a tile, or for
@@ -586,6 +593,54 @@ fp8bs_status run_act_quant(const void* x, fp8bs_dtype x_dtype, int64_t rows, int
            : launch_act_quant<float, false>(block, grid, st, xf, q, s, nblocks);
   }
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return FP8BS_OK;
+}
+
+// The fused linear launch (linear.cuh): lp.gemm_ctas CTAs run the GEMM's
+// tiles (one wave, no K split), the remaining CTAs quantize x into q and s and
+// count each chunk into the flags, which are zeroed first.
+fp8bs_status run_linear_fused(const uint16_t* x, int64_t M, int64_t K, bool ue8m0,
+                              const uint8_t* w, const float* w_s, int64_t N, uint16_t* y,
+                              uint8_t* q, float* s, int* flags, size_t flag_bytes,
+                              const LinearPlan& lp, int sms, cudaStream_t st) {
+  fp8bs_status r;
+  const Plan& pl = lp.gemm;
+  CUtensorMap ta, tw, ty, tx;
+  gemm::Params p{};
+  if ((r = make_tmap(&ta, q, M, K, 128)) != FP8BS_OK) return r;
+  if ((r = make_tmap(&tw, w, N, K, pl.bn)) != FP8BS_OK) return r;
+  if ((r = make_tmap_out(&ty, y, nullptr, M, N, 1, &p.y_tma)) != FP8BS_OK) return r;
+  {
+    // x [M, K] bf16 in boxes of 128 rows x 64 columns, 128-byte swizzle.
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2u};
+    const cuuint32_t box[2] = {64u, 128u};
+    const cuuint32_t elem[2] = {1u, 1u};
+    const CUresult cr = g_encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x),
+                                 dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(FP8BS_ERR_CUDA, "cuTensorMapEncodeTiled (x) failed (%d)", (int)cr);
+  }
+  p.sa = s;
+  p.sw = w_s;
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ws = nullptr;
+  p.m_offsets = nullptr;
+  set_schedule(p, pl, M, N, K);
+  p.gemm_ctas = lp.gemm_ctas;
+  p.fq_flags = flags;
+  p.fq_q = q;
+  p.fq_s = s;
+  p.fq_ue8m0 = ue8m0 ? 1 : 0;
+  cudaError_t e = cudaMemsetAsync(flags, 0, flag_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "fused linear flag reset");
+  const int grid = lp.gemm_ctas + lp.quant_ctas;
+  if (grid > sms) return fail(FP8BS_ERR_UNSUPPORTED, "fused linear grid %d > %d SMs", grid, sms);
+  e = pl.bn == 256 ? launch_gemm<256, false, 128, false, false, true>(ta, tw, ty, p, grid, st, tx)
+      : pl.bn == 192 ? launch_gemm<192, false, 128, false, false, true>(ta, tw, ty, p, grid, st, tx)
+                     : launch_gemm<128, false, 128, false, false, true>(ta, tw, ty, p, grid, st, tx);
+  if (e != cudaSuccess) return cuda_fail(e, "fused linear launch");
   return FP8BS_OK;
 }
 
@@ -1111,10 +1166,75 @@ fp8bs_status fp8bs_fp8_linear(const uint16_t* x, int64_t M, int64_t K, fp8bs_sca
                               void* stream) {
   fp8bs_status r = check_gemm_operands(q, s, w, w_s, y, N, K);
   if (r != FP8BS_OK) return r;
+  if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
   if (M == 0) return FP8BS_OK;
   cudaStream_t st = as_stream(stream);
+  if (x != nullptr && aligned16(x) && !gemm_too_large(M, N)) {
+    int dev;
+    DeviceInfo* info;
+    if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+    const LinearPlan lp = plan_linear(M, N, K, info->sms);
+    const size_t flag_bytes = linear_flag_bytes(M, K);
+    if (lp.fused && workspace != nullptr && aligned16(workspace) && workspace_bytes >= flag_bytes)
+      return run_linear_fused(x, M, K, fmt == FP8BS_SCALE_FMT_UE8M0, w, w_s, N, y, q, s,
+                              static_cast<int*>(workspace), flag_bytes, lp, info->sms, st);
+  }
   if ((r = run_act_quant(x, FP8BS_DTYPE_BF16, M, K, 128, fmt, q, s, st)) != FP8BS_OK) return r;
   return run_gemm(q, s, w, w_s, M, N, K, y, workspace, workspace_bytes, st);
+}
+
+fp8bs_status fp8bs_fp8_linear_fused(const uint16_t* x, int64_t M, int64_t K,
+                                    fp8bs_scale_fmt fmt, const uint8_t* w, const float* w_s,
+                                    int64_t N, uint16_t* y, uint8_t* q, float* s,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  fp8bs_status r = check_gemm_operands(q, s, w, w_s, y, N, K);
+  if (r != FP8BS_OK) return r;
+  if (x == nullptr || !aligned16(x)) return fail(FP8BS_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if (M < 0 || M > (int64_t(1) << 31)) return fail(FP8BS_ERR_INVALID_ARG, "M out of range");
+  if (fmt != FP8BS_SCALE_FMT_NONE && fmt != FP8BS_SCALE_FMT_UE8M0)
+    return fail(FP8BS_ERR_INVALID_ARG, "scale_fmt");
+  if (M == 0) return FP8BS_OK;
+  if (gemm_too_large(M, N)) return fail(FP8BS_ERR_INVALID_ARG, "M x N too large (tile count)");
+  int dev;
+  DeviceInfo* info;
+  if ((r = device_setup(&dev, &info)) != FP8BS_OK) return r;
+  const LinearPlan lp = plan_linear_fused(M, N, K, info->sms);
+  if (!lp.fused)
+    return fail(FP8BS_ERR_UNSUPPORTED,
+                "no fused launch for M=%lld N=%lld: M must exceed 128 and the GEMM's tiles must "
+                "leave %d SMs free", (long long)M, (long long)N, kMinQuantCtas);
+  const size_t flag_bytes = linear_flag_bytes(M, K);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < flag_bytes)
+    return fail(FP8BS_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", flag_bytes);
+  return run_linear_fused(x, M, K, fmt == FP8BS_SCALE_FMT_UE8M0, w, w_s, N, y, q, s,
+                          static_cast<int*>(workspace), flag_bytes, lp, info->sms,
+                          as_stream(stream));
+}
+
+size_t fp8bs_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  return std::max(fp8bs_gemm_workspace_size(M, N, K), linear_flag_bytes(M, K));
+}
+
+const char* fp8bs_linear_plan_string(int64_t M, int64_t N, int64_t K) {
+  thread_local char buf[256];
+  int dev;
+  DeviceInfo* info;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || device_setup(&dev, &info) != FP8BS_OK) {
+    snprintf(buf, sizeof(buf), "none");
+    return buf;
+  }
+  const LinearPlan lp = plan_linear(M, N, K, info->sms);
+  const LinearPlan f = plan_linear_fused(M, N, K, info->sms);
+  char alt[96] = "fused: none";
+  if (f.fused)
+    snprintf(alt, sizeof(alt), "fused: bn=%d gemm_ctas=%d quant_ctas=%d est_us=%.1f", f.gemm.bn,
+             f.gemm_ctas, f.quant_ctas, f.est_us);
+  snprintf(buf, sizeof(buf), "%s bn=%d est_us=%.1f | %s", lp.fused ? "fused" : "act_quant+gemm",
+           lp.gemm.bn, lp.est_us, alt);
+  return buf;
 }
 
 fp8bs_status fp8bs_fp8_gemm_grouped(int64_t G, const int64_t* m_offsets, int64_t M_total,

@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "linear.cuh"
 #include "quant.cuh"
 #include "sm100.cuh"
 
@@ -101,6 +102,15 @@ struct Params {
   // split: ws = y, y_tma 2 maps y as a single split; several: the reduction
   // writes FP32).  p.y is unused then.
   int out_f32;
+  // Fused linear (FUSED instantiations): CTAs from gemm_ctas on quantize x
+  // into fq_q / fq_s (the buffers tmap_a and sa read) and count the chunks
+  // into fq_flags [m_tiles][kbn] (zero at launch); the GEMM CTAs wait for a
+  // chunk's flag before reading its codes or scales.
+  int gemm_ctas;
+  int* fq_flags;
+  uint8_t* fq_q;
+  float* fq_s;
+  int fq_ue8m0;
   // Test of the bounded waits only (0 in every product launch): CTA 0's scale
   // producer withholds its arrival for its K-block step stall_step - 1
   // (counted over its units from 0), so the epilogue's wait on that step
@@ -371,15 +381,35 @@ __host__ __device__ __forceinline__ Unit grouped_unit(const Params& p, const int
 // producer, the values slowed decode by ~5 us; in the TMA warp's spare lanes
 // the divergent check ran ahead of the first TMA issue.  A compile-time
 // switch, so the other instantiations carry none of it.
-template <int BN, bool GROUPED, int ARows = 128, bool BROW = false, bool CHECK = false>
+// FUSED: the fused linear layer (linear.cuh): CTAs from p.gemm_ctas on are
+// quantizer CTAs reading x through tmap_x; the GEMM CTAs (dense, one K split,
+// every unit within one wave) wait for each chunk's ready flag before they
+// read its codes (TMA) and scales.  tmap_x is unused otherwise.
+template <int BN, bool GROUPED, int ARows = 128, bool BROW = false, bool CHECK = false,
+          bool FUSED = false>
 __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w,
-                    const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+                    const __grid_constant__ CUtensorMap tmap_y,
+                    const __grid_constant__ CUtensorMap tmap_x, const Params p) {
   using C = Cfg<BN, ARows>;
+  static_assert(!FUSED || (!GROUPED && !BROW && !CHECK && ARows == 128), "fused linear: dense GEMM");
+  static_assert(!FUSED || C::smem_bytes(false) >= kQRingBytes + kQBarBytes + 1024,
+                "quantizer ring fits the GEMM's shared memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  if (FUSED && static_cast<int>(blockIdx.x) >= p.gemm_ctas) {
+    pdl_trigger();
+    pdl_wait();
+    const int qi = static_cast<int>(blockIdx.x) - p.gemm_ctas;
+    const int nq = static_cast<int>(gridDim.x) - p.gemm_ctas;
+    if (p.fq_ue8m0)
+      quantize_cta<true>(&tmap_x, p.M, p.kbn * BK, p.fq_q, p.fq_s, p.fq_flags, smem, qi, nq);
+    else
+      quantize_cta<false>(&tmap_x, p.M, p.kbn * BK, p.fq_q, p.fq_s, p.fq_flags, smem, qi, nq);
+    return;
+  }
   uint8_t* a_tiles = smem;
   uint8_t* b_tiles = smem + C::kStages * C::kABytes;
   Ctrl<C::kStages>* ctrl = reinterpret_cast<Ctrl<C::kStages>*>(smem + C::kStages * C::kStageBytes);
@@ -402,7 +432,7 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   pdl_trigger();
   const int unit_start = static_cast<int>(blockIdx.x);
-  const int unit_step = static_cast<int>(gridDim.x);
+  const int unit_step = FUSED ? p.gemm_ctas : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -472,6 +502,12 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
         const Unit t = unit_of(u);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+          if (FUSED) {
+            // The chunk's codes are written by a quantizer CTA of this launch.
+            if (!wait_chunk_flag(p.fq_flags + (t.row0 / BM) * p.kbn + kb, abort_flag))
+              goto producer_done;
+            fence_proxy_async_global();
+          }
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
                       static_cast<int32_t>(t.row0));
@@ -575,12 +611,23 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
       if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
     };
     auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWRegs]) {
+      if (FUSED && c.valid) {
+        // The scales are written in this launch: wait for the chunk, then read
+        // them from L2 (not through the non-coherent read-only path).
+        wait_chunk_flag(p.fq_flags + (c.row0 / BM) * p.kbn + c.kb, abort_flag);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t row = c.row0 + lane + 32 * j;
-        va[j] = (c.valid && row < c.row_end)
-                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
-                    : 0.0f;
+        for (int j = 0; j < 4; ++j) {
+          const int64_t row = c.row0 + lane + 32 * j;
+          va[j] = row < c.row_end ? __ldcg(p.sa + row * p.kbn + c.kb) : 0.0f;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t row = c.row0 + lane + 32 * j;
+          va[j] = (c.valid && row < c.row_end)
+                      ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
+                      : 0.0f;
+        }
       }
       if (BROW) {
         // K-block-major tables (sa [kbn][M], sw [kbn][N]): lanes read

@@ -24,6 +24,7 @@ struct Plan {
   // Split tail (see gemm::Params): 0 = none.
   int full_units = 0, tail_tiles = 0, tail_splits = 0, tail_kbps = 0;
   int n_group = 1;   // band width of the tile order (gemm::tile_mn)
+  double est_us = 0.0;   // the planner's time estimate (prefill-sized M)
 };
 
 // Band width of the dense tile order for one K split.  m fastest (width 1)
@@ -130,7 +131,10 @@ inline Plan plan_gemm(int64_t M, int64_t N, int64_t K, int sms,
           }
         }
         better = t < best_time - 1e-9;
-        if (better) best_time = t;
+        if (better) {
+          best_time = t;
+          cand.est_us = t;
+        }
       } else {
         const double eff = wave_efficiency(units, slots);
         const double fill = static_cast<double>(std::min<int64_t>(M, 128)) / 128;
@@ -145,6 +149,74 @@ inline Plan plan_gemm(int64_t M, int64_t N, int64_t K, int sms,
   }
   if (best.splits == 1 && compute_bound) best.n_group = choose_n_group(M, K, best.bn, best.n_tiles);
   return best;
+}
+
+// The fused linear layer (act_quant inside the GEMM launch, linear.cuh).
+// When the GEMM's tiles leave SMs idle, those SMs quantize x instead: the
+// launch has gemm_ctas CTAs walking the GEMM's tiles (one wave, no K split)
+// and quant_ctas CTAs streaming x and writing q and s, each (m tile, K block)
+// chunk announced by a ready flag that the GEMM CTAs wait for before they
+// load it.
+struct LinearPlan {
+  bool fused = false;
+  Plan gemm;            // the fused launch's tile plan (fused), else the GEMM's plan
+  int gemm_ctas = 0;
+  int quant_ctas = 0;
+  double est_us = 0.0;
+};
+
+constexpr int kMinQuantCtas = 16;
+// Measured on B200 (M = 4096, K = 7168, N = 576, 52 quantizer CTAs): a
+// quantizer CTA moves ~35 GB/s (x read, q and s written; it is bound by its
+// arithmetic, as act_quant is per SM), and a GEMM CTA spends ~0.64 us per K
+// block on the round trip of reading its chunk's flag.  act_quant alone moves
+// ~5.9 TB/s over all SMs.
+constexpr double kQuantCtaGBs = 35.0;
+constexpr double kFlagRoundTripUs = 0.64;
+constexpr double kActQuantGBs = 5900.0;
+
+inline size_t linear_flag_bytes(int64_t M, int64_t K) {
+  return static_cast<size_t>((M + 127) / 128) * static_cast<size_t>(K / 128) * sizeof(int);
+}
+
+// The best fused launch for the shape (fused = false when none fits: the
+// tiles must leave at least kMinQuantCtas SMs, and M must exceed 128).
+inline LinearPlan plan_linear_fused(int64_t M, int64_t N, int64_t K, int sms) {
+  LinearPlan lp;
+  if (M <= 128) return lp;
+  const double q_bytes = static_cast<double>(M) * K * 3.0 + 4.0 * M * (K / 128);
+  const int kbn = static_cast<int>(K / 128);
+  lp.est_us = 1e30;
+  for (int bn : {256, 192, 128}) {
+    const int m_tiles = static_cast<int>((M + 127) / 128);
+    const int n_tiles = static_cast<int>((N + bn - 1) / bn);
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    if (tiles + kMinQuantCtas > sms) continue;
+    const int q = sms - static_cast<int>(tiles);
+    const double t = std::max(kbn * std::max(kb_time_us(GemmKind::kPromotion, bn), kFlagRoundTripUs),
+                              q_bytes / (q * kQuantCtaGBs * 1e3)) + 2.0;
+    if (t < lp.est_us - 1e-9) {
+      Plan g{bn, m_tiles, n_tiles, 1, kbn, static_cast<int>(tiles), sms};
+      g.est_us = t;
+      lp.fused = true;
+      lp.gemm = g;
+      lp.gemm_ctas = static_cast<int>(tiles);
+      lp.quant_ctas = q;
+      lp.est_us = t;
+    }
+  }
+  return lp;
+}
+
+// fp8_linear's choice: the fused launch when its estimate beats act_quant
+// followed by the GEMM's own plan.
+inline LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int sms) {
+  LinearPlan lp;
+  lp.gemm = plan_gemm(M, N, K, sms);
+  const double q_bytes = static_cast<double>(M) * K * 3.0 + 4.0 * M * (K / 128);
+  lp.est_us = (M > 128 ? lp.gemm.est_us : 0.0) + q_bytes / (kActQuantGBs * 1e3) + 2.0;
+  const LinearPlan f = plan_linear_fused(M, N, K, sms);
+  return (f.fused && f.est_us < lp.est_us - 1e-9) ? f : lp;
 }
 
 // Bytes of the K-block-major copies of the two scale tables that the

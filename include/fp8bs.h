@@ -421,21 +421,65 @@ FP8BS_API fp8bs_status fp8bs_fp8_linear_ue8m0(const uint16_t *x, int64_t M, int6
                                               size_t workspace_bytes, void *stream);
 
 /*
- * fp8_linear: the FP8 linear layer's forward pass, act_quant followed by
- * fp8_gemm on one stream ([ACT] notes that the linear wrapper calls act_quant
- * during the forward pass):
+ * fp8_linear: the FP8 linear layer's forward pass ([ACT] notes that the
+ * linear wrapper calls act_quant during the forward pass):
  *   (q, s) = act_quant(x, 128, fmt);  y = fp8_gemm(q, s, w, w_s)
  *
- *   x      device, [M, K] bf16
+ *   x      device, [M, K] bf16 (16-byte aligned)
  *   w, w_s as for fp8_gemm;  y  device, [M, N] bf16, written
  *   q      device, [M, K] uint8 and  s  device, [M, K / 128] fp32: caller-
  *          provided buffers that receive the quantized activations and scales
- *   workspace as for fp8_gemm (fp8bs_gemm_workspace_size(M, N, K) bytes).
+ *          (bit for bit what fp8bs_act_quant writes)
+ *   workspace  fp8bs_linear_workspace_size(M, N, K) bytes (16-byte aligned)
+ *
+ * Two forms, chosen per shape by their estimated times
+ * (fp8bs_linear_plan_string says which):
+ *  - act_quant followed by fp8_gemm, two launches on the stream (the
+ *    workspace then serves fp8_gemm, as fp8bs_gemm_workspace_size says);
+ *  - the single fused launch of fp8bs_fp8_linear_fused (below), taken only
+ *    where its estimate is lower.  With the costs measured on B200 it is
+ *    slower at every prefill shape measured, so the two launches are taken.
+ * q, s and y are the same in both forms (the GEMM's tile plan may differ, so
+ * y may differ in the last bits within the GEMM tolerance).
  */
 FP8BS_API fp8bs_status fp8bs_fp8_linear(const uint16_t *x, int64_t M, int64_t K, fp8bs_scale_fmt fmt,
                               const uint8_t *w, const float *w_s, int64_t N, uint16_t *y,
                               uint8_t *q, float *s, void *workspace, size_t workspace_bytes,
                               void *stream);
+
+/*
+ * fp8_linear_fused: the same layer as fp8bs_fp8_linear in ONE kernel launch
+ * (plus a memset of the workspace flags before it).  Where the GEMM's output
+ * tiles leave SMs idle (narrow N at M > 128, e.g. M = 4096, N = 576), those
+ * SMs quantize x while the others run the GEMM a few K blocks behind: every
+ * quantized 128-row chunk of a K block is counted into a flag in the
+ * workspace (release at GPU scope), and a GEMM CTA reads a chunk's codes and
+ * scales only after its flag (acquire).  Each chunk is quantized once, by the
+ * same arithmetic as act_quant, so q and s are bit-identical to
+ * fp8bs_act_quant's.  Useful where one launch matters more than time (a
+ * stream with a fixed kernel count); on B200 it measured slower than the two
+ * launches at the prefill shapes (the idle SMs quantize at ~35 GB/s each).
+ *
+ *   arguments as for fp8bs_fp8_linear; the workspace needs 4 bytes per
+ *   (128-row tile, K block), which fp8bs_linear_workspace_size covers.
+ * Errors: FP8BS_ERR_UNSUPPORTED when M <= 128 or the tiles leave fewer than
+ * 16 SMs free (no fused launch exists), FP8BS_ERR_WORKSPACE for a short
+ * workspace, and the checks of fp8bs_fp8_linear.
+ */
+FP8BS_API fp8bs_status fp8bs_fp8_linear_fused(const uint16_t *x, int64_t M, int64_t K,
+                                              fp8bs_scale_fmt fmt, const uint8_t *w,
+                                              const float *w_s, int64_t N, uint16_t *y,
+                                              uint8_t *q, float *s, void *workspace,
+                                              size_t workspace_bytes, void *stream);
+
+/* Workspace bytes fp8bs_fp8_linear and fp8bs_fp8_linear_fused need on the
+ * current device for an M x N x K layer (0 for invalid sizes). */
+FP8BS_API size_t fp8bs_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* Which form fp8bs_fp8_linear takes for an M x N x K layer on the current
+ * device, and its tile plan, as a NUL-terminated string in thread-local
+ * storage; for logs and benchmarks. */
+FP8BS_API const char *fp8bs_linear_plan_string(int64_t M, int64_t N, int64_t K);
 
 /*
  * fp8_gemm_grouped: G independent fp8_gemm problems (experts) that share N
