@@ -493,83 +493,80 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     if (C::kSplitRegs) reg_release<C::kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0;       // stages with a TMA load issued
-      uint32_t armed_phase = 0; // parity each armed stage completes
-      for (int u = unit_start; u < num_units; u += unit_step) {
-        const Unit t = unit_of(u);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
-          if (FUSED) {
-            // The chunk's codes are written by a quantizer CTA of this launch.
-            if (!wait_chunk_flag(p.fq_flags + (t.row0 / BM) * p.kbn + kb, abort_flag))
-              goto producer_done;
-            fence_proxy_async_global();
-          }
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.row0));
-          tma_load_2d(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.w_row0));
-          armed |= 1u << stage;
-          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+    // The whole warp walks the loop and takes the waits; one elected lane
+    // issues the loads.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0;       // stages with a TMA load issued
+    uint32_t armed_phase = 0; // parity each armed stage completes
+    for (int u = unit_start; u < num_units; u += unit_step) {
+      const Unit t = unit_of(u);
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+        if (FUSED) {
+          // The chunk's codes are written by a quantizer CTA of this launch.
+          if (!__all_sync(0xFFFFFFFFu,
+                          wait_chunk_flag(p.fq_flags + (t.row0 / BM) * p.kbn + kb, abort_flag)))
+            goto producer_done;
+          fence_proxy_async_global();
+        }
+        mbar_arrive_expect_tx_warp(&full[stage], C::kStageBytes);
+        tma_load_2d_warp(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
+                         static_cast<int32_t>(t.row0));
+        tma_load_2d_warp(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
+                         static_cast<int32_t>(t.w_row0));
+        armed |= 1u << stage;
+        armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-    producer_done:
-      if (*abort_flag) {
-        // Let every load in flight land before the CTA exits.
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
-      }
+    }
+  producer_done:
+    if (*abort_flag) {
+      // Let every load in flight land before the CTA exits.
+      for (int s = 0; s < C::kStages; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
     }
     __syncwarp();
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
-    // Two issuing threads: warp 1 takes the even and warp 3 the odd K blocks
+    // Two issuing warps: warp 1 takes the even and warp 3 the odd K blocks
     // of this CTA's sequence (i counts K blocks over all its units).  Each K
     // block writes a fresh partial into its own TMEM buffer and reads its own
-    // stage, so the two streams need no ordering between them.  One thread
-    // alone would spend about as long per K block on its barrier waits,
-    // commits and four instruction issues as the tensor core spends on the
-    // MMAs, and the tensor core would idle behind it.
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
-      const uint32_t parity = warp == 1 ? 0u : 1u;
-      uint32_t i = 0;
-      for (int u = unit_start; u < num_units; u += unit_step) {
-        const Unit t = unit_of(u);
-        for (int kb = t.kb0; kb < t.kb1; ++kb, ++i) {
-          if ((i & 1u) != parity) continue;
-          const int stage = static_cast<int>(i % C::kStages);
-          const uint32_t phase = (i / C::kStages) & 1u;
-          const int tb = static_cast<int>(i % C::kAccBufs);
-          const uint32_t tphase = (i / C::kAccBufs) & 1u;
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto mma_done;
-          if (!mbar_wait<kSpinWaits>(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
-          tc_fence_after();
-          const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
-          const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
+    // stage, so the two streams need no ordering between them.  Each warp
+    // walks its loop together and takes the waits; one elected lane issues.
+    constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+    const uint32_t parity = warp == 1 ? 0u : 1u;
+    uint32_t i = 0;
+    for (int u = unit_start; u < num_units; u += unit_step) {
+      const Unit t = unit_of(u);
+      for (int kb = t.kb0; kb < t.kb1; ++kb, ++i) {
+        if ((i & 1u) != parity) continue;
+        const int stage = static_cast<int>(i % C::kStages);
+        const uint32_t phase = (i / C::kStages) & 1u;
+        const int tb = static_cast<int>(i % C::kAccBufs);
+        const uint32_t tphase = (i / C::kAccBufs) & 1u;
+        if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto mma_done;
+        if (!mbar_wait_warp<kSpinWaits>(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
+        const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            mma_f8f6f4(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
-                       smem_desc_k_sw128(b_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
-          mma_commit(&tfull[tb]);
-          mma_commit(&empty[stage]);
-        }
+        for (int k = 0; k < BK / 32; ++k)
+          mma_f8f6f4_warp(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
+                          smem_desc_k_sw128(b_addr + 32 * k), idesc, k > 0 ? 1u : 0u);
+        mma_commit_warp(&tfull[tb]);
+        mma_commit_warp(&empty[stage]);
       }
-    mma_done:
-      // Every MMA this thread issued must finish before the TMEM columns are
-      // released.
-      mma_commit(&flush[parity]);
-      mbar_wait(&flush[parity], 0, nullptr);
     }
+  mma_done:
+    // Every MMA this warp issued must finish before the TMEM columns are
+    // released.
+    mma_commit_warp(&flush[parity]);
+    mbar_wait(&flush[parity], 0, nullptr);
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale producer

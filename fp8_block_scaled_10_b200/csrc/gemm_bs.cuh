@@ -12,20 +12,24 @@
 // accumulator therefore runs over the whole K range of a tile in TMEM, with
 // no per-K-block promotion: the epilogue reads TMEM once per tile.
 //
-// Scale factors in TMEM: for every 128 rows and one 128-wide K block, a
-// 512-byte atom whose byte 16*(r%32) + 4*(r/32) + j holds the exponent of row
-// r for the j-th 32-wide K sub-block (all four equal here: one scale per 128
-// K elements), copied from shared memory by tcgen05.cp 32x128b.warpx4 into
-// 4 TMEM columns.  The MMA for sub-block j selects byte j.
+// Scale factors in TMEM: for every 128 rows and a group of four consecutive
+// 128-wide K blocks 4g .. 4g + 3, a 512-byte atom whose byte
+// 16*(r%32) + 4*(r/32) + j holds the exponent of row r for K block 4g + j,
+// copied from shared memory by tcgen05.cp 32x128b.warpx4 into 4 TMEM
+// columns.  Each of the four MMAs (K = 32) of K block 4g + j selects byte j
+// of its scale cells (the scale factor id of the instruction descriptor):
+// one scale covers all 128 K elements of the block.  One copy per four K
+// blocks: measured on B200, three copies per K block (one per atom) kept the
+// tensor pipe busy 778 cycles per K block against 512 for the MMAs alone.
 //
 // Roles (persistent, one CTA per SM, 12 warps):
 //   warp 0      TMA producer of A [128 x 128] and W [BN x 128] tiles.
-//   warp 1      TMEM owner; one lane copies each stage's scale atoms into a
-//               TMEM ring and issues the block-scaled MMAs.
-//   warp 2      scale producer: reads a_s / w_s (prefetched four K blocks
-//               ahead), writes the exponent atoms into the stage's shared
-//               memory and checks that each scale is a positive normal power
-//               of two (else device error FP8BS_ERR_SCALE = 6).
+//   warp 1      TMEM owner; one lane copies each K-block group's scale
+//               atoms into a TMEM ring and issues the block-scaled MMAs.
+//   warp 2      scale producer: reads a_s / w_s for one K-block group at a
+//               time, writes the exponent atoms into a shared-memory ring
+//               of kSFSlots groups and checks that each scale is a positive
+//               normal power of two (else device error FP8BS_ERR_SCALE = 6).
 //   warps 4-11  epilogue: per tile, each thread reads one row of BN/2
 //               accumulator columns into registers as bf16, releases the
 //               accumulator, then stores (or writes FP32 split-K partials).
@@ -42,13 +46,15 @@ struct BsCfg {
   static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;   // TMA bytes per stage
   static constexpr int kSFAtoms = 1 + BN / 128;           // one for A, BN/128 for W
-  static constexpr int kSFBytes = 512 * kSFAtoms;
+  static constexpr int kSFBytes = 512 * kSFAtoms;         // one K-block group's atoms
+  static constexpr int kSFGroup = 4;                      // K blocks per scale atom
+  static constexpr int kSFSlots = 3;                      // groups in flight (smem and TMEM)
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kAccBufs = (BN == 256) ? 1 : 2;    // TMEM accumulators
-  static constexpr int kSFCols = 4 * kSFAtoms;            // TMEM columns per stage
+  static constexpr int kSFCols = 4 * kSFAtoms;            // TMEM columns per group slot
   static constexpr int kSFBase = kAccBufs * BN;
   static constexpr int kTmemCols = 512;
-  static_assert(kSFBase + kStages * kSFCols <= kTmemCols, "TMEM budget");
+  static_assert(kSFBase + kSFSlots * kSFCols <= kTmemCols, "TMEM budget");
   static constexpr int kEpiWarps = 8;
   static constexpr int kColsPerWarp = BN / 2;
   static constexpr int kFirstEpiWarp = 4;
@@ -56,7 +62,8 @@ struct BsCfg {
   static constexpr int kCtrlBytes = 256;
   static constexpr int kGroupBytes = 4 * kGroupTableInts;
   __host__ __device__ static constexpr int out_offset(bool grouped) {
-    return (kStages * (kStageBytes + kSFBytes) + kCtrlBytes + (grouped ? kGroupBytes : 0) + 1023) &
+    return (kStages * kStageBytes + kSFSlots * kSFBytes + kCtrlBytes +
+            (grouped ? kGroupBytes : 0) + 1023) &
            ~1023;
   }
   __host__ __device__ static constexpr int smem_bytes(bool grouped) {
@@ -66,8 +73,10 @@ struct BsCfg {
 
 template <int kStages>
 struct BsCtrl {
-  uint64_t full[kStages];    // TMA bytes + the scale producer's arrival
+  uint64_t full[kStages];    // TMA bytes
   uint64_t empty[kStages];
+  uint64_t sffull[3];        // scale-group slot written (the scale producer)
+  uint64_t sfempty[3];       // scale-group slot's MMAs complete (commit)
   uint64_t tfull[2];         // accumulator ready for the epilogue
   uint64_t tempty[2];        // accumulator drained
   uint64_t flush;
@@ -104,13 +113,16 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
   uint8_t* b_tiles = smem + C::kStages * C::kABytes;
   uint8_t* sf_tiles = smem + C::kStages * C::kStageBytes;
   BsCtrl<C::kStages>* ctrl =
-      reinterpret_cast<BsCtrl<C::kStages>*>(sf_tiles + C::kStages * C::kSFBytes);
+      reinterpret_cast<BsCtrl<C::kStages>*>(sf_tiles + C::kSFSlots * C::kSFBytes);
+  static_assert(C::kSFSlots <= 3, "scale-group barriers");
   static_assert(sizeof(BsCtrl<C::kStages>) <= C::kCtrlBytes, "control block too large");
   uint64_t* full = ctrl->full;
   uint64_t* empty = ctrl->empty;
   uint64_t* tfull = ctrl->tfull;
   uint64_t* tempty = ctrl->tempty;
   uint64_t* flush = &ctrl->flush;
+  uint64_t* sffull = ctrl->sffull;
+  uint64_t* sfempty = ctrl->sfempty;
   volatile int* abort_flag = &ctrl->abort_flag;
   int* tile_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ctrl) + C::kCtrlBytes);
   uint8_t* out_boxes = smem + C::out_offset(GROUPED);
@@ -123,8 +135,12 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 2);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int g = 0; g < C::kSFSlots; ++g) {
+      mbar_init(&sffull[g], 1);
+      mbar_init(&sfempty[g], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -171,192 +187,195 @@ __global__ void __launch_bounds__(BsCfg<BN>::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_phase = 0;
-      for (int u = unit_start; u < num_units; u += unit_step) {
-        const Unit t = unit_of(u);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.row0));
-          tma_load_2d(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
-                      static_cast<int32_t>(t.w_row0));
-          armed |= 1u << stage;
-          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-    producer_done:
-      if (*abort_flag) {
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale producer
-    // Walks the same (unit, K block) sequence as the TMA producer; a second
-    // cursor runs four steps ahead and loads the scales into a ring of
-    // registers, so the loads of step i+4 overlap the atoms of step i.
-    // W values per lane and step: one block scale per 128-row atom, or with
-    // BROW the lane's four rows of each atom.
-    constexpr int kWVals = BROW ? BN / 32 : BN / 128;
-    struct Cursor {
-      int u, kb, kb1, group, nb0, n0;
-      int64_t row0, row_end;
-      bool valid;
-    };
-    auto begin = [&](Cursor& c, int u) {
-      c.u = u;
-      c.valid = u < num_units;
-      if (c.valid) {
-        const Unit t = unit_of(u);
-        c.kb = t.kb0;
-        c.kb1 = t.kb1;
-        c.group = t.group;
-        c.nb0 = (t.n_tile * BN) / 128;
-        c.n0 = t.n_tile * BN;
-        c.row0 = t.row0;
-        c.row_end = t.row_end;
-      }
-    };
-    auto next = [&](Cursor& c) {
-      if (c.valid && ++c.kb >= c.kb1) begin(c, c.u + unit_step);
-    };
-    auto load = [&](const Cursor& c, float (&va)[4], float (&vw)[kWVals]) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t row = c.row0 + lane + 32 * j;
-        va[j] = (c.valid && row < c.row_end)
-                    ? __ldg(BROW ? p.sa + c.kb * p.M + row : p.sa + row * p.kbn + c.kb)
-                    : 1.0f;
-      }
-      if (BROW) {
-        // value 4a + j: row 128a + lane + 32j of the tile's W rows, from the
-        // K-block-major table sw [kbn][N] (coalesced across lanes)
-#pragma unroll
-        for (int i = 0; i < kWVals; ++i) {
-          const int64_t n = c.n0 + 128 * (i / 4) + lane + 32 * (i % 4);
-          vw[i] = (c.valid && n < p.N) ? __ldg(p.sw + c.kb * static_cast<int64_t>(p.N) + n) : 1.0f;
-        }
-      } else {
-#pragma unroll
-        for (int a = 0; a < BN / 128; ++a) {
-          const int nb = c.nb0 + a;
-          vw[a] = (c.valid && nb < p.nbn)
-                      ? __ldg(p.sw + (static_cast<int64_t>(c.group) * p.nbn + nb) * p.kbn + c.kb)
-                      : 1.0f;
-        }
-      }
-    };
-    float ra[4][4], rw[4][kWVals];
-    Cursor ahead, cur;
-    begin(ahead, unit_start);
-    begin(cur, unit_start);
-#pragma unroll
-    for (int d = 0; d < 4; ++d) {
-      load(ahead, ra[d], rw[d]);
-      next(ahead);
-    }
+    // The whole warp walks the loop; one elected lane issues.
     int stage = 0;
     uint32_t phase = 0;
-    bool bad = false;
-    while (cur.valid) {
-#pragma unroll
-      for (int ph = 0; ph < 4; ++ph) {
-        if (!cur.valid) break;
-        const bool ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
-        if (!__all_sync(0xFFFFFFFFu, ok)) goto scales_done;
-        uint8_t* atoms = sf_tiles + stage * C::kSFBytes;
-        uint4 v;
-        v.x = ue8m0_byte(ra[ph][0], &bad) * 0x01010101u;
-        v.y = ue8m0_byte(ra[ph][1], &bad) * 0x01010101u;
-        v.z = ue8m0_byte(ra[ph][2], &bad) * 0x01010101u;
-        v.w = ue8m0_byte(ra[ph][3], &bad) * 0x01010101u;
-        *reinterpret_cast<uint4*>(atoms + 16 * lane) = v;
-#pragma unroll
-        for (int a = 0; a < BN / 128; ++a) {
-          if (BROW) {
-            uint4 w;
-            w.x = ue8m0_byte(rw[ph][4 * a + 0], &bad) * 0x01010101u;
-            w.y = ue8m0_byte(rw[ph][4 * a + 1], &bad) * 0x01010101u;
-            w.z = ue8m0_byte(rw[ph][4 * a + 2], &bad) * 0x01010101u;
-            w.w = ue8m0_byte(rw[ph][4 * a + 3], &bad) * 0x01010101u;
-            *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = w;
-          } else {
-            const uint32_t e = ue8m0_byte(rw[ph][a], &bad) * 0x01010101u;
-            *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = make_uint4(e, e, e, e);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        load(ahead, ra[ph], rw[ph]);
-        next(ahead);
-        next(cur);
+    uint32_t armed = 0, armed_phase = 0;
+    for (int u = unit_start; u < num_units; u += unit_step) {
+      const Unit t = unit_of(u);
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+        mbar_arrive_expect_tx_warp(&full[stage], C::kStageBytes);
+        tma_load_2d_warp(a_tiles + stage * C::kABytes, &tmap_a, &full[stage], kb * BK,
+                         static_cast<int32_t>(t.row0));
+        tma_load_2d_warp(b_tiles + stage * C::kBBytes, &tmap_w, &full[stage], kb * BK,
+                         static_cast<int32_t>(t.w_row0));
+        armed |= 1u << stage;
+        armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
+  producer_done:
+    if (*abort_flag) {
+      for (int s = 0; s < C::kStages; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale producer
+    // Walks this CTA's (unit, K-block group) sequence.  Group q covers the K
+    // blocks 4q .. 4q + 3 (those outside the unit or past K are never used by
+    // an MMA; they get exponent 127, a scale of 1).  For every group it loads
+    // the scales first, all at once from clamped (always valid) indices so
+    // that their latencies overlap, then waits until the MMAs that read the
+    // slot's previous group have completed and writes the atoms: row r of A
+    // (lane + 32 j) and of W (its block's scale, or with BROW its own row
+    // scale), one exponent byte per K block.  A fence makes them visible to
+    // the tensor core's copy before the arrival on sffull.
+    constexpr int kG = C::kSFGroup;
+    constexpr int kWA = BN / 128;   // W atoms
+    bool bad = false;
+    uint32_t gi = 0;
+    for (int u = unit_start; u < num_units; u += unit_step) {
+      const Unit t = unit_of(u);
+      const int nb0 = (t.n_tile * BN) / 128;
+      const int64_t n0 = t.w_row0 - static_cast<int64_t>(t.group) * p.N;   // first W row (column of y)
+      for (int q = t.kb0 / kG; q <= (t.kb1 - 1) / kG; ++q, ++gi) {
+        const int slot = static_cast<int>(gi % C::kSFSlots);
+        int kbc[kG];
+        bool kin[kG];
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          const int kb = q * kG + j;
+          kin[j] = kb >= t.kb0 && kb < t.kb1;
+          kbc[j] = kb < t.kb0 ? t.kb0 : (kb >= t.kb1 ? t.kb1 - 1 : kb);
+        }
+        float va[4][kG];
+        bool rin[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int64_t row = t.row0 + lane + 32 * r;
+          rin[r] = row < t.row_end;
+          const int64_t rc = rin[r] ? row : t.row_end - 1;
+#pragma unroll
+          for (int j = 0; j < kG; ++j)
+            va[r][j] = __ldg(BROW ? p.sa + static_cast<int64_t>(kbc[j]) * p.M + rc
+                                  : p.sa + rc * p.kbn + kbc[j]);
+        }
+        constexpr int kWR = BROW ? 4 : 1;   // W rows per lane and atom
+        float vw[kWA][kWR][kG];
+        bool win[kWA][kWR];
+#pragma unroll
+        for (int a = 0; a < kWA; ++a) {
+#pragma unroll
+          for (int r = 0; r < kWR; ++r) {
+            const float* src;
+            if (BROW) {
+              const int64_t n = n0 + 128 * a + lane + 32 * r;
+              win[a][r] = n < p.N;
+              src = p.sw + (win[a][r] ? n : p.N - 1);
+            } else {
+              const int nb = nb0 + a;
+              win[a][r] = nb < p.nbn;
+              src = p.sw + (static_cast<int64_t>(t.group) * p.nbn + (win[a][r] ? nb : p.nbn - 1)) * p.kbn;
+            }
+#pragma unroll
+            for (int j = 0; j < kG; ++j)
+              vw[a][r][j] = __ldg(src + static_cast<int64_t>(kbc[j]) * (BROW ? p.N : 1));
+          }
+        }
+        const bool ok = mbar_wait(&sfempty[slot], ((gi / C::kSFSlots) & 1u) ^ 1u, abort_flag);
+        if (!__all_sync(0xFFFFFFFFu, ok)) goto scales_done;
+        // Exponent word of one row: byte j = K block q * kG + j.
+        auto word = [&](const float (&v)[kG], bool row_in) -> uint32_t {
+          uint32_t w = 0;
+#pragma unroll
+          for (int j = 0; j < kG; ++j) {
+            const uint32_t e = ue8m0_byte(v[j], &bad);
+            w |= (row_in && kin[j] ? e : 127u) << (8 * j);
+          }
+          return w;
+        };
+        uint8_t* atoms = sf_tiles + slot * C::kSFBytes;
+        *reinterpret_cast<uint4*>(atoms + 16 * lane) =
+            make_uint4(word(va[0], rin[0]), word(va[1], rin[1]), word(va[2], rin[2]),
+                       word(va[3], rin[3]));
+#pragma unroll
+        for (int a = 0; a < kWA; ++a) {
+          uint4 w4;
+          if (BROW) {
+            w4 = make_uint4(word(vw[a][0], win[a][0]), word(vw[a][kWR > 1 ? 1 : 0], win[a][kWR > 1 ? 1 : 0]),
+                            word(vw[a][kWR > 2 ? 2 : 0], win[a][kWR > 2 ? 2 : 0]),
+                            word(vw[a][kWR > 3 ? 3 : 0], win[a][kWR > 3 ? 3 : 0]));
+          } else {
+            const uint32_t w = word(vw[a][0], win[a][0]);
+            w4 = make_uint4(w, w, w, w);
+          }
+          *reinterpret_cast<uint4*>(atoms + 512 * (1 + a) + 16 * lane) = w4;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sffull[slot]);
+      }
+    }
   scales_done:
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report_error(6);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_block_scaled(BM, BN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int tb = 0;
-      uint32_t tphase = 0;
-      for (int u = unit_start; u < num_units; u += unit_step) {
-        const Unit t = unit_of(u);
-        // The epilogue has drained this accumulator (tile u - 2 * step).
-        if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto mma_done;
+    // The whole warp walks the loop and takes the waits; one elected lane
+    // issues the copies, MMAs and commits.
+    constexpr uint32_t idesc = idesc_e4m3_block_scaled(BM, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int tb = 0;
+    uint32_t tphase = 0;
+    uint32_t gi = 0;   // K-block groups started
+    uint32_t tsf = 0;  // TMEM scale slot of the current group
+    for (int u = unit_start; u < num_units; u += unit_step) {
+      const Unit t = unit_of(u);
+      // The epilogue has drained this accumulator (tile u - 2 * step).
+      if (!mbar_wait_warp(&tempty[tb], tphase ^ 1u, abort_flag)) goto mma_done;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * BN);
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const int slot = static_cast<int>(gi % C::kSFSlots);
+        if (kb == t.kb0 || kb % C::kSFGroup == 0) {
+          // A new K-block group: its scale atoms into the slot's TMEM
+          // columns (A, then W), once for the group's K blocks.
+          if (!mbar_wait_warp(&sffull[slot], (gi / C::kSFSlots) & 1u, abort_flag)) goto mma_done;
           tc_fence_after();
-          // Scale atoms of this stage into its TMEM slot (A, then W).
-          const uint32_t tsf = tmem_base + static_cast<uint32_t>(C::kSFBase + stage * C::kSFCols);
-          const uint8_t* atoms = sf_tiles + stage * C::kSFBytes;
+          tsf = tmem_base + static_cast<uint32_t>(C::kSFBase + slot * C::kSFCols);
+          const uint8_t* atoms = sf_tiles + slot * C::kSFBytes;
 #pragma unroll
           for (int a = 0; a < C::kSFAtoms; ++a)
-            tmem_copy_32x128b_x4(tsf + 4 * a, smem_desc_rows16(smem_addr(atoms + 512 * a)));
-          const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
-          const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
-#pragma unroll
-          for (int k = 0; k < BK / 32; ++k) {
-            const uint32_t sub = static_cast<uint32_t>(k);
-            mma_mxf8_block_scaled(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
-                                  smem_desc_k_sw128(b_addr + 32 * k),
-                                  idesc | (sub << 29) | (sub << 4), tsf | (sub << 30),
-                                  (tsf + 4) | (sub << 30), (kb > t.kb0 || k > 0) ? 1u : 0u);
-          }
-          mma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+            tmem_copy_32x128b_x4_warp(tsf + 4 * a, smem_desc_rows16(smem_addr(atoms + 512 * a)));
         }
-        mma_commit(&tfull[tb]);
-        if (++tb == C::kAccBufs) {
-          tb = 0;
-          tphase ^= 1u;
+        if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto mma_done;
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(a_tiles + stage * C::kABytes);
+        const uint32_t b_addr = smem_addr(b_tiles + stage * C::kBBytes);
+        // Byte kb % 4 of every scale cell is this K block's exponent, for
+        // all four K = 32 slices of the block.
+        const uint32_t sub = static_cast<uint32_t>(kb % C::kSFGroup);
+#pragma unroll
+        for (int k = 0; k < BK / 32; ++k)
+          mma_mxf8_block_scaled_warp(d_tmem, smem_desc_k_sw128(a_addr + 32 * k),
+                                     smem_desc_k_sw128(b_addr + 32 * k),
+                                     idesc | (sub << 29) | (sub << 4), tsf | (sub << 30),
+                                     (tsf + 4) | (sub << 30), (kb > t.kb0 || k > 0) ? 1u : 0u);
+        mma_commit_warp(&empty[stage]);
+        if (kb + 1 == t.kb1 || kb % C::kSFGroup == C::kSFGroup - 1) {
+          // The group's last MMAs: its slot is free once they complete.
+          mma_commit_warp(&sfempty[slot]);
+          ++gi;
+        }
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-    mma_done:
-      mma_commit(flush);
-      mbar_wait(flush, 0, nullptr);
+      mma_commit_warp(&tfull[tb]);
+      if (++tb == C::kAccBufs) {
+        tb = 0;
+        tphase ^= 1u;
+      }
     }
+  mma_done:
+    mma_commit_warp(flush);
+    mbar_wait(flush, 0, nullptr);
     __syncwarp();
   } else if (warp >= C::kFirstEpiWarp) {
     // ------------------------------------------------------------ epilogue

@@ -291,6 +291,84 @@ __device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sd
                : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Whole-warp issue forms.  The calling warp runs its pipeline loop together
+// (uniform control flow, every lane taking the barrier waits) and elect.sync
+// picks one lane to issue.  With all 32 lanes present that is always the same
+// lane, so its commits track its own MMAs and copies.  Measured on B200 (one
+// CTA per SM; four block-scaled MMAs of N = 128 and a commit per K block,
+// 256 cycles of tensor work): 272 cycles per K block issued this way against
+// 322 from one lane behind `if (lane == 0)`, and an mbarrier wait on a
+// completed phase inside the loop cost 45 cycles against 213.
+
+__device__ __forceinline__ void mma_f8f6f4_warp(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf8_block_scaled_warp(uint32_t tmem_d, uint64_t adesc,
+                                                           uint64_t bdesc, uint32_t idesc,
+                                                           uint32_t sfa, uint32_t sfb,
+                                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_copy_32x128b_x4_warp(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(sdesc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_warp(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_warp(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n\t}" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// mbar_wait taken by every lane of a warp, with one answer for all of them.
+template <bool kSpin = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait<kSpin>(bar, parity, abort));
+}
+
 // Shared-memory descriptor of a contiguous block of 16-byte rows (no
 // swizzle): 8-row core matrices 128 bytes apart.
 __device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t addr) {

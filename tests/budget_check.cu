@@ -47,7 +47,7 @@ constexpr bool block_scaled_ok() {
   static_assert(C::smem_bytes(G) <= kMaxSmem, "shared memory");
   static_assert(sizeof(BsCtrl<C::kStages>) <= C::kCtrlBytes, "control block");
   static_assert(C::kAccBufs <= 2, "accumulator barriers");
-  static_assert(C::kSFBase + C::kStages * C::kSFCols <= C::kTmemCols, "TMEM columns");
+  static_assert(C::kSFBase + C::kSFSlots * C::kSFCols <= C::kTmemCols, "TMEM columns");
   static_assert(C::kABytes % 1024 == 0 && C::kBBytes % 1024 == 0 && C::kSFBytes % 128 == 0,
                 "slot alignment");
   return true;
