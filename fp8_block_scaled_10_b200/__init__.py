@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "act_quant", "act_quant_static", "act_dequant", "static_dequant",
-    "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear",
+    "weight_dequant", "weight_quant", "fp8_gemm", "fp8_linear", "fp8_linear_fused",
     "fp8_gemm_grouped", "fp8_gemm_quant", "fp8_gemm_rowwise", "act_quant_transposed",
     "fp8_transpose", "gemm_workspace_size", "gemm_plan", "linear_plan", "device_error", "lib",
     "Fp8bsError",
@@ -470,6 +470,37 @@ def fp8_linear(x, weight, weight_scale, scale_fmt=None, return_quant=False,
         _check(lib().fp8bs_fp8_linear(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
                                       _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s), _ptr(ws),
                                       nws, _stream(x.device)))
+    return (y, q, s) if return_quant else y
+
+
+def fp8_linear_fused(x, weight, weight_scale, scale_fmt=None, return_quant=False):
+    """The FP8 linear forward as one launch: the SMs the GEMM's tiles leave
+    idle quantize x (act_quant, bit-identical q and s) while the GEMM
+    consumes it.  Raises (FP8BS_ERR_UNSUPPORTED) where no such launch exists:
+    decode-sized M, or tiles that fill the GPU.  fp8_linear picks this form
+    itself when the planner expects it to be faster (linear_plan names the
+    choice).  x: [..., K] bfloat16, weight: [N, K] e4m3fn, weight_scale:
+    [cdiv(N,128), K/128]; scale_fmt sets the activation scales' format."""
+    w = _codes(weight)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if w.dim() != 2 or w.shape[1] != x.shape[-1]:
+        raise ValueError("weight must be [N, K] with K = x.shape[-1]")
+    K = x.shape[-1]
+    if K <= 0 or K % 128 != 0:
+        raise ValueError("K=%d must be a positive multiple of 128" % K)
+    N = w.shape[0]
+    _scales_like(weight_scale, (_cdiv(N, 128), K // 128), "weight_scale")
+    _need_cuda(x, w, weight_scale)
+    M = x.numel() // K
+    y = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
+    q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty(*x.shape[:-1], K // 128, dtype=torch.float32, device=x.device)
+    nws = int(lib().fp8bs_linear_workspace_size(M, N, K))
+    ws = torch.empty(nws, dtype=torch.uint8, device=x.device) if nws else None
+    _check(lib().fp8bs_fp8_linear_fused(_ptr(x), M, K, _scale_fmt(scale_fmt), _ptr(w),
+                                        _ptr(weight_scale), N, _ptr(y), _ptr(q), _ptr(s),
+                                        _ptr(ws), nws, _stream(x.device)))
     return (y, q, s) if return_quant else y
 
 

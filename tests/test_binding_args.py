@@ -88,6 +88,17 @@ def test_fp8_linear_shapes():
         fp8bs.fp8_linear(x.float(), _e4m3(300, 256), _f32(3, 2))
 
 
+def test_fp8_linear_fused_shapes():
+    x = torch.zeros(3, 5, 256, dtype=torch.bfloat16)
+    _cuda_only(fp8bs.fp8_linear_fused, x, _e4m3(300, 256), _f32(3, 2))
+    with pytest.raises(ValueError, match="weight_scale must have shape"):
+        fp8bs.fp8_linear_fused(x, _e4m3(300, 256), _f32(2, 2))
+    with pytest.raises(ValueError, match="weight must be"):
+        fp8bs.fp8_linear_fused(x, _e4m3(300, 384), _f32(3, 3))
+    with pytest.raises(TypeError, match="bfloat16"):
+        fp8bs.fp8_linear_fused(x.float(), _e4m3(300, 256), _f32(3, 2))
+
+
 def test_fp8_gemm_grouped_shapes():
     G, N, K, M = 4, 384, 256, 100
     offs = torch.tensor([0, 10, 10, 60, 100], dtype=torch.int64)

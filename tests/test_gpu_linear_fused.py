@@ -145,3 +145,22 @@ def test_fused_linear_refuses_what_it_cannot_run():
     st = L.fp8bs_fp8_linear_fused(_vp(d), 1000, 2048, 0, _vp(d), _vp(d), 576, _vp(d), _vp(d),
                                   _vp(d), _vp(ws), 64, stream)
     assert st == fp8bs.ERR_WORKSPACE
+
+
+def test_python_binding_matches_two_launch_form():
+    """fp8bs.fp8_linear_fused (the binding) against fp8bs.fp8_linear on the
+    same inputs: identical q and s; y within tolerance of the oracle."""
+    M, N, K = 1000, 576, 2048
+    x = wl.normal_with_outliers(M, K, seed=81, frac=0.01, factor=50.0).cuda()
+    qw, sw = quantized_weight(N, K, seed=82)
+    w_d, sw_d = cuda_codes(qw), cuda_f32(sw)
+    y1, q1, s1 = fp8bs.fp8_linear_fused(x, w_d, sw_d, return_quant=True)
+    y2, q2, s2 = fp8bs.fp8_linear(x, w_d, sw_d, return_quant=True)
+    assert torch.equal(q1.view(torch.uint8), q2.view(torch.uint8))
+    assert torch.equal(s1.view(torch.int32), s2.view(torch.int32))
+    qa, sa = oracle.act_quant(wl.bf16_bits(x.cpu()))
+    y_ref, bnd = oracle.gemm(qa, sa, qw, sw)
+    assert_gemm_close(y1, y_ref, bnd, "fp8_linear_fused binding")
+    with pytest.raises(fp8bs.Fp8bsError):
+        fp8bs.fp8_linear_fused(x[:64], w_d, sw_d)     # decode-sized M: no fused launch
+    assert fp8bs.device_error() == 0
