@@ -747,10 +747,29 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
       float2 acc[CPW / 2];
 #pragma unroll
       for (int j = 0; j < CPW / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      // A warp whose 32 rows all lie past the unit's end (decode-sized M, an
+      // expert's last m tile) loads and accumulates nothing; it only takes
+      // the waits and releases.  Dense prefill tiles compile without the
+      // test: measured on B200, its branch cost the 256-wide dense kernel
+      // 2-5 %, while it made decode 4-7 % and the grouped GEMM 6 % faster.
+      const bool live = (ARows == 128 && !GROUPED) || t.row0 + quad * 32 < t.row_end;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         const bool ok = mbar_wait<kSpinWaits>(&tfull[tb], tphase, abort_flag);
         if (!__all_sync(0xFFFFFFFFu, ok)) goto epilogue_done;
         tc_fence_after();
+        if (!live) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&tempty[tb]);
+            if (BROW) mbar_arrive(&sempty[tb]);
+          }
+          if (++tb == C::kAccBufs) {
+            tb = 0;
+            tphase ^= 1u;
+          }
+          continue;
+        }
         // This K block's scale products a_s[row, kb] * w_s[nb, kb], read before
         // the buffer (and with it the scale slot) is released below.
         const float* src = scale_slots + tb * (C::kScaleSlotBytes / 4);
