@@ -203,15 +203,16 @@ struct Cfg {
   // TMEM partial buffers: as many as the 512 columns hold (2 of 256 columns,
   // 4 of 128), so the epilogue can lag the tensor core by kAccBufs - 1 K blocks.
   static constexpr int kAccBufs = 512 / BN;
-  // 128 x 256 tiles: warp 1 alone issues the MMAs (about 400 cycles of
-  // issue per K block against 512 of MMA work) and warps 2 and 3 both
+  // 128-row A stages with 256- or 128-wide tiles: warp 1 alone issues the
+  // MMAs (about 400 cycles of issue per K block) and warps 2 and 3 both
   // produce scales, alternate K blocks each.  A producer's step is bound by
-  // its load latency; two of them keep the scales ahead of the MMAs
-  // (measured on B200: 6-12 % faster prefill, 9 % faster grouped GEMM).
-  // Narrower tiles, and the decode stages (whose weight stream sets the
-  // pace; one issuer measured 3 % slower there), keep two MMA warps
-  // (warps 1 and 3) and one scale warp.
-  static constexpr int kScaleWarps = (BN == 256 && ARows == 128) ? 2 : 1;
+  // its load latency (~700-850 cycles); two of them keep the scales ahead
+  // (measured on B200: 6-14 % faster at 128 x 256, 3-10 % at 128 x 128,
+  // 9 % faster grouped GEMM).  192-wide tiles (384 cycles of MMA per K
+  // block) and the decode stages (whose weight stream sets the pace; one
+  // issuer measured 3 % slower there) keep two MMA warps (warps 1 and 3)
+  // and one scale warp.
+  static constexpr int kScaleWarps = (BN != 192 && ARows == 128) ? 2 : 1;
   static constexpr int kTmemCols = 512;
   static constexpr int kCtrlBytes = 512;
   // Scale ring: per K block the tile's 128 activation scales and its
