@@ -15,18 +15,22 @@
 // it into register accumulators with one FMA per element by
 // a_s[m, kb] * w_s[nb, kb], while the tensor core fills the other buffer.
 //
-// Roles (persistent CTAs, one per SM, walking work units in a fixed order):
-//   warp 0     TMA producer: A tile [128 x 128] and W tile into a ring of
+// Roles (persistent CTAs, one per SM, walking work units in a fixed order;
+// every control warp runs its loop with all 32 lanes and issues through
+// elect.sync):
+//   warp 0     TMA producer: A tile [ARows x 128] and W tile into a ring of
 //              shared-memory stages (128B swizzle).
-//   warps 1, 3 one lane each issues the MMAs of alternate K blocks; warp 1
-//              owns the TMEM allocation.
-//   warp 2     scale producer: for every K block of every unit it loads the
-//              128 activation scales a_s[rows, kb] and the weight scales
-//              w_s[nb, kb] of the tile (four K blocks ahead, in registers)
-//              into a small shared-memory ring that the epilogue reads.  The
-//              epilogue threads would otherwise each wait on a scattered
-//              global load per K block, which measured slower than the drain
-//              of the TMEM partial itself.
+//   warp 1     MMA issuer and owner of the TMEM allocation.  With 192-wide
+//              tiles and decode-sized A stages warp 3 issues too, the two
+//              taking alternate K blocks.
+//   warp 2     scale producer (and warp 3, on alternate K blocks, with
+//              128-row A stages and 128- or 256-wide tiles): for its K
+//              blocks it loads the 128 activation scales a_s[rows, kb] and
+//              the weight scales w_s[nb, kb] of the tile (four of its steps
+//              ahead, in registers) into a small shared-memory ring that the
+//              epilogue reads.  The epilogue threads would otherwise each
+//              wait on a scattered global load per K block, which measured
+//              slower than the drain of the TMEM partial itself.
 //   epilogue   8 warps from kFirstEpiWarp: warp w reads TMEM lanes
 //              32*(w%4)..+31 (one output row per thread) and BN/2 columns
 //              (column half (w - kFirstEpiWarp) / 4).  Loads of the next
@@ -580,10 +584,13 @@ __global__ void __launch_bounds__(Cfg<BN, ARows>::kThreads, 1)
     __syncwarp();
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ scale producer(s)
-    // Walks the same (unit, K block) sequence as the epilogue.  A second
-    // cursor runs kAhead steps ahead and loads the scales into a ring of
-    // registers, so the global loads of step i + kAhead overlap the shared-
-    // memory writes of step i.  Step i uses the slot of its TMEM buffer,
+    // Walks the same (unit, K block) sequence as the epilogue (with two
+    // scale warps, each its alternate steps).  A second cursor runs kAhead
+    // of its steps ahead and loads the scales into a ring of registers.
+    // (The warp barrier and the release before each arrival wait for the
+    // lane's loads in flight, so a warp's step costs about one load latency,
+    // ~700-850 cycles measured on B200; hence two warps where a K block's
+    // MMAs take less.)  Step i uses the slot of its TMEM buffer,
     // i % kAccBufs, once the epilogue has released that buffer (tempty), and
     // then arrives on its tfull: a_s of the tile's 128 rows (0 past the last
     // row) and w_s of the weight blocks the tile touches (0 past the last),

@@ -22,10 +22,11 @@
 // blocks: measured on B200, three copies per K block (one per atom) kept the
 // tensor pipe busy 778 cycles per K block against 512 for the MMAs alone.
 //
-// Roles (persistent, one CTA per SM, 12 warps):
+// Roles (persistent, one CTA per SM, 12 warps; the TMA and MMA warps run
+// their loops with all 32 lanes and issue through elect.sync):
 //   warp 0      TMA producer of A [128 x 128] and W [BN x 128] tiles.
-//   warp 1      TMEM owner; one lane copies each K-block group's scale
-//               atoms into a TMEM ring and issues the block-scaled MMAs.
+//   warp 1      TMEM owner; copies each K-block group's scale atoms into a
+//               TMEM ring and issues the block-scaled MMAs.
 //   warp 2      scale producer: reads a_s / w_s for one K-block group at a
 //               time, writes the exponent atoms into a shared-memory ring
 //               of kSFSlots groups and checks that each scale is a positive

@@ -198,27 +198,6 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major e4m3, fp32 accumulator.
-// accumulate == 0 overwrites D.
-__device__ __forceinline__ void mma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrives once on *bar when all tcgen05 operations this thread issued so far
-// have completed.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_addr(bar))
-      : "memory");
-}
-
 // Each lane of the warp reads 32 consecutive fp32 columns of its own TMEM lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -267,31 +246,6 @@ __device__ __forceinline__ void reg_acquire() {
 }
 
 // ---------------------------------------------------------------------------
-// Block-scaled MMA (kind::mxf8f6f4.block_scale): e4m3 operands with one ue8m0
-// scale factor per 32 K elements for every row of A and of B, read from TMEM.
-// ---------------------------------------------------------------------------
-// D (+)= (SFA x A) * (SFB x B)^T; sfa/sfb are TMEM addresses whose top two
-// bits select the scale byte (the 32-K sub-block) within each 32-bit cell.
-__device__ __forceinline__ void mma_mxf8_block_scaled(uint32_t tmem_d, uint64_t adesc,
-                                                      uint64_t bdesc, uint32_t idesc,
-                                                      uint32_t sfa, uint32_t sfb,
-                                                      uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
-}
-
-// Copies a 32-row x 16-byte block from shared memory into TMEM lanes 0-31 and
-// replicates it into the other three 32-lane quadrants.
-__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
-// ---------------------------------------------------------------------------
 // Whole-warp issue forms.  The calling warp runs its pipeline loop together
 // (uniform control flow, every lane taking the barrier waits) and elect.sync
 // picks one lane to issue.  With all 32 lanes present that is always the same
@@ -301,6 +255,8 @@ __device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sd
 // 322 from one lane behind `if (lane == 0)`, and an mbarrier wait on a
 // completed phase inside the loop cost 45 cycles against 213.
 
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major e4m3, fp32 accumulator;
+// accumulate == 0 overwrites D.
 __device__ __forceinline__ void mma_f8f6f4_warp(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -312,6 +268,11 @@ __device__ __forceinline__ void mma_f8f6f4_warp(uint32_t tmem_d, uint64_t adesc,
       : "memory");
 }
 
+// Block-scaled MMA (kind::mxf8f6f4.block_scale): D (+)= (SFA x A) *
+// (SFB x B)^T for e4m3 operands with one ue8m0 scale factor per 32 K
+// elements for every row of A and of B, read from TMEM; sfa / sfb are TMEM
+// addresses whose top two bits select the scale byte within each 32-bit cell
+// (the instruction descriptor carries the same selection).
 __device__ __forceinline__ void mma_mxf8_block_scaled_warp(uint32_t tmem_d, uint64_t adesc,
                                                            uint64_t bdesc, uint32_t idesc,
                                                            uint32_t sfa, uint32_t sfb,
@@ -325,6 +286,8 @@ __device__ __forceinline__ void mma_mxf8_block_scaled_warp(uint32_t tmem_d, uint
       : "memory");
 }
 
+// Arrives once on *bar when all tcgen05 operations the issuing lane started
+// so far have completed.
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -334,6 +297,8 @@ __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
       : "memory");
 }
 
+// Copies a 32-row x 16-byte block from shared memory into TMEM lanes 0-31 and
+// replicates it into the other three 32-lane quadrants.
 __device__ __forceinline__ void tmem_copy_32x128b_x4_warp(uint32_t taddr, uint64_t sdesc) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
